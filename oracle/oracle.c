@@ -1,0 +1,234 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU reference for causal linear attention
+ * ("Lightning Attention").
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the CUDA library and
+ * its Python binding) may include, link, load or call this file.  Only the
+ * tests, the smoke check and the benchmark's CPU-baseline leg use it.  It shares
+ * no code, header, table or helper with the CUDA kernels.
+ *
+ * What is computed (all forms are the same mathematical object):
+ *
+ *     o_t = sum_{s <= t} (q_t . k_s) v_s            (causal, diagonal included,
+ *                                                    no softmax, no scale,
+ *                                                    no normaliser)
+ *     S_t = sum_{s <= t} k_s^T v_s                   (d x d running state,
+ *                                                    row = key dim, col = value dim)
+ *     o_t = q_t S_t
+ *
+ * Sources (web pages about the MiniMax-01 report):
+ *  - "MiniMax-01技術報告解讀以及與DeepSeek-V3對比" (m.futurefh.com), section 1
+ *    ("core innovation: linear attention"): lightning attention splits the
+ *    attention computation into an intra-block part computed with the left
+ *    product and an inter-block part computed with the right product, which
+ *    avoids the slow cumulative sum.
+ *  - "MiniMax M2.1 (the 'linear' revolution)" (nabfollower.com), section
+ *    "The Core Tech: Lightning Attention": by associativity of matrix products
+ *    (Q K^T) V is regrouped as Q (K^T V), bringing the cost from O(N^2 d) to
+ *    O(N d^2); the closing analogy of the same page: linear attention keeps a
+ *    fixed-size summary (hidden state) while it scans the sequence.
+ *  - Section 3 of the first page ("efficient inference framework"): prefill and
+ *    decode are executed separately.  Section 4 ("long-context training"):
+ *    sequences are packed (data packing), which the varlen form models.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ * no decay, no feature map, no 1/sqrt(d) scale, no normalising denominator;
+ * the diagonal s == t is included; the state used for block i excludes block
+ * i; a decode step updates the state with the new token before reading it.
+ *
+ * Layouts: q, k, v, o are [BH][N][d] row-major (BH = batch*heads flattened);
+ * states are [BH][d][d] row-major with row index = key dim.  Varlen inputs are
+ * packed [H][T][d]; cu_seqlens has num_seqs+1 entries; states are
+ * [num_seqs][H][d][d].
+ */
+#include <stddef.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Quadratic masked form, straight from the definition (the "left product"
+ * (Q K^T ⊙ M) V of section 1 of the futurefh page, applied to the whole
+ * sequence with M lower-triangular including the diagonal).  O(N^2 d).
+ */
+void oracle_prefill_quadratic(const double* q, const double* k, const double* v,
+                              double* o, long BH, long N, long d) {
+    long bh;
+#pragma omp parallel for schedule(dynamic)
+    for (bh = 0; bh < BH; ++bh) {
+        const double* Q = q + bh * N * d;
+        const double* K = k + bh * N * d;
+        const double* V = v + bh * N * d;
+        double* O = o + bh * N * d;
+        for (long t = 0; t < N; ++t) {
+            for (long j = 0; j < d; ++j) O[t * d + j] = 0.0;
+            for (long s = 0; s <= t; ++s) {
+                double score = 0.0;
+                for (long c = 0; c < d; ++c) score += Q[t * d + c] * K[s * d + c];
+                for (long j = 0; j < d; ++j) O[t * d + j] += score * V[s * d + j];
+            }
+        }
+    }
+}
+
+/*
+ * Recurrent (scan) form: the fixed-size state of the nabfollower page's
+ * analogy.  For t = 0..N-1:  S <- S + k_t^T v_t ;  o_t = q_t S.
+ * state_in may be NULL (S starts at zero); state_out may be NULL.  O(N d^2).
+ */
+void oracle_prefill_recurrent(const double* q, const double* k, const double* v,
+                              const double* state_in, double* o, double* state_out,
+                              long BH, long N, long d) {
+    long bh;
+#pragma omp parallel for schedule(dynamic)
+    for (bh = 0; bh < BH; ++bh) {
+        const double* Q = q + bh * N * d;
+        const double* K = k + bh * N * d;
+        const double* V = v + bh * N * d;
+        double* O = o + bh * N * d;
+        double* S = (double*)malloc((size_t)(d * d) * sizeof(double));
+        if (state_in)
+            memcpy(S, state_in + bh * d * d, (size_t)(d * d) * sizeof(double));
+        else
+            memset(S, 0, (size_t)(d * d) * sizeof(double));
+        for (long t = 0; t < N; ++t) {
+            for (long i = 0; i < d; ++i)
+                for (long j = 0; j < d; ++j) S[i * d + j] += K[t * d + i] * V[t * d + j];
+            for (long j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (long i = 0; i < d; ++i) acc += Q[t * d + i] * S[i * d + j];
+                O[t * d + j] = acc;
+            }
+        }
+        if (state_out) memcpy(state_out + bh * d * d, S, (size_t)(d * d) * sizeof(double));
+        free(S);
+    }
+}
+
+/*
+ * Block form with block size blk, in the order section 1 of the futurefh page
+ * describes: for block i (rows [i*blk, min((i+1)*blk, N)) ),
+ *     O_i = tril(Q_i K_i^T) V_i   (intra-block, left product)
+ *         + Q_i S_{i-1}           (inter-block, right product)
+ *     S_i = S_{i-1} + K_i^T V_i
+ * with S_{-1} = 0.  The last block may be partial.  It exists to show that the
+ * split is exact (it must agree with the two forms above).
+ */
+void oracle_prefill_blockwise(const double* q, const double* k, const double* v,
+                              double* o, double* state_out, long BH, long N, long d,
+                              long blk) {
+    long bh;
+#pragma omp parallel for schedule(dynamic)
+    for (bh = 0; bh < BH; ++bh) {
+        const double* Q = q + bh * N * d;
+        const double* K = k + bh * N * d;
+        const double* V = v + bh * N * d;
+        double* O = o + bh * N * d;
+        double* S = (double*)calloc((size_t)(d * d), sizeof(double));
+        double* P = (double*)malloc((size_t)(blk * blk) * sizeof(double));
+        for (long b0 = 0; b0 < N; b0 += blk) {
+            long nb = (N - b0 < blk) ? (N - b0) : blk;
+            /* P = tril(Q_i K_i^T), diagonal included */
+            for (long r = 0; r < nb; ++r)
+                for (long c = 0; c < nb; ++c) {
+                    double acc = 0.0;
+                    if (c <= r)
+                        for (long x = 0; x < d; ++x) acc += Q[(b0 + r) * d + x] * K[(b0 + c) * d + x];
+                    P[r * blk + c] = acc;
+                }
+            /* O_i = P V_i + Q_i S_{i-1} */
+            for (long r = 0; r < nb; ++r)
+                for (long j = 0; j < d; ++j) {
+                    double intra = 0.0, inter = 0.0;
+                    for (long c = 0; c < nb; ++c) intra += P[r * blk + c] * V[(b0 + c) * d + j];
+                    for (long x = 0; x < d; ++x) inter += Q[(b0 + r) * d + x] * S[x * d + j];
+                    O[(b0 + r) * d + j] = intra + inter;
+                }
+            /* S_i = S_{i-1} + K_i^T V_i */
+            for (long x = 0; x < d; ++x)
+                for (long j = 0; j < d; ++j) {
+                    double acc = 0.0;
+                    for (long c = 0; c < nb; ++c) acc += K[(b0 + c) * d + x] * V[(b0 + c) * d + j];
+                    S[x * d + j] += acc;
+                }
+        }
+        if (state_out) memcpy(state_out + bh * d * d, S, (size_t)(d * d) * sizeof(double));
+        free(P);
+        free(S);
+    }
+}
+
+/*
+ * One decode step (section 3 of the futurefh page runs decode separately from
+ * prefill; the recurrence is the nabfollower page's fixed-size state):
+ *     S <- S + k^T v ;  o = q S        (update first, then read)
+ * q, k, v, o are [BH][d]; S is [BH][d][d] and is updated in place.
+ */
+void oracle_decode_step(const double* q, const double* k, const double* v,
+                        double* S, double* o, long BH, long d) {
+    long bh;
+#pragma omp parallel for schedule(static)
+    for (bh = 0; bh < BH; ++bh) {
+        double* Sb = S + bh * d * d;
+        const double* qb = q + bh * d;
+        const double* kb = k + bh * d;
+        const double* vb = v + bh * d;
+        for (long i = 0; i < d; ++i)
+            for (long j = 0; j < d; ++j) Sb[i * d + j] += kb[i] * vb[j];
+        for (long j = 0; j < d; ++j) {
+            double acc = 0.0;
+            for (long i = 0; i < d; ++i) acc += qb[i] * Sb[i * d + j];
+            o[bh * d + j] = acc;
+        }
+    }
+}
+
+/*
+ * Packed variable-length prefill (data packing, section 4 of the futurefh
+ * page): the recurrent form run separately on every sequence
+ * [cu_seqlens[j], cu_seqlens[j+1]) of every head, the state starting at zero at
+ * each sequence start.  q, k, v, o are [H][T][d]; state_out (may be NULL) is
+ * [num_seqs][H][d][d].  An empty sequence leaves a zero state.
+ * head_list (may be NULL = all heads) restricts the work to n_heads listed
+ * heads; o and state_out are still indexed by the real head number.
+ */
+void oracle_prefill_varlen(const double* q, const double* k, const double* v,
+                           const int* cu_seqlens, long num_seqs, long H, long T, long d,
+                           double* o, double* state_out,
+                           const int* head_list, long n_heads) {
+    long nh = head_list ? n_heads : H;
+    long item;
+#pragma omp parallel for schedule(dynamic)
+    for (item = 0; item < nh * num_seqs; ++item) {
+        long h = head_list ? head_list[item / num_seqs] : item / num_seqs;
+        long j = item % num_seqs;
+        long t0 = cu_seqlens[j], t1 = cu_seqlens[j + 1];
+        const double* Q = q + h * T * d;
+        const double* K = k + h * T * d;
+        const double* V = v + h * T * d;
+        double* O = o + h * T * d;
+        double* S = (double*)calloc((size_t)(d * d), sizeof(double));
+        for (long t = t0; t < t1; ++t) {
+            for (long i = 0; i < d; ++i)
+                for (long c = 0; c < d; ++c) S[i * d + c] += K[t * d + i] * V[t * d + c];
+            for (long c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (long i = 0; i < d; ++i) acc += Q[t * d + i] * S[i * d + c];
+                O[t * d + c] = acc;
+            }
+        }
+        if (state_out) memcpy(state_out + (j * H + h) * d * d, S, (size_t)(d * d) * sizeof(double));
+        free(S);
+    }
+}

@@ -1,0 +1,249 @@
+"""Pins for the fp64 oracle: checks against things other than the oracle itself.
+
+Each pin states what fixes the expected value:
+  * a hand-worked example from the definition (tests/golden/),
+  * the associativity identity (QK^T)V = Q(K^T V) of the nabfollower page
+    ("The Core Tech: Lightning Attention") in its masked consequences:
+    quadratic == recurrent == block form, final state == K^T V (a numpy GEMM),
+    last row == q_{N-1} K^T V,
+  * special cases that reduce to textbook routines (d = 1 is a prefix sum,
+    numpy.cumsum; N = 1 is (q.k) v),
+  * exact brute force in Python integers on small ternary inputs,
+  * the running-state semantics of the closing analogy of the same page:
+    prefill(N) followed by one decode step equals prefill(N+1),
+  * packing (section 4 of the futurefh page): varlen == dense per sequence.
+
+``test_pins_catch_planted_mistakes`` compiles altered copies of oracle.c (a
+dropped diagonal, a transposed operand, a wrong sign, ...) and checks that every
+one of them fails at least one pin, so the pins are strong enough to trust.
+"""
+from __future__ import annotations
+
+import json
+import os
+import tempfile
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _rel(a, b):
+    return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-300))
+
+
+# ----------------------------------------------------------------------------
+# pins, each a function of one compiled oracle
+# ----------------------------------------------------------------------------
+
+def pin_golden(orc):
+    g = json.load(open(os.path.join(GOLDEN, "worked_example_n3_d2.json")))
+    q = np.array(g["q"], float)[None]
+    k = np.array(g["k"], float)[None]
+    v = np.array(g["v"], float)[None]
+    o_ref = np.array(g["o"], float)
+    s_ref = np.array(g["state"], float)
+    assert np.array_equal(orc.prefill_quadratic(q, k, v)[0], o_ref)
+    o, s = orc.prefill_recurrent(q, k, v)
+    assert np.array_equal(o[0], o_ref) and np.array_equal(s[0], s_ref)
+    for blk in (1, 2, 3, 4):
+        o, s = orc.prefill_blockwise(q, k, v, blk)
+        assert np.array_equal(o[0], o_ref) and np.array_equal(s[0], s_ref)
+
+
+def pin_forms_agree(orc):
+    r = _rng(1)
+    for (BH, N, d) in ((3, 67, 8), (2, 130, 16)):
+        q, k, v = (r.standard_normal((BH, N, d)) for _ in range(3))
+        o_quad = orc.prefill_quadratic(q, k, v)
+        o_rec, s_rec = orc.prefill_recurrent(q, k, v)
+        assert _rel(o_rec, o_quad) < 1e-12
+        for blk in (1, 2, 3, 7, 16, 64, N, N + 5):
+            o_blk, s_blk = orc.prefill_blockwise(q, k, v, blk)
+            assert _rel(o_blk, o_quad) < 1e-12, blk
+            assert _rel(s_blk, s_rec) < 1e-12, blk
+
+
+def pin_state_is_KtV(orc):
+    r = _rng(2)
+    q, k, v = (r.standard_normal((2, 50, 12)) for _ in range(3))
+    ktv = np.einsum("bnd,bne->bde", k, v)            # one GEMM per head (numpy)
+    _, s_rec = orc.prefill_recurrent(q, k, v)
+    _, s_blk = orc.prefill_blockwise(q, k, v, 8)
+    assert _rel(s_rec, ktv) < 1e-12
+    assert _rel(s_blk, ktv) < 1e-12
+
+
+def pin_last_row(orc):
+    r = _rng(3)
+    q, k, v = (r.standard_normal((2, 41, 10)) for _ in range(3))
+    ktv = np.einsum("bnd,bne->bde", k, v)
+    want = np.einsum("bd,bde->be", q[:, -1], ktv)     # q_{N-1} (K^T V)
+    for o in (orc.prefill_quadratic(q, k, v), orc.prefill_recurrent(q, k, v)[0],
+              orc.prefill_blockwise(q, k, v, 16)[0]):
+        assert _rel(o[:, -1], want) < 1e-12
+
+
+def pin_d1_prefix_sum(orc):
+    r = _rng(4)
+    q, k, v = (r.standard_normal((3, 90, 1)) for _ in range(3))
+    want = q[..., 0] * np.cumsum(k[..., 0] * v[..., 0], axis=1)   # textbook prefix sum
+    for o in (orc.prefill_quadratic(q, k, v), orc.prefill_recurrent(q, k, v)[0],
+              orc.prefill_blockwise(q, k, v, 7)[0]):
+        assert _rel(o[..., 0], want) < 1e-12
+
+
+def pin_N1(orc):
+    r = _rng(5)
+    q, k, v = (r.standard_normal((4, 1, 9)) for _ in range(3))
+    want = np.sum(q * k, axis=-1, keepdims=True) * v      # (q.k) v
+    for o in (orc.prefill_quadratic(q, k, v), orc.prefill_recurrent(q, k, v)[0],
+              orc.prefill_blockwise(q, k, v, 4)[0]):
+        assert _rel(o, want) < 1e-13
+
+
+def _brute_int(q, k, v):
+    """Exact causal linear attention in Python integers (one head)."""
+    N, d = len(q), len(q[0])
+    o = [[0] * d for _ in range(N)]
+    for t in range(N):
+        for s in range(t + 1):
+            sc = sum(q[t][c] * k[s][c] for c in range(d))
+            for j in range(d):
+                o[t][j] += sc * v[s][j]
+    st = [[sum(k[s][i] * v[s][j] for s in range(N)) for j in range(d)] for i in range(d)]
+    return o, st
+
+
+def pin_ternary_bruteforce(orc):
+    r = _rng(6)
+    for (N, d) in ((1, 3), (5, 2), (23, 6), (40, 4)):
+        q, k, v = (r.integers(-1, 2, (N, d)) for _ in range(3))
+        o_ref, s_ref = _brute_int(q.tolist(), k.tolist(), v.tolist())
+        o_ref = np.array(o_ref, float)[None]
+        s_ref = np.array(s_ref, float)[None]
+        qf, kf, vf = (x[None].astype(float) for x in (q, k, v))
+        assert np.array_equal(orc.prefill_quadratic(qf, kf, vf), o_ref)
+        o, s = orc.prefill_recurrent(qf, kf, vf)
+        assert np.array_equal(o, o_ref) and np.array_equal(s, s_ref)
+        for blk in (1, 3, 8):
+            o, s = orc.prefill_blockwise(qf, kf, vf, blk)
+            assert np.array_equal(o, o_ref) and np.array_equal(s, s_ref)
+
+
+def pin_state_in(orc):
+    """Running from the state of a prefix continues the full sequence."""
+    r = _rng(7)
+    q, k, v = (r.standard_normal((2, 60, 8)) for _ in range(3))
+    o_full, s_full = orc.prefill_quadratic(q, k, v), np.einsum("bnd,bne->bde", k, v)
+    m = 23
+    s_pre = np.einsum("bnd,bne->bde", k[:, :m], v[:, :m])
+    o_tail, s_tail = orc.prefill_recurrent(q[:, m:], k[:, m:], v[:, m:], state_in=s_pre)
+    assert _rel(o_tail, o_full[:, m:]) < 1e-12
+    assert _rel(s_tail, s_full) < 1e-12
+
+
+def pin_decode(orc):
+    r = _rng(8)
+    q, k, v = (r.standard_normal((3, 31, 8)) for _ in range(3))
+    _, s_prev = orc.prefill_recurrent(q[:, :-1], k[:, :-1], v[:, :-1])
+    o1, s1 = orc.decode_step(q[:, -1], k[:, -1], v[:, -1], s_prev)
+    o_full = orc.prefill_quadratic(q, k, v)
+    assert _rel(o1, o_full[:, -1]) < 1e-12
+    assert _rel(s1, np.einsum("bnd,bne->bde", k, v)) < 1e-12
+    # closed form of one step: o = q (S + k^T v)
+    want = np.einsum("bd,bde->be", q[:, -1], s_prev + np.einsum("bd,be->bde", k[:, -1], v[:, -1]))
+    assert _rel(o1, want) < 1e-12
+
+
+def pin_varlen(orc):
+    r = _rng(9)
+    lens = [5, 0, 17, 1, 30]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    H, T, d = 3, int(cu[-1]), 6
+    q, k, v = (r.integers(-1, 2, (H, T, d)).astype(float) for _ in range(3))
+    o, st = orc.prefill_varlen(q, k, v, cu)
+    for j, n in enumerate(lens):
+        a, b = cu[j], cu[j + 1]
+        for h in range(H):
+            if n == 0:
+                assert not np.any(st[j, h])
+                continue
+            o_ref, s_ref = _brute_int(q[h, a:b].astype(int).tolist(), k[h, a:b].astype(int).tolist(),
+                                     v[h, a:b].astype(int).tolist())
+            assert np.array_equal(o[h, a:b], np.array(o_ref, float))
+            assert np.array_equal(st[j, h], np.array(s_ref, float))
+    o2, st2 = orc.prefill_varlen(q, k, v, cu, heads=[2])
+    assert np.array_equal(o2[2], o[2]) and not np.any(o2[:2])
+    assert np.array_equal(st2[:, 2], st[:, 2])
+
+
+PINS = [pin_golden, pin_forms_agree, pin_state_is_KtV, pin_last_row, pin_d1_prefix_sum, pin_N1,
+        pin_ternary_bruteforce, pin_state_in, pin_decode, pin_varlen]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_pin(pin):
+    pin(oracle._get())
+
+
+# ----------------------------------------------------------------------------
+# planted mistakes: every altered oracle must fail at least one pin
+# ----------------------------------------------------------------------------
+
+MUTANTS = {
+    "quadratic_drops_diagonal": ("for (long s = 0; s <= t; ++s)", "for (long s = 0; s < t; ++s)"),
+    "quadratic_wrong_v_index": ("O[t * d + j] += score * V[s * d + j]",
+                                "O[t * d + j] += score * V[t * d + j]"),
+    "recurrent_transposed_update": ("S[i * d + j] += K[t * d + i] * V[t * d + j]",
+                                    "S[i * d + j] += K[t * d + j] * V[t * d + i]"),
+    "recurrent_transposed_read": ("acc += Q[t * d + i] * S[i * d + j]",
+                                  "acc += Q[t * d + i] * S[j * d + i]"),
+    "recurrent_ignores_state_in": ("if (state_in)\n", "if (0 && state_in)\n"),
+    "blockwise_drops_diagonal": ("if (c <= r)", "if (c < r)"),
+    "blockwise_inter_sign": ("= intra + inter;", "= intra - inter;"),
+    "blockwise_state_not_accumulated": ("S[x * d + j] += acc;", "S[x * d + j] = acc;"),
+    "decode_transposed_update": ("Sb[i * d + j] += kb[i] * vb[j]", "Sb[i * d + j] += kb[j] * vb[i]"),
+    "decode_reads_before_update": (
+        "        for (long i = 0; i < d; ++i)\n            for (long j = 0; j < d; ++j) Sb[i * d + j] += kb[i] * vb[j];\n",
+        ""),
+    "varlen_skips_first_token": ("long t0 = cu_seqlens[j], t1", "long t0 = cu_seqlens[j] + 1, t1"),
+    "varlen_no_state_reset_shared_offset": ("O[t * d + c] = acc;", "O[t * d + c] = acc + (t == t0);"),
+}
+
+
+def _pins_fail(orc) -> list:
+    failed = []
+    for p in PINS:
+        try:
+            p(orc)
+        except AssertionError:
+            failed.append(p.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistakes(name):
+    src = open(oracle.SOURCE).read()
+    old, new = MUTANTS[name]
+    assert src.count(old) == 1, "mutation anchor must occur exactly once"
+    if name == "decode_reads_before_update":
+        # move the state update after the read: o = q S_old, then S += k^T v
+        read_end = "            o[bh * d + j] = acc;\n        }\n"
+        assert src.count(read_end) == 1
+        mutated = src.replace(old, "").replace(read_end, read_end + old)
+    else:
+        mutated = src.replace(old, new)
+    with tempfile.TemporaryDirectory() as td:
+        c_path = os.path.join(td, "mut.c")
+        open(c_path, "w").write(mutated)
+        orc = oracle.Oracle(oracle.compile_source(c_path, os.path.join(td, "libmut.so")))
+        failed = _pins_fail(orc)
+    assert failed, f"planted mistake {name} passed every pin"
