@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the Lightning Attention hot path on B200; prints ONE JSON line.
+
+Headline workload (the configuration the metric is quoted on): bf16 prefill,
+B=4, H=16, N=8192, d=128, blk=128, q,k ~ N(0,1/d), v ~ N(0,1), seed 0 (seed +
+rank under torchrun).  A step is one la_prefill call over that batch
+(chunk-state pass, scan over chunks, outputs).  Inputs (384 MiB) and outputs
+exceed the 126 MB L2, so no flush is needed between steps.
+
+  value     tokens/s of the whole job with inputs resident in HBM (max over ranks)
+  e2e       the same metric through the public API with the inputs copied from
+            pinned host memory and o/state copied back inside the timed region
+  roofline  the dominant kernel (prefill_tc_kernel) against measured HBM
+            bandwidth: algorithmic bytes per launch / CUDA-event launch time
+  secondary decode GB/s (128 seq x 64 heads, 256 steps), long-context prefill
+            (B=1, H=64, N=262144), the bf16 blk=64 prefill and the packed
+            varlen prefill where supported (single-GPU runs only)
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm of this
+build) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "lightning-attn prefill tokens/s & % bf16 tensor peak; decode HBM GB/s"
+UNIT = "tokens/s"
+B, H, N, D, BLK = 4, 16, 8192, 128, 128
+BYTES_PER_TOKEN_HEAD = 8 * D                       # q,k,v read + o write, bf16
+FLOPS_PER_TOKEN_HEAD = 4 * BLK * D + 4 * D * D     # dense-tile count (blk 128)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- env
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS)
+
+
+class Dist:
+    """One process per GPU (torchrun env); a no-op when WORLD_SIZE is 1."""
+
+    def __init__(self, backend="nccl"):
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
+        self.pg = None
+
+    def init(self, device=None):
+        if self.world > 1:
+            import torch.distributed as dist
+            kw = {}
+            if self.backend == "nccl" and device is not None:
+                kw["device_id"] = device
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=120), **kw)
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float, device=None) -> float:
+        if self.pg is None:
+            return float(x)
+        import torch
+        t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+            self.pg = None
+
+
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons via NVML in a thread."""
+
+    REASONS = {  # NVML clocks-event reason bits
+        0x8: "hw_slowdown",
+        0x40: "hw_thermal_slowdown",
+        0x20: "sw_thermal_slowdown",
+        0x4: "sw_power_cap",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.05):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 - report instead of failing the bench
+            self.error = repr(e)
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((sm, pw, rs))
+            except Exception:  # noqa: BLE001
+                pass
+            self._stop.wait(self.period)
+
+    def start(self):
+        if self.handle is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+        return self.summary()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": getattr(self, "error", "no samples in the timed region")}
+        reasons = set()
+        for _, _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons),
+                "power_w_max": max(s[1] for s in self.samples),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- ours
+def timed(stream, fn, steps, warmup, dist, device):
+    """W untimed steps, then exactly `steps` timed between CUDA events on
+    `stream`, bracketed by barrier + synchronize; returns max-over-ranks ms."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = start.elapsed_time(end)
+    return dist.max(ms, device)
+
+
+def kernel_times(la):
+    out = {}
+    for kid in range(la.LA_NUM_KERNEL_IDS):
+        st, ms, n = la.la_timing_read(kid)
+        if st == la.LA_OK and n > 0:
+            out[la.la_kernel_name(kid)] = {"total_ms": ms, "launches": n}
+    return out
+
+
+def bench_ours(args, dist):
+    import torch
+    import linear_attention_13_b200 as la
+    from linear_attention_13_b200 import build as labuild
+    from linear_attention_13_b200 import inputs
+
+    labuild.build()
+    device = torch.device("cuda", dist.local_rank)
+    torch.cuda.set_device(device)
+    dist.init(device)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    q, k, v = inputs.qkv((B, H, N, D), dtype=torch.bfloat16, device=device, seed=dist.rank)
+    o = torch.empty_like(q)
+    st = torch.empty((B, H, D, D), dtype=torch.float32, device=device)
+
+    def step():
+        la.prefill(q, k, v, blk=BLK, out=o, state_out=st)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    if la.la_get_last_error() != la.LA_OK:
+        raise RuntimeError("prefill reported a device error")
+
+    sampler = ClockSampler(dist.local_rank).start()
+    la.la_timing_enable(args.steps * 4 + 64)
+    ms = timed(stream, step, args.steps, args.warmup, dist, device)
+    clocks = sampler.stop()
+    ktimes = kernel_times(la)
+    la.la_timing_enable(0)
+    if la.la_get_last_error() != la.LA_OK:
+        raise RuntimeError("prefill reported a device error in the timed region")
+
+    ms_step = ms / args.steps
+    tokens_step = B * N
+    value = dist.world * tokens_step * args.steps / (ms / 1e3)
+    flops_step = B * H * N * FLOPS_PER_TOKEN_HEAD
+    bytes_step = B * H * N * BYTES_PER_TOKEN_HEAD
+    # launches during the timed region = totals minus warm-up launches (the
+    # timing pool was enabled for warm-up + timed steps)
+    launches_total = sum(v["launches"] for v in ktimes.values())
+    launches_timed = launches_total * args.steps // (args.steps + args.warmup)
+
+    main = ktimes.get("prefill_tc_kernel", {"total_ms": float("nan"), "launches": 1})
+    main_ms = main["total_ms"] / max(main["launches"], 1)
+    achieved = bytes_step / (main_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "prefill_tc_kernel", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "algorithmic_bytes_per_launch": bytes_step,
+                "launch_ms": round(main_ms, 5)}
+    step_tflops = flops_step / (ms_step / 1e3) / 1e12
+    tensor = {"tflops": round(step_tflops, 2), "peak_tflops": peaks["bf16_tflops"],
+              "frac_of_peak": round(step_tflops / peaks["bf16_tflops"], 4),
+              "flops_per_token_head": FLOPS_PER_TOKEN_HEAD,
+              "step_hbm_frac": round(bytes_step / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+
+    e2e = bench_e2e(args, dist, device, stream, q, k, v)
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "prefill bf16 B=4 H=16 N=8192 d=128 blk=128",
+                   "global_batch": B * dist.world, "seq_len": N, "heads": H, "head_dim": D,
+                   "blk": BLK, "parallelism": f"dp{dist.world}" if dist.world > 1 else "single",
+                   "l2": "inputs (384 MiB) larger than L2; no flush"},
+        "roofline": roofline,
+        "tensor": tensor,
+        "kernels": {k_: {"avg_ms": round(v_["total_ms"] / max(v_["launches"], 1), 5),
+                         "launches": v_["launches"]} for k_, v_ in ktimes.items()},
+        "gpu_launches": launches_timed,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    del q, k, v, o, st
+    torch.cuda.empty_cache()
+    if dist.world == 1 and not args.no_secondary:
+        result["secondary"] = bench_secondary(args, device, stream, peaks)
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
+    return result
+
+
+def bench_e2e(args, dist, device, stream, qd, kd, vd):
+    """Same metric through the public API with host buffers: every step copies
+    q, k, v from pinned host memory, runs la_prefill, copies o and the state
+    back."""
+    import torch
+    import linear_attention_13_b200 as la
+    hq, hk, hv = (t.to("cpu").pin_memory() for t in (qd, kd, vd))
+    ho = torch.empty(qd.shape, dtype=qd.dtype).pin_memory()
+    hs = torch.empty((B, H, D, D), dtype=torch.float32).pin_memory()
+    dq, dk, dv = (torch.empty_like(qd) for _ in range(3))
+    do = torch.empty_like(qd)
+    ds = torch.empty((B, H, D, D), dtype=torch.float32, device=device)
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        la.prefill(dq, dk, dv, blk=BLK, out=do, state_out=ds)
+        ho.copy_(do, non_blocking=True)
+        hs.copy_(ds, non_blocking=True)
+
+    steps = max(3, min(args.steps, args.e2e_steps))
+    ms = timed(stream, step, steps, 2, dist, device)
+    h2d = 3 * qd.numel() * qd.element_size()
+    d2h = do.numel() * do.element_size() + ds.numel() * 4
+    return {"value": round(dist.world * B * N * steps / (ms / 1e3), 1), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 4)}
+
+
+def bench_secondary(args, device, stream, peaks):
+    import torch
+    import linear_attention_13_b200 as la
+    from linear_attention_13_b200 import inputs
+
+    class _Solo:
+        world = 1
+
+        def barrier(self):
+            pass
+
+        def max(self, x, device=None):
+            return x
+
+    solo = _Solo()
+    out = {}
+
+    # -- decode: 128 sequences x 64 heads, d=128; state from a 4096-token prefill
+    n_seq, Hd, N0, steps = 128, 64, 4096, 256
+    q0, k0, v0 = inputs.qkv((n_seq, Hd, N0, D), dtype=torch.bfloat16, device=device, seed=0)
+    S = torch.empty((n_seq, Hd, D, D), dtype=torch.float32, device=device)
+    o0 = torch.empty_like(q0)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    la.prefill(q0, k0, v0, blk=BLK, out=o0, state_out=S)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    pre_ms = t0.elapsed_time(t1)
+    out["decode_init_prefill"] = {
+        "workload": "prefill bf16 B=128 H=64 N=4096 d=128 (decode initial state, one call)",
+        "tokens_per_s": round(n_seq * N0 / (pre_ms / 1e3), 1), "ms": round(pre_ms, 3),
+        "hbm_frac": round(n_seq * Hd * N0 * BYTES_PER_TOKEN_HEAD / (pre_ms / 1e3) / 1e9 /
+                          peaks["hbm_gbs"], 4)}
+    del q0, k0, v0, o0
+    torch.cuda.empty_cache()
+    step_inputs = [inputs.decode_step_inputs(n_seq, Hd, D, s, device=device)
+                   for s in range(1, steps + 1)]
+    od = torch.empty((n_seq, Hd, D), dtype=torch.bfloat16, device=device)
+    it = iter(range(10 ** 9))
+
+    def dstep():
+        i = next(it) % steps
+        qq, kk, vv = step_inputs[i]
+        la.decode_step(qq, kk, vv, S, out=od)
+
+    la.la_timing_enable(steps + 64)
+    ms = timed(stream, dstep, steps, 5, solo, device)
+    kt = kernel_times(la)
+    la.la_timing_enable(0)
+    dec = kt.get("decode_step_kernel", {"total_ms": float("nan"), "launches": 1})
+    k_ms = dec["total_ms"] / max(dec["launches"], 1)
+    bytes_step = n_seq * Hd * (8 * D * D + 8 * D)
+    out["decode"] = {
+        "workload": "decode step, 128 seq x 64 heads, d=128, fp32 state, 256 steps",
+        "ms_per_step": round(ms / steps, 5), "GB/s": round(bytes_step / (ms / steps / 1e3) / 1e9, 1),
+        "kernel_GB/s": round(bytes_step / (k_ms / 1e3) / 1e9, 1),
+        "hbm_frac": round(bytes_step / (k_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+        "bytes_per_step": bytes_step}
+    del step_inputs, S, od
+    torch.cuda.empty_cache()
+
+    # -- long-context prefill B=1 H=64 N=262144
+    Hl, Nl = 64, 262144
+    q, k, v = inputs.qkv((1, Hl, Nl, D), dtype=torch.bfloat16, device=device, seed=0)
+    o = torch.empty_like(q)
+    st = torch.empty((1, Hl, D, D), dtype=torch.float32, device=device)
+    la.la_timing_enable(64)
+    ms = timed(stream, lambda: la.prefill(q, k, v, blk=BLK, out=o, state_out=st), 5, 2, solo, device)
+    kt = kernel_times(la)
+    la.la_timing_enable(0)
+    bytes_step = Hl * Nl * BYTES_PER_TOKEN_HEAD
+    out["long_prefill"] = {
+        "workload": "prefill bf16 B=1 H=64 N=262144 d=128 blk=128",
+        "tokens_per_s": round(Nl / (ms / 5 / 1e3), 1), "ms_per_step": round(ms / 5, 4),
+        "hbm_frac": round(bytes_step / (ms / 5 / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+        "tensor_frac": round(Hl * Nl * FLOPS_PER_TOKEN_HEAD / (ms / 5 / 1e3) / 1e12 /
+                             peaks["bf16_tflops"], 4),
+        "kernels": {k_: round(v_["total_ms"] / max(v_["launches"], 1), 4) for k_, v_ in kt.items()}}
+    del q, k, v, o, st
+    torch.cuda.empty_cache()
+    return out
+
+
+# ----------------------------------------------------------------------------- oracle
+def cpu_baseline(budget_s: float = 15.0):
+    """The fp64 oracle (recurrent form, OpenMP over heads) on a bounded sample
+    of the headline workload: whole 8192-token heads, as many as fit the time
+    budget; tokens/s = token-heads/s / H."""
+    import torch
+    import oracle
+    from linear_attention_13_b200 import inputs
+    cores = oracle.num_threads()
+    q, k, v = inputs.qkv((1, cores, N, D), dtype=torch.bfloat16, device="cpu", seed=0)
+    q, k, v = (t.to(torch.float64).numpy() for t in (q, k, v))
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.prefill_recurrent(q, k, v)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    token_heads = reps * cores * N
+    return {"value": round(token_heads / dt / H, 1), "unit": UNIT, "cores": cores,
+            "kind": "oracle",
+            "sample": f"{reps} x {cores} heads of N={N}, d={D} (fp64 recurrent form), "
+                      f"{dt:.1f} s; tokens/s = token-heads/s / H ({H})"}
+
+
+def bench_reference(args, dist):
+    """Reference arm: the fp64 CPU oracle, as it stands, on host cores."""
+    import torch
+    import oracle
+    from linear_attention_13_b200 import inputs
+    cores = oracle.num_threads()
+    # size one step so that warm-up + timed steps stay within ~2 minutes
+    step_budget = max(0.05, 120.0 / max(args.steps + args.warmup, 1))
+    q, k, v = inputs.qkv((1, cores, N, D), dtype=torch.bfloat16, device="cpu", seed=0)
+    q, k, v = (t.to(torch.float64).numpy() for t in (q, k, v))
+    t0 = time.perf_counter()
+    oracle.prefill_recurrent(q[:, :, :512], k[:, :, :512], v[:, :, :512])
+    per_token = (time.perf_counter() - t0) / 512
+    n_tok = int(max(128, min(N, step_budget / max(per_token, 1e-9))))
+    qs, ks, vs = q[:, :, :n_tok].copy(), k[:, :, :n_tok].copy(), v[:, :, :n_tok].copy()
+    for _ in range(args.warmup):
+        oracle.prefill_recurrent(qs, ks, vs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.prefill_recurrent(qs, ks, vs)
+    dt = time.perf_counter() - t0
+    value = args.steps * cores * n_tok / dt / H
+    sample = (f"each step: {cores} heads x {n_tok} tokens of the N={N}, d={D} workload "
+              f"(fp64 recurrent oracle); tokens/s = token-heads/s / H ({H})")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT,
+            "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "prefill bf16 B=4 H=16 N=8192 d=128 blk=128 (sampled)",
+                       "global_batch": B, "seq_len": N},
+            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    dist = Dist()
+    if args.impl == "reference":
+        if dist.rank != 0:
+            return 0
+        print(json.dumps(bench_reference(args, dist)), flush=True)
+        return 0
+    res = bench_ours(args, dist)
+    if dist.rank == 0:
+        print(json.dumps(res), flush=True)
+    dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,160 @@
+/*
+ * lightning.h -- C ABI of liblightning.so: causal linear attention
+ * ("Lightning Attention") prefill, packed variable-length prefill and decode
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The operation (no softmax, no scale, no normaliser, diagonal included):
+ *
+ *     S_t = sum_{s <= t} k_s^T v_s          (d x d state, row = key dim)
+ *     o_t = q_t S_t = sum_{s <= t} (q_t . k_s) v_s
+ *
+ * computed block-wise: inside a block of `blk` tokens with the masked left
+ * product (Q K^T ⊙ M) V, across blocks with the right product Q (K^T V) from
+ * the running state, so no cumulative sum over tokens is formed.  Sources:
+ * section 1 of "MiniMax-01技術報告解讀以及與DeepSeek-V3對比" (m.futurefh.com:
+ * intra-block left product, inter-block right product, no slow cumsum);
+ * "The Core Tech: Lightning Attention" of "MiniMax M2.1" (nabfollower.com:
+ * associativity (QK^T)V = Q(K^T V)); section 3 of the futurefh page (prefill and
+ * decode run separately); section 4 (packed sequences).
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - Every pointer is a DEVICE pointer owned by the caller; the library never
+ *    frees or retains it.  Tensors are dense, contiguous, row-major.
+ *  - q, k, v, o have element type `dt` (fp32 or bf16); states are always fp32.
+ *  - Pointers must be 16-byte aligned (LA_ERR_INVALID_ARG otherwise).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    All work is enqueued asynchronously on it; the call returns after
+ *    launching.  Argument errors are returned synchronously and nothing is
+ *    launched.  Errors detected on the device (malformed cu_seqlens, a bounded
+ *    wait that gave up) are recorded in a device status word that
+ *    la_get_last_error() reports.  The library never aborts, prints or traps.
+ *  - Supported sizes: d in {64, 128}; the bf16 tensor-core path needs d == 128
+ *    and blk in {64, 128}; the fp32 path accepts any blk >= 1 with d in {64, 128}.
+ *    N may be any value >= 1 (need not be a multiple of blk).
+ *  - Scratch: long sequences are split into chunks processed in parallel; the
+ *    per-chunk states live in a workspace the library takes from the stream-
+ *    ordered allocator (cudaMallocAsync / cudaFreeAsync on `stream`).
+ *  - Thread safety: calls on different streams may run concurrently.
+ */
+#ifndef LIGHTNING_H_
+#define LIGHTNING_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = -1,   /* null/misaligned pointer, non-positive size  */
+    LA_ERR_UNSUPPORTED = -2,   /* valid but unsupported (d, blk, dtype) combo */
+    LA_ERR_CUDA = -3,          /* a CUDA runtime/driver call failed           */
+    LA_ERR_ALLOC = -4,         /* workspace allocation failed                 */
+    LA_ERR_TIMEOUT = -5,       /* a bounded device-side wait gave up          */
+    LA_ERR_BAD_SEQLENS = -6    /* cu_seqlens not 0..total_tokens non-decreasing */
+} la_status;
+
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+
+/*
+ * la_prefill -- causal linear attention over B*H independent sequences.
+ *   q, k, v  : [B, H, N, d] of dt (read only)
+ *   o        : [B, H, N, d] of dt (written)
+ *   state_out: [B, H, d, d] fp32, final state S_{N-1} = K^T V (written; may be
+ *              NULL when the caller does not need it)
+ *   blk      : block size of the intra/inter split (section 1 of the futurefh
+ *              page).  The result is mathematically independent of blk; blk
+ *              changes only the rounding path.
+ * Returns LA_OK or an la_status error.
+ */
+int la_prefill(const void* q, const void* k, const void* v, void* o, float* state_out,
+               int B, int H, int N, int d, int blk, la_dtype dt, void* stream);
+
+/*
+ * la_prefill_ex -- la_prefill with explicit scheduling controls.
+ *   chunk_tokens: length of the sequence chunks processed in parallel (a
+ *                 multiple of 128 on the bf16 path); 0 = library heuristic;
+ *                 a value >= N forces one chunk per sequence.
+ *   flags       : LA_FLAG_* bits below; 0 = default schedule.
+ */
+#define LA_FLAG_THREE_PASS 1   /* chunk states, scan, then outputs (3 launches) */
+#define LA_FLAG_FUSED      2   /* single persistent launch with look-back      */
+int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* state_out,
+                  int B, int H, int N, int d, int blk, la_dtype dt, void* stream,
+                  int chunk_tokens, int flags);
+
+/*
+ * la_prefill_varlen -- packed variable-length prefill (data packing, section 4
+ * of the futurefh page).  Sequence j occupies tokens [cu_seqlens[j],
+ * cu_seqlens[j+1]) of every head; the state restarts at zero at each sequence
+ * start.
+ *   q, k, v, o : [H, total_tokens, d] of dt, head-major packed
+ *   cu_seqlens : [num_seqs + 1] int32 DEVICE array, cu_seqlens[0] == 0,
+ *                non-decreasing, cu_seqlens[num_seqs] == total_tokens.  It is
+ *                checked on the device; a malformed array sets
+ *                LA_ERR_BAD_SEQLENS in the device status and no output is
+ *                written.  Empty sequences are allowed (zero state).
+ *   state_out  : [num_seqs, H, d, d] fp32 final state per sequence (may be NULL)
+ */
+int la_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* state_out,
+                      const int32_t* cu_seqlens, int num_seqs, int total_tokens,
+                      int H, int d, int blk, la_dtype dt, void* stream);
+
+/*
+ * la_decode_step -- one token per sequence (prefill and decode are separate,
+ * section 3 of the futurefh page):  S <- S + k^T v ;  o = q S  (the update
+ * includes the current token, so prefill(N) + step == prefill(N+1)).
+ *   q, k, v : [B, H, d] of dt (read only)
+ *   state   : [B, H, d, d] fp32, read and updated in place
+ *   o       : [B, H, d] of dt (written)
+ */
+int la_decode_step(const void* q, const void* k, const void* v, float* state, void* o,
+                   int B, int H, int d, la_dtype dt, void* stream);
+
+/* Human-readable name of an la_status value (static storage). */
+const char* la_status_string(int status);
+
+/*
+ * la_get_last_error -- sticky error: the first device-side error recorded
+ * since the last call (see la_status), else the last asynchronous CUDA error,
+ * else LA_OK.  It synchronises the current device and clears the status.
+ */
+int la_get_last_error(void);
+
+/* Number of SMs the library schedules for on the current device (0 on error). */
+int la_device_sm_count(void);
+
+/*
+ * Per-kernel timing (instrumentation).  While enabled, every kernel launch the
+ * library makes on the current device is bracketed by a pair of CUDA events
+ * recorded on the launch's own stream, into a pool of `max_launches` pairs
+ * (launches beyond the pool are counted but not timed).  Kernel ids:
+ *   LA_KERNEL_PREFILL_TC  main tensor-core prefill kernel (outputs)
+ *   LA_KERNEL_CHUNK_STATE per-chunk K^T V (first pass of the chunk scan)
+ *   LA_KERNEL_CHUNK_SCAN  exclusive prefix over chunk states
+ *   LA_KERNEL_PREFILL_F32 fp32 CUDA-core prefill (dense and varlen)
+ *   LA_KERNEL_DECODE      decode step
+ *   LA_KERNEL_AUX         small helper kernels (cu_seqlens check, ...)
+ * la_timing_enable(n) starts a new measurement with room for n launches
+ * (n <= 0 disables timing and releases the events).  la_timing_read
+ * synchronises the device and returns the summed event time in milliseconds
+ * and the launch count of one kernel id since la_timing_enable.
+ */
+#define LA_KERNEL_PREFILL_TC 0
+#define LA_KERNEL_CHUNK_STATE 1
+#define LA_KERNEL_CHUNK_SCAN 2
+#define LA_KERNEL_PREFILL_F32 3
+#define LA_KERNEL_DECODE 4
+#define LA_KERNEL_AUX 5
+#define LA_NUM_KERNEL_IDS 6
+int la_timing_enable(int max_launches);
+int la_timing_read(int kernel_id, double* total_ms, int* launches);
+const char* la_kernel_name(int kernel_id);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIGHTNING_H_ */

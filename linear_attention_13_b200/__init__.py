@@ -1,0 +1,231 @@
+"""linear_attention_13_b200 -- B200-native causal linear attention (Lightning Attention).
+
+Thin Python binding over the C ABI of ``liblightning.so`` (declared in
+``include/lightning.h``).  Every step of the computation runs in the CUDA
+kernels of that library; this module only marshals torch tensors (device
+pointers, sizes, the current CUDA stream) into the C calls and raises on a
+non-OK status.  There is no CPU fallback: if the library is missing or fails
+to load, every call raises.
+
+The raw entry points keep the C names (``la_prefill``, ``la_prefill_ex``,
+``la_prefill_varlen``, ``la_decode_step``, ``la_status_string``,
+``la_get_last_error``, ``la_device_sm_count``).  The tensor-level helpers
+``prefill``, ``prefill_varlen`` and ``decode_step`` allocate outputs and call
+them.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "liblightning.so")
+
+LA_OK = 0
+LA_ERR_INVALID_ARG = -1
+LA_ERR_UNSUPPORTED = -2
+LA_ERR_CUDA = -3
+LA_ERR_ALLOC = -4
+LA_ERR_TIMEOUT = -5
+LA_ERR_BAD_SEQLENS = -6
+
+LA_F32 = 0
+LA_BF16 = 1
+
+LA_FLAG_THREE_PASS = 1
+LA_FLAG_FUSED = 2
+
+LA_KERNEL_PREFILL_TC = 0
+LA_KERNEL_CHUNK_STATE = 1
+LA_KERNEL_CHUNK_SCAN = 2
+LA_KERNEL_PREFILL_F32 = 3
+LA_KERNEL_DECODE = 4
+LA_KERNEL_AUX = 5
+LA_NUM_KERNEL_IDS = 6
+
+EXPORTED = ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step",
+            "la_status_string", "la_get_last_error", "la_device_sm_count",
+            "la_timing_enable", "la_timing_read", "la_kernel_name")
+
+_lib = None
+
+
+class LightningError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load liblightning.so and declare the C signatures.  Raises if absent."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"CUDA library not built: {path} is missing (run __graft_entry__.build() or "
+            "python linear_attention_13_b200/build.py)")
+    lib = ctypes.CDLL(path)
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.la_prefill.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+    lib.la_prefill_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
+    lib.la_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+    lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, vp]
+    lib.la_status_string.argtypes = [i]
+    lib.la_status_string.restype = ctypes.c_char_p
+    lib.la_get_last_error.argtypes = []
+    lib.la_device_sm_count.argtypes = []
+    lib.la_timing_enable.argtypes = [i]
+    lib.la_timing_read.argtypes = [i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]
+    lib.la_kernel_name.argtypes = [i]
+    lib.la_kernel_name.restype = ctypes.c_char_p
+    for name in ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step",
+                 "la_get_last_error", "la_device_sm_count", "la_timing_enable",
+                 "la_timing_read"):
+        getattr(lib, name).restype = ctypes.c_int
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().la_status_string(int(status)).decode()
+
+
+# ---------------------------------------------------------------- raw C names
+def la_prefill(q, k, v, o, state_out, B, H, N, d, blk, dt, stream):
+    return load_library().la_prefill(q, k, v, o, state_out, B, H, N, d, blk, dt, stream)
+
+
+def la_prefill_ex(q, k, v, o, state_out, B, H, N, d, blk, dt, stream, chunk_tokens, flags):
+    return load_library().la_prefill_ex(q, k, v, o, state_out, B, H, N, d, blk, dt, stream,
+                                        chunk_tokens, flags)
+
+
+def la_prefill_varlen(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens, H, d, blk, dt,
+                      stream):
+    return load_library().la_prefill_varlen(q, k, v, o, state_out, cu_seqlens, num_seqs,
+                                            total_tokens, H, d, blk, dt, stream)
+
+
+def la_decode_step(q, k, v, state, o, B, H, d, dt, stream):
+    return load_library().la_decode_step(q, k, v, state, o, B, H, d, dt, stream)
+
+
+def la_status_string(status):
+    return status_string(status)
+
+
+def la_get_last_error():
+    return load_library().la_get_last_error()
+
+
+def la_device_sm_count():
+    return load_library().la_device_sm_count()
+
+
+def la_timing_enable(max_launches):
+    return load_library().la_timing_enable(max_launches)
+
+
+def la_timing_read(kernel_id):
+    """Returns (status, total_ms, launches) for one kernel id."""
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_int(0)
+    st = load_library().la_timing_read(kernel_id, ctypes.byref(ms), ctypes.byref(n))
+    return st, ms.value, n.value
+
+
+def la_kernel_name(kernel_id):
+    return load_library().la_kernel_name(kernel_id).decode()
+
+
+# ---------------------------------------------------------------- tensor helpers
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return LA_BF16
+    if t.dtype == torch.float32:
+        return LA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; expected bfloat16 or float32")
+
+
+def _check(t, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream_ptr(stream):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _raise(status, where):
+    if status != LA_OK:
+        raise LightningError(status, where)
+
+
+def prefill(q, k, v, blk: int = 128, want_state: bool = True, chunk_tokens: int = 0,
+            flags: int = 0, out=None, state_out=None, stream=None):
+    """Causal linear attention prefill of [B,H,N,d] tensors.  Returns (o, state)."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B,H,N,d] shape")
+    B, H, N, d = q.shape
+    o = out if out is not None else torch.empty_like(q)
+    st = state_out
+    if st is None and want_state:
+        st = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    status = la_prefill_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                           st.data_ptr() if st is not None else None, B, H, N, d, blk,
+                           _dtype_code(q), _stream_ptr(stream), chunk_tokens, flags)
+    _raise(status, "la_prefill")
+    return o, st
+
+
+def prefill_varlen(q, k, v, cu_seqlens, blk: int = 128, want_state: bool = True, out=None,
+                   state_out=None, stream=None):
+    """Packed prefill of [H,T,d] tensors split by int32 device cu_seqlens.
+
+    Returns (o, state [num_seqs,H,d,d])."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (cu_seqlens, "cu_seqlens")):
+        _check(t, n)
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    H, T, d = q.shape
+    S = cu_seqlens.numel() - 1
+    o = out if out is not None else torch.empty_like(q)
+    st = state_out
+    if st is None and want_state:
+        st = torch.empty((S, H, d, d), dtype=torch.float32, device=q.device)
+    status = la_prefill_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                               st.data_ptr() if st is not None else None, cu_seqlens.data_ptr(), S,
+                               T, H, d, blk, _dtype_code(q), _stream_ptr(stream))
+    _raise(status, "la_prefill_varlen")
+    return o, st
+
+
+def decode_step(q, k, v, state, out=None, stream=None):
+    """One decode step on [B,H,d] inputs; updates ``state`` [B,H,d,d] fp32 in place."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (state, "state")):
+        _check(t, n)
+    if state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    B, H, d = q.shape
+    o = out if out is not None else torch.empty_like(q)
+    status = la_decode_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), state.data_ptr(),
+                            o.data_ptr(), B, H, d, _dtype_code(q), _stream_ptr(stream))
+    _raise(status, "la_decode_step")
+    return o

@@ -1,0 +1,475 @@
+// lightning.cu -- the C ABI of liblightning.so (declared in include/lightning.h):
+// argument validation, dispatch to the kernels, TMA descriptor creation,
+// stream-ordered workspace, device status.  One translation unit holds every
+// kernel so that the device status word needs no separate device link.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "lightning.h"
+#include "common.cuh"
+#include "ptx.cuh"
+#include "prefill_tc.cuh"
+#include "prefill_simt.cuh"
+#include "decode.cuh"
+
+namespace la {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int sm_count = 0;
+    bool smem_attrs_set = false;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+int g_host_status = LA_OK;   // last asynchronous CUDA error seen by the host
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int note_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return LA_OK;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (g_host_status == LA_OK) g_host_status = LA_ERR_CUDA;
+    return LA_ERR_CUDA;
+}
+
+// Per-device setup: SM count, kernel attributes, the driver entry point.
+int device_setup(int* dev_out, int* sms_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return LA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    DeviceInfo& di = g_dev[dev];
+    if (!di.ready) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return LA_ERR_CUDA;
+        if (cudaFuncSetAttribute(tc::prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(tc::chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::cs::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(simt::prefill_simt_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 simt::smem_bytes<64>()) != cudaSuccess ||
+            cudaFuncSetAttribute(simt::prefill_simt_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 simt::smem_bytes<128>()) != cudaSuccess ||
+            cudaFuncSetAttribute(simt::prefill_simt_varlen_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 simt::smem_bytes<64>()) != cudaSuccess ||
+            cudaFuncSetAttribute(simt::prefill_simt_varlen_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 simt::smem_bytes<128>()) != cudaSuccess) {
+            cudaGetLastError();
+            return LA_ERR_CUDA;
+        }
+        if (g_encode == nullptr) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                                 cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr)
+                return LA_ERR_CUDA;
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+        // Keep up to 2 GiB of freed workspace in the default stream-ordered pool
+        // instead of returning it to the driver at every synchronisation.
+        cudaMemPool_t pool;
+        if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+            uint64_t keep = 2ull << 30;
+            cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        }
+        cudaGetLastError();
+        di.sm_count = sms;
+        di.ready = true;
+    }
+    *dev_out = dev;
+    *sms_out = di.sm_count;
+    return LA_OK;
+}
+
+// ------------------------------------------------------------ kernel timing
+struct Timing {
+    bool enabled = false;
+    int cap = 0;
+    int used = 0;
+    std::vector<cudaEvent_t> ev;     // 2 * cap events (start, stop)
+    std::vector<int> kid;            // kernel id of each used pair
+    int launches[LA_NUM_KERNEL_IDS] = {0};
+};
+Timing g_timing;
+
+void timing_release() {
+    for (cudaEvent_t e : g_timing.ev) cudaEventDestroy(e);
+    g_timing.ev.clear();
+    g_timing.kid.clear();
+    g_timing.cap = g_timing.used = 0;
+    g_timing.enabled = false;
+    for (int& c : g_timing.launches) c = 0;
+}
+
+// Record the start event of a launch of kernel `id` on `s`; returns the slot
+// (or -1 when timing is off or the pool is full).
+int timing_begin(int id, cudaStream_t s) {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (!g_timing.enabled) return -1;
+    g_timing.launches[id]++;
+    if (g_timing.used >= g_timing.cap) return -1;
+    const int slot = g_timing.used++;
+    g_timing.kid[slot] = id;
+    cudaEventRecord(g_timing.ev[2 * slot], s);
+    return slot;
+}
+
+void timing_end(int slot, cudaStream_t s) {
+    if (slot < 0) return;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (slot < g_timing.used) cudaEventRecord(g_timing.ev[2 * slot + 1], s);
+}
+
+// Brackets one kernel launch with timing events.
+struct TimedLaunch {
+    int slot;
+    cudaStream_t s;
+    TimedLaunch(int id, cudaStream_t st) : slot(timing_begin(id, st)), s(st) {}
+    ~TimedLaunch() { timing_end(slot, s); }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D bf16 tensor map over [outer][rows][128] with a {64, 128, 1} box and the
+// 128-byte swizzle; rows past `rows` read as zero.
+int make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t outer) {
+    cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows, (cuuint64_t)outer};
+    cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)rows * kHeadDim * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)kTileRows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LA_OK : LA_ERR_CUDA;
+}
+
+// Chunk length (tokens, multiple of 128) for the bf16 dense path: the
+// makespan of ceil(items / CTAs) rounds of (blocks per chunk + per-chunk
+// overhead) is minimised, with chunks of at least 512 tokens.
+int choose_chunk_tokens(int BH, int N, int ctas) {
+    const int nblk = (N + kTileRows - 1) / kTileRows;
+    int best_blocks = nblk;
+    double best_cost = 1e300;
+    const int min_blocks = std::min(4, nblk);
+    for (int cb = nblk; cb >= min_blocks; --cb) {
+        const int nchunks = (nblk + cb - 1) / cb;
+        if (nchunks > 1 && cb * (nchunks - 1) >= nblk) continue;
+        const long items = (long)BH * nchunks;
+        const long rounds = (items + ctas - 1) / ctas;
+        const double cost = (double)rounds * (cb + 1.5) + (nchunks > 1 ? 3.0 : 0.0);
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best_blocks = cb;
+        }
+    }
+    return best_blocks * kTileRows;
+}
+
+int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, float* state_out,
+                        int BH, int N, int blk, cudaStream_t stream, int sms, int chunk_tokens) {
+    if (blk != 128) return LA_ERR_UNSUPPORTED;
+    CUtensorMap tq, tk, tv;
+    if (make_tmap_bf16(&tq, q, N, BH) || make_tmap_bf16(&tk, k, N, BH) ||
+        make_tmap_bf16(&tv, v, N, BH))
+        return LA_ERR_CUDA;
+    if (chunk_tokens <= 0) chunk_tokens = choose_chunk_tokens(BH, N, sms);
+    chunk_tokens = ((chunk_tokens + kTileRows - 1) / kTileRows) * kTileRows;
+    const int n_chunks = (N + chunk_tokens - 1) / chunk_tokens;
+
+    tc::DenseParams p;
+    p.BH = BH;
+    p.N = N;
+    p.chunk_tokens = chunk_tokens;
+    p.n_chunks = n_chunks;
+    p.n_items = BH * n_chunks;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.prefix = nullptr;
+    p.state_out = nullptr;
+    p.chunk_delta = nullptr;
+    const int grid = std::min(p.n_items, sms);
+
+    if (n_chunks == 1) {
+        p.state_out = state_out;
+        {
+            TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
+            tc::prefill_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(tq, tk, tv, p);
+        }
+        return note_cuda(cudaGetLastError());
+    }
+    float* ws = nullptr;
+    const size_t ws_bytes = (size_t)BH * n_chunks * kHeadDim * kHeadDim * sizeof(float);
+    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), ws_bytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_ALLOC;
+    }
+    p.chunk_delta = ws;
+    {
+        TimedLaunch tl(LA_KERNEL_CHUNK_STATE, stream);
+        tc::chunk_state_kernel<<<grid, tc::kThreads, tc::cs::kSmemBytes, stream>>>(tk, tv, p);
+    }
+    {
+        TimedLaunch tl(LA_KERNEL_CHUNK_SCAN, stream);
+        dim3 sgrid(kHeadDim * kHeadDim / 4 / 256, BH);
+        tc::chunk_scan_kernel<<<sgrid, 256, 0, stream>>>(ws, state_out, n_chunks);
+    }
+    p.prefix = ws;
+    p.state_out = nullptr;
+    {
+        TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
+        tc::prefill_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(tq, tk, tv, p);
+    }
+    int st = note_cuda(cudaGetLastError());
+    cudaFreeAsync(ws, stream);
+    return st;
+}
+
+int validate_common(const void* q, const void* k, const void* v, const void* o, int d, int blk,
+                    la_dtype dt) {
+    if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LA_ERR_INVALID_ARG;
+    if (blk < 1) return LA_ERR_INVALID_ARG;
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
+    if (dt == LA_BF16 && (d != 128 || (blk != 64 && blk != 128))) return LA_ERR_UNSUPPORTED;
+    return LA_OK;
+}
+
+}  // namespace
+}  // namespace la
+
+using namespace la;
+
+extern "C" {
+
+int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* state_out, int B,
+                  int H, int N, int d, int blk, la_dtype dt, void* stream, int chunk_tokens,
+                  int flags) {
+    (void)flags;
+    if (B < 1 || H < 1 || N < 1) return LA_ERR_INVALID_ARG;
+    int st = validate_common(q, k, v, o, d, blk, dt);
+    if (st != LA_OK) return st;
+    if (state_out && !aligned16(state_out)) return LA_ERR_INVALID_ARG;
+    if ((long long)B * H > (1ll << 30) || (long long)N > (1ll << 30)) return LA_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    st = device_setup(&dev, &sms);
+    if (st != LA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int BH = B * H;
+    if (dt == LA_F32) {
+        const float* qf = reinterpret_cast<const float*>(q);
+        const float* kf = reinterpret_cast<const float*>(k);
+        const float* vf = reinterpret_cast<const float*>(v);
+        float* of = reinterpret_cast<float*>(o);
+        TimedLaunch tl(LA_KERNEL_PREFILL_F32, s);
+        if (d == 64)
+            simt::prefill_simt_kernel<64><<<BH, simt::kThreads, simt::smem_bytes<64>(), s>>>(
+                qf, kf, vf, of, state_out, N, blk);
+        else
+            simt::prefill_simt_kernel<128><<<BH, simt::kThreads, simt::smem_bytes<128>(), s>>>(
+                qf, kf, vf, of, state_out, N, blk);
+        return note_cuda(cudaGetLastError());
+    }
+    return launch_prefill_bf16(q, k, v, o, state_out, BH, N, blk, s, sms, chunk_tokens);
+}
+
+int la_prefill(const void* q, const void* k, const void* v, void* o, float* state_out, int B, int H,
+               int N, int d, int blk, la_dtype dt, void* stream) {
+    return la_prefill_ex(q, k, v, o, state_out, B, H, N, d, blk, dt, stream, 0, 0);
+}
+
+int la_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* state_out,
+                      const int32_t* cu_seqlens, int num_seqs, int total_tokens, int H, int d,
+                      int blk, la_dtype dt, void* stream) {
+    if (num_seqs < 1 || total_tokens < 0 || H < 1 || cu_seqlens == nullptr) return LA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return LA_ERR_INVALID_ARG;
+    int st = validate_common(q, k, v, o, d, blk, dt);
+    if (st != LA_OK) return st;
+    if (state_out && !aligned16(state_out)) return LA_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    st = device_setup(&dev, &sms);
+    if (st != LA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dt != LA_F32) return LA_ERR_UNSUPPORTED;
+    int* ok = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&ok), sizeof(int), s) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_ALLOC;
+    }
+    {
+        TimedLaunch tl(LA_KERNEL_AUX, s);
+        check_seqlens_kernel<<<1, 256, 0, s>>>(cu_seqlens, num_seqs, total_tokens, ok);
+    }
+    dim3 grid(num_seqs, H);
+    const float* qf = reinterpret_cast<const float*>(q);
+    const float* kf = reinterpret_cast<const float*>(k);
+    const float* vf = reinterpret_cast<const float*>(v);
+    float* of = reinterpret_cast<float*>(o);
+    {
+    TimedLaunch tl(LA_KERNEL_PREFILL_F32, s);
+    if (d == 64)
+        simt::prefill_simt_varlen_kernel<64><<<grid, simt::kThreads, simt::smem_bytes<64>(), s>>>(
+            qf, kf, vf, of, state_out, cu_seqlens, ok, num_seqs, H, total_tokens, blk);
+    else
+        simt::prefill_simt_varlen_kernel<128><<<grid, simt::kThreads, simt::smem_bytes<128>(), s>>>(
+            qf, kf, vf, of, state_out, cu_seqlens, ok, num_seqs, H, total_tokens, blk);
+    }
+    st = note_cuda(cudaGetLastError());
+    cudaFreeAsync(ok, s);
+    return st;
+}
+
+int la_decode_step(const void* q, const void* k, const void* v, float* state, void* o, int B, int H,
+                   int d, la_dtype dt, void* stream) {
+    if (B < 1 || H < 1) return LA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o || !state) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state))
+        return LA_ERR_INVALID_ARG;
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1ll << 31) - 1) return LA_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    int st = device_setup(&dev, &sms);
+    if (st != LA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const unsigned grid = (unsigned)(B * H);
+    TimedLaunch tl(LA_KERNEL_DECODE, s);
+    if (dt == LA_BF16) {
+        const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(q);
+        const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(k);
+        const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(v);
+        __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(o);
+        if (d == 128)
+            decode::decode_step_kernel<__nv_bfloat16, 128><<<grid, decode::kThreads, 0, s>>>(qb, kb, vb, state, ob);
+        else
+            decode::decode_step_kernel<__nv_bfloat16, 64><<<grid, decode::kThreads, 0, s>>>(qb, kb, vb, state, ob);
+    } else {
+        const float* qf = reinterpret_cast<const float*>(q);
+        const float* kf = reinterpret_cast<const float*>(k);
+        const float* vf = reinterpret_cast<const float*>(v);
+        float* of = reinterpret_cast<float*>(o);
+        if (d == 128)
+            decode::decode_step_kernel<float, 128><<<grid, decode::kThreads, 0, s>>>(qf, kf, vf, state, of);
+        else
+            decode::decode_step_kernel<float, 64><<<grid, decode::kThreads, 0, s>>>(qf, kf, vf, state, of);
+    }
+    return note_cuda(cudaGetLastError());
+}
+
+const char* la_status_string(int status) {
+    switch (status) {
+        case LA_OK: return "LA_OK";
+        case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA";
+        case LA_ERR_ALLOC: return "LA_ERR_ALLOC";
+        case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT";
+        case LA_ERR_BAD_SEQLENS: return "LA_ERR_BAD_SEQLENS";
+        default: return "LA_UNKNOWN_STATUS";
+    }
+}
+
+int la_get_last_error(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    int dev_status = LA_OK;
+    if (cudaMemcpyFromSymbol(&dev_status, la::g_device_status, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    const int zero = LA_OK;
+    cudaMemcpyToSymbol(la::g_device_status, &zero, sizeof(int));
+    int host_status;
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        host_status = g_host_status;
+        g_host_status = LA_OK;
+    }
+    if (dev_status != LA_OK) return dev_status;
+    return host_status;
+}
+
+int la_device_sm_count(void) {
+    int dev = 0, sms = 0;
+    if (device_setup(&dev, &sms) != LA_OK) return 0;
+    return sms;
+}
+
+int la_timing_enable(int max_launches) {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (!g_timing.ev.empty()) cudaDeviceSynchronize();
+    timing_release();
+    if (max_launches <= 0) return LA_OK;
+    g_timing.ev.resize(2 * (size_t)max_launches);
+    g_timing.kid.assign(max_launches, -1);
+    for (auto& e : g_timing.ev) {
+        if (cudaEventCreate(&e) != cudaSuccess) {
+            cudaGetLastError();
+            e = nullptr;
+            timing_release();
+            return LA_ERR_CUDA;
+        }
+    }
+    g_timing.cap = max_launches;
+    g_timing.enabled = true;
+    return LA_OK;
+}
+
+int la_timing_read(int kernel_id, double* total_ms, int* launches) {
+    if (kernel_id < 0 || kernel_id >= LA_NUM_KERNEL_IDS || !total_ms || !launches)
+        return LA_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lk(g_mutex);
+    double sum = 0.0;
+    for (int i = 0; i < g_timing.used; ++i) {
+        if (g_timing.kid[i] != kernel_id) continue;
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, g_timing.ev[2 * i], g_timing.ev[2 * i + 1]) != cudaSuccess) {
+            cudaGetLastError();
+            return LA_ERR_CUDA;
+        }
+        sum += ms;
+    }
+    *total_ms = sum;
+    *launches = g_timing.launches[kernel_id];
+    return LA_OK;
+}
+
+const char* la_kernel_name(int kernel_id) {
+    switch (kernel_id) {
+        case LA_KERNEL_PREFILL_TC: return "prefill_tc_kernel";
+        case LA_KERNEL_CHUNK_STATE: return "chunk_state_kernel";
+        case LA_KERNEL_CHUNK_SCAN: return "chunk_scan_kernel";
+        case LA_KERNEL_PREFILL_F32: return "prefill_simt_kernel";
+        case LA_KERNEL_DECODE: return "decode_step_kernel";
+        case LA_KERNEL_AUX: return "check_seqlens_kernel";
+        default: return "unknown";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+"""The C-ABI library builds, loads and exports every entry point that
+include/lightning.h declares; host-side argument validation answers without a
+GPU (no compute call is made: validation fails before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_13_b200 as la
+from linear_attention_13_b200 import build as labuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_entry_points():
+    text = open(os.path.join(ROOT, "include", "lightning.h")).read()
+    return sorted(set(re.findall(r"^(?:int|const char\*)\s+(la_\w+)\s*\(", text, re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    labuild.build()
+    return la.load_library()
+
+
+def test_header_declares_expected_entry_points():
+    names = _declared_entry_points()
+    for n in ("la_prefill", "la_prefill_varlen", "la_decode_step", "la_status_string",
+              "la_get_last_error"):
+        assert n in names
+    assert set(names) == set(la.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in _declared_entry_points():
+        assert hasattr(lib, n), n
+        assert isinstance(getattr(lib, n), ctypes._CFuncPtr)
+
+
+def test_library_is_built_for_sm100a():
+    labuild.build()
+    out = open(la.LIB_PATH, "rb").read()
+    assert b"sm_100a" in out
+
+
+def test_status_strings(lib):
+    assert la.status_string(la.LA_OK) == "LA_OK"
+    assert la.status_string(la.LA_ERR_BAD_SEQLENS) == "LA_ERR_BAD_SEQLENS"
+    assert la.status_string(12345) == "LA_UNKNOWN_STATUS"
+
+
+FAKE = 0x100000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((None, FAKE, FAKE, FAKE, None, 1, 1, 16, 128, 128, la.LA_BF16, None), la.LA_ERR_INVALID_ARG),
+    ((FAKE + 2, FAKE, FAKE, FAKE, None, 1, 1, 16, 128, 128, la.LA_BF16, None), la.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, None, 0, 1, 16, 128, 128, la.LA_BF16, None), la.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 1, 0, 128, 128, la.LA_BF16, None), la.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 1, 16, 96, 128, la.LA_BF16, None), la.LA_ERR_UNSUPPORTED),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 1, 16, 64, 128, la.LA_BF16, None), la.LA_ERR_UNSUPPORTED),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 1, 16, 128, 32, la.LA_BF16, None), la.LA_ERR_UNSUPPORTED),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 1, 16, 128, 0, la.LA_F32, None), la.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 1, 16, 128, 64, 7, None), la.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE + 4, 1, 1, 16, 128, 64, la.LA_F32, None), la.LA_ERR_INVALID_ARG),
+])
+def test_prefill_argument_validation(lib, args, expect):
+    assert la.la_prefill(*args) == expect
+
+
+def test_varlen_and_decode_argument_validation(lib):
+    assert la.la_prefill_varlen(FAKE, FAKE, FAKE, FAKE, None, None, 1, 16, 1, 128, 128,
+                                la.LA_BF16, None) == la.LA_ERR_INVALID_ARG
+    assert la.la_prefill_varlen(FAKE, FAKE, FAKE, FAKE, None, FAKE + 2, 1, 16, 1, 128, 128,
+                                la.LA_BF16, None) == la.LA_ERR_INVALID_ARG
+    assert la.la_prefill_varlen(FAKE, FAKE, FAKE, FAKE, None, FAKE, 0, 16, 1, 128, 128,
+                                la.LA_BF16, None) == la.LA_ERR_INVALID_ARG
+    assert la.la_decode_step(FAKE, FAKE, FAKE, None, FAKE, 1, 1, 128, la.LA_BF16,
+                             None) == la.LA_ERR_INVALID_ARG
+    assert la.la_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 32, la.LA_BF16,
+                             None) == la.LA_ERR_UNSUPPORTED
+    assert la.la_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 128, la.LA_BF16,
+                             None) == la.LA_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="not built"):
+        la.load_library(str(tmp_path / "nope.so"))

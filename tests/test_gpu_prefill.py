@@ -1,0 +1,143 @@
+"""GPU parity of la_prefill (called through the C ABI) against the fp64 oracle.
+
+Inputs are the seeded synthetic draws of linear_attention_13_b200.inputs; the
+oracle consumes the same rounded values.  Bars: per-head relative error of o
+<= 1e-4 (fp32) / 2e-2 (bf16), of the final state <= 1e-3; bit-exact equality
+on small-integer inputs where every intermediate is exactly representable.
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_13_b200 as la
+from linear_attention_13_b200 import inputs
+import oracle
+from _util import TOL_O_BF16, TOL_O_F32, TOL_STATE, host64, per_head_rel_err, round_like
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _run(q, k, v, blk, **kw):
+    o, st = la.prefill(q, k, v, blk=blk, **kw)
+    assert la.la_get_last_error() == la.LA_OK
+    return o, st
+
+
+def test_tiny_fp32_config():
+    # B=1, H=2, N=256, d=64, blk=64, fp32, seed 0
+    q, k, v = inputs.qkv((1, 2, 256, 64), dtype=torch.float32, device=DEV, seed=0)
+    o, st = _run(q, k, v, 64)
+    o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert per_head_rel_err(host64(o), o_ref) <= TOL_O_F32
+    assert per_head_rel_err(host64(st), s_ref) <= TOL_STATE
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("blk", [1, 7, 64, 100, 256, 1000])
+def test_fp32_block_sizes(d, blk):
+    q, k, v = inputs.qkv((1, 3, 300, d), dtype=torch.float32, device=DEV, seed=blk)
+    o, st = _run(q, k, v, blk)
+    o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert per_head_rel_err(host64(o), o_ref) <= TOL_O_F32
+    assert per_head_rel_err(host64(st), s_ref) <= TOL_STATE
+
+
+def test_fp32_ternary_exact():
+    q, k, v = inputs.ternary_qkv((2, 2, 200, 64), dtype=torch.float32, device=DEV, seed=3)
+    o, st = _run(q, k, v, 64)
+    o_ref, s_ref = oracle.prefill_quadratic(host64(q), host64(k), host64(v)), None
+    _, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert np.array_equal(host64(o), o_ref)
+    assert np.array_equal(host64(st), s_ref)
+
+
+@pytest.mark.parametrize("N", [1, 2, 127, 128, 129, 255, 300, 1000, 2049])
+@pytest.mark.parametrize("chunk", [0, 128, 384])
+def test_bf16_ragged_lengths_and_chunks(N, chunk):
+    q, k, v = inputs.qkv((2, 3, N, 128), dtype=torch.bfloat16, device=DEV, seed=N + chunk)
+    o, st = _run(q, k, v, 128, chunk_tokens=chunk)
+    o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16
+    assert per_head_rel_err(host64(st), s_ref) <= TOL_STATE
+
+
+@pytest.mark.parametrize("N,chunk", [(100, 0), (256, 0), (256, 128), (200, 128)])
+def test_bf16_ternary_bit_exact(N, chunk):
+    # |q.k| <= 128 and |S| <= N <= 256 are exact in bf16; fp32 sums are exact;
+    # only the final o conversion rounds, with round-to-nearest-even.
+    q, k, v = inputs.ternary_qkv((1, 4, N, 128), dtype=torch.bfloat16, device=DEV, seed=N)
+    o, st = _run(q, k, v, 128, chunk_tokens=chunk)
+    o_ref = oracle.prefill_quadratic(host64(q), host64(k), host64(v))
+    _, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert np.array_equal(host64(o), round_like(o_ref, torch.bfloat16))
+    assert np.array_equal(host64(st), s_ref)
+
+
+@pytest.mark.parametrize("chunk", [0, 1024, 8192])
+def test_bf16_onehot_long_bit_exact(chunk):
+    # one nonzero per key row keeps every state entry a small integer, so even
+    # the multi-chunk path (chunk states, scan, prefix start) is exact.
+    q, k, v = inputs.onehot_k_qkv((1, 4, 8192, 128), dtype=torch.bfloat16, device=DEV, seed=11)
+    o, st = _run(q, k, v, 128, chunk_tokens=chunk)
+    o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert np.max(np.abs(s_ref)) <= 256
+    assert np.array_equal(host64(o), round_like(o_ref, torch.bfloat16))
+    assert np.array_equal(host64(st), s_ref)
+
+
+@pytest.mark.parametrize("blk", [128])
+def test_bf16_prefill_config_all_heads(blk):
+    # B=4, H=16, N=8192, d=128: every head against the oracle, in the launch
+    # configuration the benchmark times (library-chosen chunking).
+    q, k, v = inputs.qkv((4, 16, 8192, 128), dtype=torch.bfloat16, device=DEV, seed=0)
+    o, st = _run(q, k, v, blk)
+    o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16
+    assert per_head_rel_err(host64(st), s_ref) <= TOL_STATE
+
+
+def test_bf16_long_context_sampled_heads():
+    # B=1, H=64, N=262144, d=128: 4 sampled heads (first, last, two seeded).
+    B, H, N, d = 1, 64, 262144, 128
+    q, k, v = inputs.qkv((B, H, N, d), dtype=torch.bfloat16, device=DEV, seed=0)
+    o, st = _run(q, k, v, 128)
+    rng = np.random.default_rng(0)
+    heads = [0, H - 1] + sorted(rng.choice(np.arange(1, H - 1), 2, replace=False).tolist())
+    hq, hk, hv = (host64(x[0, heads]) for x in (q, k, v))
+    o_ref, s_ref = oracle.prefill_recurrent(hq, hk, hv)
+    assert per_head_rel_err(host64(o[0, heads]), o_ref) <= TOL_O_BF16
+    assert per_head_rel_err(host64(st[0, heads]), s_ref) <= TOL_STATE
+
+
+def test_bf16_scaling_is_exact():
+    q, k, v = inputs.qkv((1, 2, 700, 128), dtype=torch.bfloat16, device=DEV, seed=5)
+    o1, s1 = _run(q, k, v, 128, chunk_tokens=256)
+    o2, s2 = _run(q * 2, k, v, 128, chunk_tokens=256)
+    o3, s3 = _run(q, k, v * 2, 128, chunk_tokens=256)
+    assert torch.equal(o2, o1 * 2) and torch.equal(s2, s1)
+    assert torch.equal(o3, o1 * 2) and torch.equal(s3, s1 * 2)
+
+
+def test_no_writes_outside_outputs():
+    B, H, N, d = 1, 3, 333, 128
+    q, k, v = inputs.qkv((B, H, N, d), dtype=torch.bfloat16, device=DEV, seed=9)
+    pad = 4096
+    o_buf = torch.full((pad + B * H * N * d + pad,), 7.0, dtype=torch.bfloat16, device=DEV)
+    s_buf = torch.full((pad + B * H * d * d + pad,), 7.0, dtype=torch.float32, device=DEV)
+    o = o_buf[pad:pad + B * H * N * d].view(B, H, N, d)
+    s = s_buf[pad:pad + B * H * d * d].view(B, H, d, d)
+    la.prefill(q, k, v, blk=128, out=o, state_out=s, chunk_tokens=128)
+    assert la.la_get_last_error() == la.LA_OK
+    assert torch.all(o_buf[:pad] == 7.0) and torch.all(o_buf[-pad:] == 7.0)
+    assert torch.all(s_buf[:pad] == 7.0) and torch.all(s_buf[-pad:] == 7.0)
+    o_ref, _ = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16
+
+
+def test_without_state_output():
+    q, k, v = inputs.qkv((1, 2, 600, 128), dtype=torch.bfloat16, device=DEV, seed=6)
+    o, st = la.prefill(q, k, v, blk=128, want_state=False, chunk_tokens=256)
+    assert st is None and la.la_get_last_error() == la.LA_OK
+    o_ref, _ = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16
