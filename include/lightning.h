@@ -153,6 +153,35 @@ int la_timing_enable(int max_launches);
 int la_timing_read(int kernel_id, double* total_ms, int* launches);
 const char* la_kernel_name(int kernel_id);
 
+/*
+ * la_prefill_noalloc -- la_prefill (bf16, d = 128) that allocates no device
+ * memory.  The paper has no counterpart to this entry point: it is a
+ * packaging variant of the bf16 prefill for callers that cannot call
+ * cudaMalloc or the stream-ordered allocator, for example code running inside
+ * a framework that has already reserved nearly all device memory for its own
+ * pool (so any allocation by a library would fail), or a runtime that forbids
+ * allocations outside its planned arena.
+ *
+ * Arguments, layouts, results and errors are those of la_prefill.  The
+ * per-chunk states that la_prefill keeps in an allocated workspace live here
+ * in one fixed array inside the library, LA_NOALLOC_SCRATCH_BYTES large,
+ * which every GPU that loads the library holds until the process exits.  The
+ * chunking is the one la_prefill chooses; if B*H*n_chunks*d*d*4 bytes of chunk
+ * states exceed the array, the call returns LA_ERR_UNSUPPORTED and launches
+ * nothing.  (A sequence that fits one chunk needs no scratch at all.)
+ *
+ * The first call on each device looks up the device address of the array
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls on a device share the one array and
+ * it keeps whatever the last call left in it (every entry is overwritten
+ * before it is read, so nothing needs clearing); two calls whose work
+ * overlaps on the GPU (different streams, no ordering between them) race on
+ * it and must not be issued.
+ */
+#define LA_NOALLOC_SCRATCH_BYTES (16u << 20)
+int la_prefill_noalloc(const void* q, const void* k, const void* v, void* o, float* state_out,
+                       int B, int H, int N, int d, int blk, la_dtype dt, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

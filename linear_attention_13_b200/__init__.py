@@ -45,7 +45,9 @@ LA_NUM_KERNEL_IDS = 6
 
 EXPORTED = ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step",
             "la_status_string", "la_get_last_error", "la_device_sm_count",
-            "la_timing_enable", "la_timing_read", "la_kernel_name")
+            "la_timing_enable", "la_timing_read", "la_kernel_name", "la_prefill_noalloc")
+
+LA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 _lib = None
 
@@ -77,11 +79,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la_device_sm_count.argtypes = []
     lib.la_timing_enable.argtypes = [i]
     lib.la_timing_read.argtypes = [i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]
+    lib.la_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.la_kernel_name.argtypes = [i]
     lib.la_kernel_name.restype = ctypes.c_char_p
     for name in ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step",
                  "la_get_last_error", "la_device_sm_count", "la_timing_enable",
-                 "la_timing_read"):
+                 "la_timing_read", "la_prefill_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -106,6 +109,11 @@ def la_prefill_varlen(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens,
                       stream):
     return load_library().la_prefill_varlen(q, k, v, o, state_out, cu_seqlens, num_seqs,
                                             total_tokens, H, d, blk, dt, stream)
+
+
+def la_prefill_noalloc(q, k, v, o, state_out, B, H, N, d, blk, dt, stream):
+    """la_prefill that allocates no device memory (fixed in-library scratch)."""
+    return load_library().la_prefill_noalloc(q, k, v, o, state_out, B, H, N, d, blk, dt, stream)
 
 
 def la_decode_step(q, k, v, state, o, B, H, d, dt, stream):

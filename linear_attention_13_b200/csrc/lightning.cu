@@ -255,6 +255,78 @@ int validate_common(const void* q, const void* k, const void* v, const void* o, 
     return LA_OK;
 }
 
+// ------------------------------------------------------------ no-alloc scratch
+// Fixed scratch for la_prefill_noalloc: chunk states of the bf16 prefill for
+// callers that cannot allocate device memory.  Host code must not use the
+// name as a device address; it asks for the address per device below.
+static __device__ __align__(256) float g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+float* g_noalloc_addr[kMaxDevices] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device `dev`, looked up
+// once per device (the first call on a device does it).
+int noalloc_scratch(int dev, float** out) {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* ptr = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || ptr == nullptr) {
+            cudaGetLastError();
+            return LA_ERR_CUDA;
+        }
+        g_noalloc_addr[dev] = static_cast<float*>(ptr);
+    }
+    *out = g_noalloc_addr[dev];
+    return LA_OK;
+}
+
+// The bf16 chunked prefill with the chunk states in the fixed scratch.
+int launch_prefill_bf16_noalloc(const void* q, const void* k, const void* v, void* o,
+                                float* state_out, int BH, int N, int blk, cudaStream_t stream,
+                                int dev, int sms) {
+    if (blk != 128) return LA_ERR_UNSUPPORTED;
+    int chunk_tokens = choose_chunk_tokens(BH, N, sms);
+    const int n_chunks = (N + chunk_tokens - 1) / chunk_tokens;
+    const size_t ws_bytes = (size_t)BH * n_chunks * kHeadDim * kHeadDim * sizeof(float);
+    if (n_chunks > 1 && ws_bytes > (size_t)LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_UNSUPPORTED;
+    float* ws = nullptr;
+    if (n_chunks > 1) {
+        const int st = noalloc_scratch(dev, &ws);
+        if (st != LA_OK) return st;
+    }
+    CUtensorMap tq, tk, tv;
+    if (make_tmap_bf16(&tq, q, N, BH) || make_tmap_bf16(&tk, k, N, BH) ||
+        make_tmap_bf16(&tv, v, N, BH))
+        return LA_ERR_CUDA;
+    tc::DenseParams p;
+    p.BH = BH;
+    p.N = N;
+    p.chunk_tokens = chunk_tokens;
+    p.n_chunks = n_chunks;
+    p.n_items = BH * n_chunks;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.prefix = nullptr;
+    p.state_out = n_chunks == 1 ? state_out : nullptr;
+    p.chunk_delta = ws;
+    const int grid = std::min(p.n_items, sms);
+    if (n_chunks > 1) {
+        {
+            TimedLaunch tl(LA_KERNEL_CHUNK_STATE, stream);
+            tc::chunk_state_kernel<<<grid, tc::kThreads, tc::cs::kSmemBytes, stream>>>(tk, tv, p);
+        }
+        {
+            TimedLaunch tl(LA_KERNEL_CHUNK_SCAN, stream);
+            dim3 sgrid(kHeadDim * kHeadDim / 4 / 256, BH);
+            tc::chunk_scan_kernel<<<sgrid, 256, 0, stream>>>(ws, state_out, n_chunks);
+        }
+        p.prefix = ws;
+    }
+    {
+        TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
+        tc::prefill_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(tq, tk, tv, p);
+    }
+    return note_cuda(cudaGetLastError());
+}
+
 }  // namespace
 }  // namespace la
 
@@ -415,6 +487,21 @@ int la_device_sm_count(void) {
     int dev = 0, sms = 0;
     if (device_setup(&dev, &sms) != LA_OK) return 0;
     return sms;
+}
+
+int la_prefill_noalloc(const void* q, const void* k, const void* v, void* o, float* state_out,
+                       int B, int H, int N, int d, int blk, la_dtype dt, void* stream) {
+    if (B < 1 || H < 1 || N < 1) return LA_ERR_INVALID_ARG;
+    int st = validate_common(q, k, v, o, d, blk, dt);
+    if (st != LA_OK) return st;
+    if (dt != LA_BF16) return LA_ERR_UNSUPPORTED;
+    if (state_out && !aligned16(state_out)) return LA_ERR_INVALID_ARG;
+    if ((long long)B * H > (1ll << 30) || (long long)N > (1ll << 30)) return LA_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    st = device_setup(&dev, &sms);
+    if (st != LA_OK) return st;
+    return launch_prefill_bf16_noalloc(q, k, v, o, state_out, B * H, N, blk,
+                                       reinterpret_cast<cudaStream_t>(stream), dev, sms);
 }
 
 int la_timing_enable(int max_launches) {
