@@ -390,6 +390,28 @@ def bench_secondary(args, device, stream, peaks):
         "kernels": {k_: round(v_["total_ms"] / max(v_["launches"], 1), 4) for k_, v_ in kt.items()}}
     del q, k, v, o, st
     torch.cuda.empty_cache()
+
+    # -- packed variable-length prefill: 2^20 tokens, lengths U[1024, 65536], H=64
+    Tv, Hv = 1 << 20, 64
+    lens = inputs.varlen_lengths(Tv, 1024, 65536, seed=0)
+    cu = torch.from_numpy(inputs.cu_seqlens_from_lengths(lens)).to(device)
+    q, k, v = inputs.qkv((Hv, Tv, D), dtype=torch.bfloat16, device=device, seed=0)
+    o = torch.empty_like(q)
+    st = torch.empty((len(lens), Hv, D, D), dtype=torch.float32, device=device)
+    la.la_timing_enable(64)
+    ms = timed(stream, lambda: la.prefill_varlen(q, k, v, cu, blk=BLK, out=o, state_out=st), 3, 2,
+               solo, device)
+    kt = kernel_times(la)
+    la.la_timing_enable(0)
+    bytes_step = Hv * Tv * BYTES_PER_TOKEN_HEAD
+    out["varlen_prefill"] = {
+        "workload": f"packed prefill bf16 T=2^20 ({len(lens)} sequences, lengths U[1024,65536] "
+                    "seed 0), H=64, d=128, blk=128",
+        "tokens_per_s": round(Tv / (ms / 3 / 1e3), 1), "ms_per_step": round(ms / 3, 4),
+        "hbm_frac": round(bytes_step / (ms / 3 / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+        "kernels": {k_: round(v_["total_ms"] / max(v_["launches"], 1), 4) for k_, v_ in kt.items()}}
+    del q, k, v, o, st
+    torch.cuda.empty_cache()
     return out
 
 

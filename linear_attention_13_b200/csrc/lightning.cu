@@ -186,6 +186,40 @@ int choose_chunk_tokens(int BH, int N, int ctas) {
     return best_blocks * kTileRows;
 }
 
+tc::Params dense_params(int BH, int N, int chunk_tokens, void* o) {
+    tc::Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.mode = tc::kModeDense;
+    p.Z = BH;
+    p.rows = N;
+    p.chunk_tokens = chunk_tokens;
+    p.n_chunks = (N + chunk_tokens - 1) / chunk_tokens;
+    p.n_items = BH * p.n_chunks;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    return p;
+}
+
+// chunk states -> scan -> outputs, with the chunk states in `ws`
+void launch_three_pass(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       tc::Params p, float* ws, float* state_out, int grid, cudaStream_t stream) {
+    p.chunk_delta = ws;
+    {
+        TimedLaunch tl(LA_KERNEL_CHUNK_STATE, stream);
+        tc::chunk_state_kernel<<<grid, tc::cs::kThreads, tc::cs::kSmemBytes, stream>>>(tk, tv, p);
+    }
+    {
+        TimedLaunch tl(LA_KERNEL_CHUNK_SCAN, stream);
+        dim3 sgrid(kHeadDim * kHeadDim / 4 / 256, p.Z);
+        tc::chunk_scan_kernel<<<sgrid, 256, 0, stream>>>(ws, state_out, p.n_chunks);
+    }
+    p.prefix = ws;
+    p.state_out = nullptr;
+    {
+        TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
+        tc::prefill_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(tq, tk, tv, p);
+    }
+}
+
 int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, float* state_out,
                         int BH, int N, int blk, cudaStream_t stream, int sms, int chunk_tokens) {
     if (blk != 128) return LA_ERR_UNSUPPORTED;
@@ -195,21 +229,10 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
         return LA_ERR_CUDA;
     if (chunk_tokens <= 0) chunk_tokens = choose_chunk_tokens(BH, N, sms);
     chunk_tokens = ((chunk_tokens + kTileRows - 1) / kTileRows) * kTileRows;
-    const int n_chunks = (N + chunk_tokens - 1) / chunk_tokens;
-
-    tc::DenseParams p;
-    p.BH = BH;
-    p.N = N;
-    p.chunk_tokens = chunk_tokens;
-    p.n_chunks = n_chunks;
-    p.n_items = BH * n_chunks;
-    p.o = reinterpret_cast<__nv_bfloat16*>(o);
-    p.prefix = nullptr;
-    p.state_out = nullptr;
-    p.chunk_delta = nullptr;
+    tc::Params p = dense_params(BH, N, chunk_tokens, o);
     const int grid = std::min(p.n_items, sms);
 
-    if (n_chunks == 1) {
+    if (p.n_chunks == 1) {
         p.state_out = state_out;
         {
             TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
@@ -218,29 +241,83 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
         return note_cuda(cudaGetLastError());
     }
     float* ws = nullptr;
-    const size_t ws_bytes = (size_t)BH * n_chunks * kHeadDim * kHeadDim * sizeof(float);
+    const size_t ws_bytes = (size_t)BH * p.n_chunks * kHeadDim * kHeadDim * sizeof(float);
     if (cudaMallocAsync(reinterpret_cast<void**>(&ws), ws_bytes, stream) != cudaSuccess) {
         cudaGetLastError();
         return LA_ERR_ALLOC;
     }
+    launch_three_pass(tq, tk, tv, p, ws, state_out, grid, stream);
+    int st = note_cuda(cudaGetLastError());
+    cudaFreeAsync(ws, stream);
+    return st;
+}
+
+// Chunk length for packed sequences: long enough to keep the chunk-state
+// traffic small, short enough for about eight rounds of work items.
+int choose_varlen_chunk_tokens(int H, int T, int ctas) {
+    long target = ((long)H * T) / (8L * ctas);
+    target = std::max(1024L, std::min(16384L, target));
+    return (int)(((target + kTileRows - 1) / kTileRows) * kTileRows);
+}
+
+int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void* o,
+                               float* state_out, const int32_t* cu_seqlens, int num_seqs, int T,
+                               int H, int blk, cudaStream_t stream, int sms) {
+    if (blk != 128) return LA_ERR_UNSUPPORTED;
+    const int chunk_tokens = choose_varlen_chunk_tokens(H, std::max(T, 1), sms);
+    const long max_chunks = (long)(T + chunk_tokens - 1) / chunk_tokens + num_seqs;
+    if ((long)H * max_chunks > (1L << 30)) return LA_ERR_UNSUPPORTED;
+    CUtensorMap tq, tk, tv;
+    const int rows = std::max(T, 1);
+    if (make_tmap_bf16(&tq, q, rows, H) || make_tmap_bf16(&tk, k, rows, H) ||
+        make_tmap_bf16(&tv, v, rows, H))
+        return LA_ERR_CUDA;
+    const size_t aux_bytes = ((size_t)(num_seqs + 2) * sizeof(int32_t) + 255) / 256 * 256;
+    const size_t ws_bytes = (size_t)H * max_chunks * kHeadDim * kHeadDim * sizeof(float);
+    uint8_t* buf = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&buf), aux_bytes + ws_bytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_ALLOC;
+    }
+    int* ok = reinterpret_cast<int*>(buf);
+    int32_t* chunk_off = reinterpret_cast<int32_t*>(buf) + 1;
+    float* ws = reinterpret_cast<float*>(buf + aux_bytes);
+    {
+        TimedLaunch tl(LA_KERNEL_AUX, stream);
+        tc::varlen_prepare_kernel<<<1, 256, 0, stream>>>(cu_seqlens, num_seqs, T, chunk_tokens, ok,
+                                                        chunk_off);
+    }
+    tc::Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.mode = tc::kModeVarlen;
+    p.Z = H;
+    p.rows = rows;
+    p.chunk_tokens = chunk_tokens;
+    p.n_items = (int)std::min<long>((long)H * max_chunks, 1L << 30);
+    p.cu_seqlens = cu_seqlens;
+    p.chunk_off = chunk_off;
+    p.seq_ok = ok;
+    p.num_seqs = num_seqs;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
     p.chunk_delta = ws;
+    const int grid = (int)std::min<long>(p.n_items, sms);
     {
         TimedLaunch tl(LA_KERNEL_CHUNK_STATE, stream);
-        tc::chunk_state_kernel<<<grid, tc::kThreads, tc::cs::kSmemBytes, stream>>>(tk, tv, p);
+        tc::chunk_state_kernel<<<grid, tc::cs::kThreads, tc::cs::kSmemBytes, stream>>>(tk, tv, p);
     }
     {
         TimedLaunch tl(LA_KERNEL_CHUNK_SCAN, stream);
-        dim3 sgrid(kHeadDim * kHeadDim / 4 / 256, BH);
-        tc::chunk_scan_kernel<<<sgrid, 256, 0, stream>>>(ws, state_out, n_chunks);
+        dim3 sgrid(num_seqs, H);
+        tc::chunk_scan_varlen_kernel<<<sgrid, 256, 0, stream>>>(ws, state_out, chunk_off, ok, H,
+                                                               num_seqs);
     }
     p.prefix = ws;
-    p.state_out = nullptr;
     {
         TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
         tc::prefill_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(tq, tk, tv, p);
     }
-    int st = note_cuda(cudaGetLastError());
-    cudaFreeAsync(ws, stream);
+    const int st = note_cuda(cudaGetLastError());
+    cudaFreeAsync(buf, stream);
     return st;
 }
 
@@ -297,30 +374,12 @@ int launch_prefill_bf16_noalloc(const void* q, const void* k, const void* v, voi
     if (make_tmap_bf16(&tq, q, N, BH) || make_tmap_bf16(&tk, k, N, BH) ||
         make_tmap_bf16(&tv, v, N, BH))
         return LA_ERR_CUDA;
-    tc::DenseParams p;
-    p.BH = BH;
-    p.N = N;
-    p.chunk_tokens = chunk_tokens;
-    p.n_chunks = n_chunks;
-    p.n_items = BH * n_chunks;
-    p.o = reinterpret_cast<__nv_bfloat16*>(o);
-    p.prefix = nullptr;
-    p.state_out = n_chunks == 1 ? state_out : nullptr;
-    p.chunk_delta = ws;
+    tc::Params p = dense_params(BH, N, chunk_tokens, o);
     const int grid = std::min(p.n_items, sms);
     if (n_chunks > 1) {
-        {
-            TimedLaunch tl(LA_KERNEL_CHUNK_STATE, stream);
-            tc::chunk_state_kernel<<<grid, tc::kThreads, tc::cs::kSmemBytes, stream>>>(tk, tv, p);
-        }
-        {
-            TimedLaunch tl(LA_KERNEL_CHUNK_SCAN, stream);
-            dim3 sgrid(kHeadDim * kHeadDim / 4 / 256, BH);
-            tc::chunk_scan_kernel<<<sgrid, 256, 0, stream>>>(ws, state_out, n_chunks);
-        }
-        p.prefix = ws;
-    }
-    {
+        launch_three_pass(tq, tk, tv, p, ws, state_out, grid, stream);
+    } else {
+        p.state_out = state_out;
         TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
         tc::prefill_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(tq, tk, tv, p);
     }
@@ -382,7 +441,9 @@ int la_prefill_varlen(const void* q, const void* k, const void* v, void* o, floa
     st = device_setup(&dev, &sms);
     if (st != LA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (dt != LA_F32) return LA_ERR_UNSUPPORTED;
+    if (dt == LA_BF16)
+        return launch_prefill_varlen_bf16(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens,
+                                          H, blk, s, sms);
     int* ok = nullptr;
     if (cudaMallocAsync(reinterpret_cast<void**>(&ok), sizeof(int), s) != cudaSuccess) {
         cudaGetLastError();

@@ -42,3 +42,69 @@ def test_bad_seqlens_detected_on_device(bad):
     assert la.la_get_last_error() == la.LA_ERR_BAD_SEQLENS
     assert torch.all(o == 3.0) and torch.all(st == 3.0)
     assert la.la_get_last_error() == la.LA_OK   # cleared after reading
+
+
+# ---------------------------------------------------------------- bf16 tensor-core path
+from _util import TOL_O_BF16, round_like  # noqa: E402
+
+
+@pytest.mark.parametrize("lens", [
+    [5, 0, 130, 1, 64, 257],
+    [128, 127, 129, 1, 0, 0, 1000],
+    [3000, 1, 2049, 5000],
+])
+def test_varlen_bf16(lens):
+    cu = _cu(lens)
+    H, T = 3, sum(lens)
+    q, k, v = inputs.qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=len(lens))
+    o = torch.full_like(q, 5.0)
+    o, st = la.prefill_varlen(q, k, v, cu, blk=128, out=o)
+    assert la.la_get_last_error() == la.LA_OK
+    o_ref, s_ref = oracle.prefill_varlen(host64(q), host64(k), host64(v), cu.cpu().numpy())
+    assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16
+    assert per_head_rel_err(host64(st), s_ref) <= TOL_STATE
+    for j, n in enumerate(lens):
+        if n == 0:
+            assert not torch.any(st[j])
+
+
+def test_varlen_bf16_onehot_bit_exact():
+    # one-hot keys keep all intermediates small integers: the packed path,
+    # including sequences longer than one chunk and ragged tails, is exact.
+    lens = [2500, 1, 4097, 0, 1300, 128, 9000]
+    cu = _cu(lens)
+    H, T = 2, sum(lens)
+    q, k, v = inputs.onehot_k_qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=21)
+    o, st = la.prefill_varlen(q, k, v, cu, blk=128)
+    assert la.la_get_last_error() == la.LA_OK
+    o_ref, s_ref = oracle.prefill_varlen(host64(q), host64(k), host64(v), cu.cpu().numpy())
+    assert np.array_equal(host64(o), round_like(o_ref, torch.bfloat16))
+    assert np.array_equal(host64(st), s_ref)
+
+
+def test_varlen_bf16_bad_seqlens_detected():
+    H, T = 2, 300
+    q, k, v = inputs.qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=1)
+    cu = torch.tensor([0, 200, 100, 300], dtype=torch.int32, device=DEV)
+    o = torch.full_like(q, 3.0)
+    st = torch.full((3, H, 128, 128), 3.0, device=DEV)
+    la.prefill_varlen(q, k, v, cu, blk=128, out=o, state_out=st)
+    assert la.la_get_last_error() == la.LA_ERR_BAD_SEQLENS
+    assert torch.all(o == 3.0) and torch.all(st == 3.0)
+
+
+def test_varlen_bf16_packed_config_sampled_heads():
+    # 2^20 packed tokens, lengths uniform in [1024, 65536] (seeded, last
+    # trimmed), H = 64, d = 128: every sequence of 8 sampled heads.
+    T, H = 1 << 20, 64
+    lens = inputs.varlen_lengths(T, 1024, 65536, seed=0)
+    cu = _cu(lens)
+    q, k, v = inputs.qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=0)
+    o, st = la.prefill_varlen(q, k, v, cu, blk=128)
+    assert la.la_get_last_error() == la.LA_OK
+    rng = np.random.default_rng(0)
+    heads = [0, H - 1] + sorted(rng.choice(np.arange(1, H - 1), 6, replace=False).tolist())
+    hq, hk, hv = (host64(x[heads]) for x in (q, k, v))
+    o_ref, s_ref = oracle.prefill_varlen(hq, hk, hv, cu.cpu().numpy())
+    assert per_head_rel_err(host64(o[heads]), o_ref) <= TOL_O_BF16
+    assert per_head_rel_err(host64(st[:, heads]), s_ref) <= TOL_STATE
