@@ -80,7 +80,12 @@ int la_prefill(const void* q, const void* k, const void* v, void* o, float* stat
  *   flags       : LA_FLAG_* bits below; 0 = default schedule.
  */
 #define LA_FLAG_THREE_PASS 1   /* chunk states, scan, then outputs (3 launches) */
-#define LA_FLAG_FUSED      2   /* single persistent launch with look-back      */
+#define LA_FLAG_FUSED      2   /* single persistent launch with look-back (the
+                                  default): each chunk publishes its inclusive
+                                  state prefix for the next one              */
+#define LA_FLAG_SPLIT_V    4   /* split the value columns of every head over two
+                                  CTAs (independent halves of S and O)        */
+#define LA_FLAG_NO_SPLIT_V 8   /* never split the value columns               */
 int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* state_out,
                   int B, int H, int N, int d, int blk, la_dtype dt, void* stream,
                   int chunk_tokens, int flags);
@@ -101,6 +106,16 @@ int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* s
 int la_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* state_out,
                       const int32_t* cu_seqlens, int num_seqs, int total_tokens,
                       int H, int d, int blk, la_dtype dt, void* stream);
+
+/*
+ * la_prefill_varlen_ex -- la_prefill_varlen with the scheduling controls of
+ * la_prefill_ex (chunk_tokens: chunk length, a multiple of 128, 0 = library
+ * choice; flags: LA_FLAG_THREE_PASS or LA_FLAG_FUSED, 0 = default).
+ */
+int la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o, float* state_out,
+                         const int32_t* cu_seqlens, int num_seqs, int total_tokens,
+                         int H, int d, int blk, la_dtype dt, void* stream,
+                         int chunk_tokens, int flags);
 
 /*
  * la_decode_step -- one token per sequence (prefill and decode are separate,

@@ -34,6 +34,8 @@ LA_BF16 = 1
 
 LA_FLAG_THREE_PASS = 1
 LA_FLAG_FUSED = 2
+LA_FLAG_SPLIT_V = 4
+LA_FLAG_NO_SPLIT_V = 8
 
 LA_KERNEL_PREFILL_TC = 0
 LA_KERNEL_CHUNK_STATE = 1
@@ -45,7 +47,8 @@ LA_NUM_KERNEL_IDS = 6
 
 EXPORTED = ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step",
             "la_status_string", "la_get_last_error", "la_device_sm_count",
-            "la_timing_enable", "la_timing_read", "la_kernel_name", "la_prefill_noalloc")
+            "la_timing_enable", "la_timing_read", "la_kernel_name", "la_prefill_noalloc",
+            "la_prefill_varlen_ex")
 
 LA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -72,6 +75,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la_prefill.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.la_prefill_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
     lib.la_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+    lib.la_prefill_varlen_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
     lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, vp]
     lib.la_status_string.argtypes = [i]
     lib.la_status_string.restype = ctypes.c_char_p
@@ -82,7 +86,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.la_kernel_name.argtypes = [i]
     lib.la_kernel_name.restype = ctypes.c_char_p
-    for name in ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step",
+    for name in ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_prefill_varlen_ex",
+                 "la_decode_step",
                  "la_get_last_error", "la_device_sm_count", "la_timing_enable",
                  "la_timing_read", "la_prefill_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
@@ -114,6 +119,13 @@ def la_prefill_varlen(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens,
 def la_prefill_noalloc(q, k, v, o, state_out, B, H, N, d, blk, dt, stream):
     """la_prefill that allocates no device memory (fixed in-library scratch)."""
     return load_library().la_prefill_noalloc(q, k, v, o, state_out, B, H, N, d, blk, dt, stream)
+
+
+def la_prefill_varlen_ex(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens, H, d, blk,
+                         dt, stream, chunk_tokens, flags):
+    return load_library().la_prefill_varlen_ex(q, k, v, o, state_out, cu_seqlens, num_seqs,
+                                               total_tokens, H, d, blk, dt, stream, chunk_tokens,
+                                               flags)
 
 
 def la_decode_step(q, k, v, state, o, B, H, d, dt, stream):
@@ -202,7 +214,7 @@ def prefill(q, k, v, blk: int = 128, want_state: bool = True, chunk_tokens: int 
 
 
 def prefill_varlen(q, k, v, cu_seqlens, blk: int = 128, want_state: bool = True, out=None,
-                   state_out=None, stream=None):
+                   state_out=None, stream=None, chunk_tokens: int = 0, flags: int = 0):
     """Packed prefill of [H,T,d] tensors split by int32 device cu_seqlens.
 
     Returns (o, state [num_seqs,H,d,d])."""
@@ -217,9 +229,10 @@ def prefill_varlen(q, k, v, cu_seqlens, blk: int = 128, want_state: bool = True,
     st = state_out
     if st is None and want_state:
         st = torch.empty((S, H, d, d), dtype=torch.float32, device=q.device)
-    status = la_prefill_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                               st.data_ptr() if st is not None else None, cu_seqlens.data_ptr(), S,
-                               T, H, d, blk, _dtype_code(q), _stream_ptr(stream))
+    status = la_prefill_varlen_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                  st.data_ptr() if st is not None else None, cu_seqlens.data_ptr(),
+                                  S, T, H, d, blk, _dtype_code(q), _stream_ptr(stream),
+                                  chunk_tokens, flags)
     _raise(status, "la_prefill_varlen")
     return o, st
 

@@ -57,8 +57,12 @@ int device_setup(int* dev_out, int* sms_out) {
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return LA_ERR_CUDA;
-        if (cudaFuncSetAttribute(tc::prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tc::kSmemBytes) != cudaSuccess ||
+        if (cudaFuncSetAttribute(tc::prefill_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::smem_bytes(128)) != cudaSuccess ||
+            cudaFuncSetAttribute(tc::prefill_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::smem_bytes(64)) != cudaSuccess ||
+            cudaFuncSetAttribute(tc::prefill_seq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::sq::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(tc::chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tc::cs::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(simt::prefill_simt_kernel<64>,
@@ -186,6 +190,19 @@ int choose_chunk_tokens(int BH, int N, int ctas) {
     return best_blocks * kTileRows;
 }
 
+// Main kernel for p.vparts value parts per head (1: 128 columns per CTA, 2: 64).
+// Split value columns without a look-back chain run the sequential kernel
+// with the fully double-buffered block pipeline.
+void launch_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                 const CUtensorMap& to, const tc::Params& p, int grid, cudaStream_t stream) {
+    if (p.vparts == 2 && !p.fused)
+        tc::prefill_seq_kernel<<<grid, tc::sq::kThreads, tc::sq::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+    else if (p.vparts == 2)
+        tc::prefill_tc_kernel<64><<<grid, tc::kThreads, tc::smem_bytes(64), stream>>>(tq, tk, tv, to, p);
+    else
+        tc::prefill_tc_kernel<128><<<grid, tc::kThreads, tc::smem_bytes(128), stream>>>(tq, tk, tv, to, p);
+}
+
 tc::Params dense_params(int BH, int N, int chunk_tokens, void* o) {
     tc::Params p;
     std::memset(&p, 0, sizeof(p));
@@ -196,16 +213,32 @@ tc::Params dense_params(int BH, int N, int chunk_tokens, void* o) {
     p.n_chunks = (N + chunk_tokens - 1) / chunk_tokens;
     p.n_items = BH * p.n_chunks;
     p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.vparts = 1;
     return p;
+}
+
+// Split the value columns of every head over two CTAs when the heads alone
+// would leave many SMs idle and the sequences are short enough that one CTA
+// per (head, half) finishes in time (measured on B200: at 64 heads the split
+// wins at 8K tokens and loses to chunking at 256K).
+bool want_split_v(long slices, long N, int sms, int flags) {
+    if (flags & LA_FLAG_NO_SPLIT_V) return false;
+    if (flags & LA_FLAG_SPLIT_V) return true;
+    return slices * 4 < (long)sms * 3 && N <= 16384;
 }
 
 // chunk states -> scan -> outputs, with the chunk states in `ws`
 void launch_three_pass(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       tc::Params p, float* ws, float* state_out, int grid, cudaStream_t stream) {
+                       const CUtensorMap& to, tc::Params p, float* ws, float* state_out, int grid, cudaStream_t stream) {
     p.chunk_delta = ws;
     {
+        // chunk states are computed once per chunk over all value columns
+        tc::Params pc = p;
+        pc.vparts = 1;
+        pc.n_items = p.Z * p.n_chunks;
         TimedLaunch tl(LA_KERNEL_CHUNK_STATE, stream);
-        tc::chunk_state_kernel<<<grid, tc::cs::kThreads, tc::cs::kSmemBytes, stream>>>(tk, tv, p);
+        tc::chunk_state_kernel<<<std::min(grid, pc.n_items), tc::cs::kThreads, tc::cs::kSmemBytes,
+                                 stream>>>(tk, tv, pc);
     }
     {
         TimedLaunch tl(LA_KERNEL_CHUNK_SCAN, stream);
@@ -216,27 +249,97 @@ void launch_three_pass(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     p.state_out = nullptr;
     {
         TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
-        tc::prefill_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(tq, tk, tv, p);
+        launch_main(tq, tk, tv, to, p, grid, stream);
     }
 }
 
+// Chunk length for the single-pass schedule: minimise rounds of work items
+// times (blocks per chunk + a per-chunk overhead of about two blocks), with
+// chunks of at least 512 tokens.
+int choose_fused_chunk_tokens(int Z, int N, int ctas) {
+    const int nblk = (N + kTileRows - 1) / kTileRows;
+    int best = nblk;
+    double best_cost = 1e300;
+    for (int cb = nblk; cb >= std::min(4, nblk); --cb) {
+        const int nch = (nblk + cb - 1) / cb;
+        if (nch > 1 && cb * (nch - 1) >= nblk) continue;
+        const long rounds = ((long)Z * nch + ctas - 1) / ctas;
+        const double cost = (double)rounds * (cb + (nch > 1 ? 2.0 : 0.5));
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = cb;
+        }
+    }
+    return best * kTileRows;
+}
+
+// Single pass with look-back: one launch (plus a memset of the chunk flags).
+int launch_fused(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                 const CUtensorMap& to, tc::Params p,
+                 long n_chunk_slots, float* state_out, int grid, cudaStream_t stream) {
+    p.state_out = state_out;
+    if (n_chunk_slots > 0) {
+        const size_t chain_bytes = (size_t)n_chunk_slots * kHeadDim * kHeadDim * sizeof(float);
+        const size_t flag_words = (size_t)n_chunk_slots * p.vparts * tc::kChainWarps;
+        const size_t flag_bytes = (flag_words * sizeof(int) + 255) / 256 * 256;
+        uint8_t* buf = nullptr;
+        if (cudaMallocAsync(reinterpret_cast<void**>(&buf), chain_bytes + flag_bytes, stream) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return LA_ERR_ALLOC;
+        }
+        p.flags = reinterpret_cast<int*>(buf);
+        p.chain = reinterpret_cast<float*>(buf + flag_bytes);
+        p.fused = 1;
+        cudaMemsetAsync(p.flags, 0, flag_words * sizeof(int), stream);
+        {
+            TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
+            launch_main(tq, tk, tv, to, p, grid, stream);
+        }
+        const int st = note_cuda(cudaGetLastError());
+        cudaFreeAsync(buf, stream);
+        return st;
+    }
+    p.fused = 0;
+    {
+        TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
+        launch_main(tq, tk, tv, to, p, grid, stream);
+    }
+    return note_cuda(cudaGetLastError());
+}
+
 int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, float* state_out,
-                        int BH, int N, int blk, cudaStream_t stream, int sms, int chunk_tokens) {
+                        int BH, int N, int blk, cudaStream_t stream, int sms, int chunk_tokens,
+                        int flags) {
     if (blk != 128) return LA_ERR_UNSUPPORTED;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (make_tmap_bf16(&tq, q, N, BH) || make_tmap_bf16(&tk, k, N, BH) ||
-        make_tmap_bf16(&tv, v, N, BH))
+        make_tmap_bf16(&tv, v, N, BH) || make_tmap_bf16(&to, o, N, BH))
         return LA_ERR_CUDA;
-    if (chunk_tokens <= 0) chunk_tokens = choose_chunk_tokens(BH, N, sms);
+    const bool three_pass = (flags & LA_FLAG_THREE_PASS) != 0;
+    const int vparts = want_split_v(BH, N, sms, flags) ? 2 : 1;
+    if (!three_pass) {
+        if (chunk_tokens <= 0) chunk_tokens = choose_fused_chunk_tokens(BH * vparts, N, sms);
+        chunk_tokens = ((chunk_tokens + kTileRows - 1) / kTileRows) * kTileRows;
+        tc::Params p = dense_params(BH, N, chunk_tokens, o);
+        p.vparts = vparts;
+        p.n_items *= vparts;
+        const int grid = std::min(p.n_items, sms);
+        return launch_fused(tq, tk, tv, to, p, p.n_chunks > 1 ? (long)BH * p.n_chunks : 0, state_out,
+                            grid, stream);
+    }
+    if (chunk_tokens <= 0) chunk_tokens = choose_chunk_tokens(BH * vparts, N, sms);
     chunk_tokens = ((chunk_tokens + kTileRows - 1) / kTileRows) * kTileRows;
     tc::Params p = dense_params(BH, N, chunk_tokens, o);
+    p.vparts = vparts;
+    p.n_items *= vparts;
     const int grid = std::min(p.n_items, sms);
 
     if (p.n_chunks == 1) {
         p.state_out = state_out;
         {
             TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
-            tc::prefill_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(tq, tk, tv, p);
+            launch_main(tq, tk, tv, to, p, grid, stream);
         }
         return note_cuda(cudaGetLastError());
     }
@@ -246,10 +349,20 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
         cudaGetLastError();
         return LA_ERR_ALLOC;
     }
-    launch_three_pass(tq, tk, tv, p, ws, state_out, grid, stream);
+    launch_three_pass(tq, tk, tv, to, p, ws, state_out, grid, stream);
     int st = note_cuda(cudaGetLastError());
     cudaFreeAsync(ws, stream);
     return st;
+}
+
+// Single pass over packed sequences: chunks of 8192 tokens (best of the
+// measured 1K-8K range on B200 for 2^20 tokens x 64 heads: fewer look-back
+// links outweigh the lost L2 reuse).
+int choose_varlen_fused_chunk_tokens(int H, int T, int ctas) {
+    (void)H;
+    (void)T;
+    (void)ctas;
+    return 8192;
 }
 
 // Chunk length for packed sequences: long enough to keep the chunk-state
@@ -262,20 +375,26 @@ int choose_varlen_chunk_tokens(int H, int T, int ctas) {
 
 int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void* o,
                                float* state_out, const int32_t* cu_seqlens, int num_seqs, int T,
-                               int H, int blk, cudaStream_t stream, int sms) {
+                               int H, int blk, cudaStream_t stream, int sms, bool three_pass,
+                               int chunk_tokens) {
     if (blk != 128) return LA_ERR_UNSUPPORTED;
-    const int chunk_tokens = choose_varlen_chunk_tokens(H, std::max(T, 1), sms);
+    if (chunk_tokens <= 0)
+        chunk_tokens = three_pass ? choose_varlen_chunk_tokens(H, std::max(T, 1), sms)
+                                  : choose_varlen_fused_chunk_tokens(H, std::max(T, 1), sms);
+    chunk_tokens = ((chunk_tokens + kTileRows - 1) / kTileRows) * kTileRows;
     const long max_chunks = (long)(T + chunk_tokens - 1) / chunk_tokens + num_seqs;
     if ((long)H * max_chunks > (1L << 30)) return LA_ERR_UNSUPPORTED;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     const int rows = std::max(T, 1);
     if (make_tmap_bf16(&tq, q, rows, H) || make_tmap_bf16(&tk, k, rows, H) ||
-        make_tmap_bf16(&tv, v, rows, H))
+        make_tmap_bf16(&tv, v, rows, H) || make_tmap_bf16(&to, o, rows, H))
         return LA_ERR_CUDA;
     const size_t aux_bytes = ((size_t)(num_seqs + 2) * sizeof(int32_t) + 255) / 256 * 256;
     const size_t ws_bytes = (size_t)H * max_chunks * kHeadDim * kHeadDim * sizeof(float);
+    const size_t flag_bytes = three_pass ? 0 : (size_t)H * max_chunks * tc::kChainWarps * sizeof(int);
     uint8_t* buf = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void**>(&buf), aux_bytes + ws_bytes, stream) != cudaSuccess) {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&buf), aux_bytes + ws_bytes + flag_bytes, stream) !=
+        cudaSuccess) {
         cudaGetLastError();
         return LA_ERR_ALLOC;
     }
@@ -290,6 +409,7 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
     tc::Params p;
     std::memset(&p, 0, sizeof(p));
     p.mode = tc::kModeVarlen;
+    p.vparts = 1;
     p.Z = H;
     p.rows = rows;
     p.chunk_tokens = chunk_tokens;
@@ -299,8 +419,29 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
     p.seq_ok = ok;
     p.num_seqs = num_seqs;
     p.o = reinterpret_cast<__nv_bfloat16*>(o);
-    p.chunk_delta = ws;
     const int grid = (int)std::min<long>(p.n_items, sms);
+    if (!three_pass) {
+        // single pass: chunk prefixes in `ws`, flags after cu_seqlens bookkeeping
+        int* chunk_flags = reinterpret_cast<int*>(buf + aux_bytes + ws_bytes);
+        cudaMemsetAsync(chunk_flags, 0, flag_bytes, stream);
+        if (state_out != nullptr) {
+            TimedLaunch tl(LA_KERNEL_AUX, stream);
+            tc::zero_empty_states_kernel<<<dim3(num_seqs, H), 256, 0, stream>>>(state_out, cu_seqlens,
+                                                                              ok, H);
+        }
+        p.fused = 1;
+        p.chain = ws;
+        p.flags = chunk_flags;
+        p.state_out = state_out;
+        {
+            TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
+            launch_main(tq, tk, tv, to, p, grid, stream);
+        }
+        const int st = note_cuda(cudaGetLastError());
+        cudaFreeAsync(buf, stream);
+        return st;
+    }
+    p.chunk_delta = ws;
     {
         TimedLaunch tl(LA_KERNEL_CHUNK_STATE, stream);
         tc::chunk_state_kernel<<<grid, tc::cs::kThreads, tc::cs::kSmemBytes, stream>>>(tk, tv, p);
@@ -314,7 +455,7 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
     p.prefix = ws;
     {
         TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
-        tc::prefill_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(tq, tk, tv, p);
+        launch_main(tq, tk, tv, to, p, grid, stream);
     }
     const int st = note_cuda(cudaGetLastError());
     cudaFreeAsync(buf, stream);
@@ -370,18 +511,18 @@ int launch_prefill_bf16_noalloc(const void* q, const void* k, const void* v, voi
         const int st = noalloc_scratch(dev, &ws);
         if (st != LA_OK) return st;
     }
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (make_tmap_bf16(&tq, q, N, BH) || make_tmap_bf16(&tk, k, N, BH) ||
-        make_tmap_bf16(&tv, v, N, BH))
+        make_tmap_bf16(&tv, v, N, BH) || make_tmap_bf16(&to, o, N, BH))
         return LA_ERR_CUDA;
     tc::Params p = dense_params(BH, N, chunk_tokens, o);
     const int grid = std::min(p.n_items, sms);
     if (n_chunks > 1) {
-        launch_three_pass(tq, tk, tv, p, ws, state_out, grid, stream);
+        launch_three_pass(tq, tk, tv, to, p, ws, state_out, grid, stream);
     } else {
         p.state_out = state_out;
         TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
-        tc::prefill_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(tq, tk, tv, p);
+        launch_main(tq, tk, tv, to, p, grid, stream);
     }
     return note_cuda(cudaGetLastError());
 }
@@ -396,8 +537,12 @@ extern "C" {
 int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* state_out, int B,
                   int H, int N, int d, int blk, la_dtype dt, void* stream, int chunk_tokens,
                   int flags) {
-    (void)flags;
     if (B < 1 || H < 1 || N < 1) return LA_ERR_INVALID_ARG;
+    constexpr int kAllFlags = LA_FLAG_THREE_PASS | LA_FLAG_FUSED | LA_FLAG_SPLIT_V | LA_FLAG_NO_SPLIT_V;
+    if ((flags & ~kAllFlags) != 0 ||
+        (flags & (LA_FLAG_THREE_PASS | LA_FLAG_FUSED)) == (LA_FLAG_THREE_PASS | LA_FLAG_FUSED) ||
+        (flags & (LA_FLAG_SPLIT_V | LA_FLAG_NO_SPLIT_V)) == (LA_FLAG_SPLIT_V | LA_FLAG_NO_SPLIT_V))
+        return LA_ERR_INVALID_ARG;
     int st = validate_common(q, k, v, o, d, blk, dt);
     if (st != LA_OK) return st;
     if (state_out && !aligned16(state_out)) return LA_ERR_INVALID_ARG;
@@ -421,7 +566,7 @@ int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* s
                 qf, kf, vf, of, state_out, N, blk);
         return note_cuda(cudaGetLastError());
     }
-    return launch_prefill_bf16(q, k, v, o, state_out, BH, N, blk, s, sms, chunk_tokens);
+    return launch_prefill_bf16(q, k, v, o, state_out, BH, N, blk, s, sms, chunk_tokens, flags);
 }
 
 int la_prefill(const void* q, const void* k, const void* v, void* o, float* state_out, int B, int H,
@@ -432,6 +577,16 @@ int la_prefill(const void* q, const void* k, const void* v, void* o, float* stat
 int la_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* state_out,
                       const int32_t* cu_seqlens, int num_seqs, int total_tokens, int H, int d,
                       int blk, la_dtype dt, void* stream) {
+    return la_prefill_varlen_ex(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens, H, d,
+                                blk, dt, stream, 0, 0);
+}
+
+int la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o, float* state_out,
+                         const int32_t* cu_seqlens, int num_seqs, int total_tokens, int H, int d,
+                         int blk, la_dtype dt, void* stream, int chunk_tokens, int flags) {
+    if ((flags & ~(LA_FLAG_THREE_PASS | LA_FLAG_FUSED)) != 0 ||
+        flags == (LA_FLAG_THREE_PASS | LA_FLAG_FUSED) || chunk_tokens < 0)
+        return LA_ERR_INVALID_ARG;
     if (num_seqs < 1 || total_tokens < 0 || H < 1 || cu_seqlens == nullptr) return LA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return LA_ERR_INVALID_ARG;
     int st = validate_common(q, k, v, o, d, blk, dt);
@@ -443,7 +598,8 @@ int la_prefill_varlen(const void* q, const void* k, const void* v, void* o, floa
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (dt == LA_BF16)
         return launch_prefill_varlen_bf16(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens,
-                                          H, blk, s, sms);
+                                          H, blk, s, sms, (flags & LA_FLAG_THREE_PASS) != 0,
+                                          chunk_tokens);
     int* ok = nullptr;
     if (cudaMallocAsync(reinterpret_cast<void**>(&ok), sizeof(int), s) != cudaSuccess) {
         cudaGetLastError();

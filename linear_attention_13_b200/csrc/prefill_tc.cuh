@@ -39,21 +39,38 @@ namespace la {
 namespace tc {
 
 // ---------------------------------------------------------------- geometry
+// Shared memory of the main kernel for a CTA handling kNV value columns: two
+// stages of Q, K (128 x 128) and V (128 x kNV) tiles, the bf16 state copy S̄
+// (128 x kNV), then the barriers.
 constexpr int kStages = 2;
-constexpr int kStageBytes = 3 * kTileBytes;            // Q, K, V tiles: 96 KiB
-constexpr int kSbarOff = kStages * kStageBytes;        // bf16 state copy S̄ (32 KiB)
-constexpr int kCtrlOff = kSbarOff + kTileBytes;        // barriers etc.
-constexpr int kSmemBytes = kCtrlOff + 256 + 1024;      // + slack for 1 KiB alignment
+__host__ __device__ constexpr int stage_bytes(int nv) { return 2 * kTileBytes + (nv / 64) * kHalfBytes; }
+__host__ __device__ constexpr int sbar_offset(int nv) { return kStages * stage_bytes(nv); }
+__host__ __device__ constexpr int ctrl_offset(int nv) { return sbar_offset(nv) + (nv / 64) * kHalfBytes; }
+__host__ __device__ constexpr int smem_bytes(int nv) { return ctrl_offset(nv) + 256 + 1024; }
 
 // TMEM columns (fp32 cells; 128 lanes each)
 constexpr uint32_t kColState = 0;    // S      [k-dim lanes][v-dim cols]
-constexpr uint32_t kColS = 128;      // scores Q K^T
-constexpr uint32_t kColP = 256;      // masked scores, bf16 pairs (64 cols)
-constexpr uint32_t kColO = 384;      // output accumulator
+constexpr uint32_t kColS = 128;      // scores Q K^T; the masked scores P (bf16
+                                     // pairs) overwrite columns [128,160) (keys
+                                     // 0-63) and [192,224) (keys 64-127)
+constexpr uint32_t kColO = 256;      // output accumulator
+constexpr uint32_t kColDelta = 384;  // single pass: chunk increment K_c^T V_c
 constexpr uint32_t kTmemCols = 512;
 
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 32 * (2 + kEpiWarps);
+// TMEM column of the bf16 P pairs for keys [16*kk, 16*kk+16): each epilogue
+// thread writes its packed keys into the first half of the score columns it
+// has just read itself.
+__host__ __device__ constexpr uint32_t p_col(int kk) {
+    return kColS + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
+}
+
+// 14 warps: warp 0 producer, warp 1 MMA issuer, warps 2-9 epilogue, warps
+// 10-13 chain warps.
+constexpr int kEpiWarps = 8;       // P / S̄ / O / final state: 64 columns of one row per thread
+constexpr int kChainWarps = 4;     // phase B (single pass) and starting states, full rows
+constexpr int kFirstEpiWarp = 2;
+constexpr int kFirstChainWarp = kFirstEpiWarp + kEpiWarps;
+constexpr int kThreads = 32 * (kFirstChainWarp + kChainWarps);
 
 constexpr int kModeDense = 0;
 constexpr int kModeVarlen = 1;
@@ -64,10 +81,15 @@ struct Ctrl {
     uint64_t tail_ld;      // TMA completion of a packed-sequence tail block
     uint64_t s_full;       // MMA1 complete (scores in TMEM)
     uint64_t p_ready;      // epilogue wrote P (one arrival per epilogue warp)
-    uint64_t sbar_ready;   // epilogue wrote S̄ / the initial state
+    uint64_t sbar_ready;   // epilogue released / initialised TMEM S and wrote S̄
     uint64_t state_done;   // MMA4 complete (state updated)
     uint64_t o_full;       // MMA2 complete (output accumulated)
     uint64_t o_free;       // epilogue drained O
+    uint64_t delta_done;   // single pass: chunk increment K_c^T V_c complete
+    uint64_t delta_free;   // single pass: chain warps read the increment
+    uint64_t state_free;   // epilogue finished with TMEM S / S̄ of an item
+    uint64_t o_staged;     // every epilogue warp wrote its part of O (bf16) to smem
+    uint64_t o_stored[kStages];  // O tile staged in stage s has left shared memory
     uint32_t tmem_base;
     int abort;
 };
@@ -86,29 +108,47 @@ struct Params {
     int num_seqs;
     __nv_bfloat16* o;           // [Z][rows][128]
     const float* prefix;        // [Z][chunks][128][128] exclusive chunk prefixes, or null
-    float* state_out;           // [Z][128][128] written at the end of each item, or null
+    float* state_out;           // final states, or null: dense [Z][128][128], packed
+                                // [num_seqs][H][128][128]
     float* chunk_delta;         // chunk_state output, same layout as prefix
+    int fused;                  // single pass: chunk prefixes found by look-back
+    float* chain;               // single pass: inclusive chunk prefixes, layout of prefix
+    int* flags;                 // single pass: "prefix published" words, one per chunk,
+                                // value part and chain warp ([chunks][vparts][4], zeroed)
+    int vparts;                 // value columns split over this many CTAs (1 or 2)
 };
 
+// One work item: rows [t0, t1) of slice z, chunk c of its sequence, value
+// columns [vp * 128 / vparts, (vp + 1) * 128 / vparts).
+//   ws    index of the chunk in the per-chunk state arrays
+//   sidx  index of the sequence's final state in state_out
+//   last  the chunk ends its sequence
 struct Item {
-    int z, c, t0, t1, ws;
+    int z, c, t0, t1, ws, sidx, vp;
+    bool last;
 };
 
 __device__ __forceinline__ int num_items(const Params& p) {
     if (p.mode == kModeDense) return p.n_items;
     if (*p.seq_ok == 0) return 0;
-    return p.Z * p.chunk_off[p.num_seqs];
+    return p.Z * p.chunk_off[p.num_seqs] * p.vparts;
 }
 
+// Items are ordered chunk-major, then slice, then value part: the value parts
+// of one chunk are neighbours (they run together and share Q and K in L2).
 __device__ __forceinline__ Item get_item(const Params& p, int item) {
     Item it;
+    it.vp = item % p.vparts;
+    item /= p.vparts;
     it.z = item % p.Z;
-    const int g = item / p.Z;                     // chunk-major order
+    const int g = item / p.Z;
     if (p.mode == kModeDense) {
         it.c = g;
         it.t0 = g * p.chunk_tokens;
         it.t1 = min(it.t0 + p.chunk_tokens, p.rows);
         it.ws = it.z * p.n_chunks + g;
+        it.sidx = it.z;
+        it.last = g == p.n_chunks - 1;
     } else {
         // sequence j with chunk_off[j] <= g < chunk_off[j+1] (empty sequences
         // own no chunk and are skipped by taking the largest such j)
@@ -121,6 +161,8 @@ __device__ __forceinline__ Item get_item(const Params& p, int item) {
         it.t0 = p.cu_seqlens[lo] + it.c * p.chunk_tokens;
         it.t1 = min(it.t0 + p.chunk_tokens, (int)p.cu_seqlens[lo + 1]);
         it.ws = it.z * p.chunk_off[p.num_seqs] + g;
+        it.sidx = lo * p.Z + it.z;
+        it.last = g == p.chunk_off[lo + 1] - 1;
     }
     return it;
 }
@@ -147,14 +189,14 @@ __device__ __forceinline__ void store_row32_bf16_sw128(uint8_t* tile, int row, i
     }
 }
 
-// Zero rows [valid, 128) of a V tile (both 64-column halves), by one warp.
-// Used for the last block of a packed sequence, whose trailing rows belong to
-// the next sequence: they must not enter K^T V.
-__device__ __forceinline__ void zero_tail_rows(uint8_t* vtile, int valid, int lane) {
-    const int n = (kTileRows - valid) * 16;       // 16-byte chunks to clear
+// Zero rows [valid, 128) of a V tile of `halves` 64-column halves, by one
+// warp.  Used for the last block of a packed sequence, whose trailing rows
+// belong to the next sequence: they must not enter K^T V.
+__device__ __forceinline__ void zero_tail_rows(uint8_t* vtile, int valid, int lane, int halves) {
+    const int n = (kTileRows - valid) * 8 * halves;   // 16-byte chunks to clear
     for (int i = lane; i < n; i += 32) {
-        const int row = valid + (i >> 4);
-        const int ch = i & 15;
+        const int row = valid + i / (8 * halves);
+        const int ch = i % (8 * halves);
         *reinterpret_cast<uint4*>(vtile + (ch >> 3) * kHalfBytes + row * 128 + (ch & 7) * 16) =
             make_uint4(0u, 0u, 0u, 0u);
     }
@@ -164,28 +206,30 @@ __device__ __forceinline__ void zero_tail_rows(uint8_t* vtile, int valid, int la
 // (optional), K and V tiles of rows [t, t+128) of slice z.  For a packed tail
 // (fewer than 128 valid rows) the load completes on `tail_ld`, the warp clears
 // the foreign rows of V and then releases `full`.  Returns false on abort.
-template <bool kLoadQ>
+// The V tile holds kVHalves 64-column halves starting at column v_x.
+template <bool kLoadQ, int kVHalves = 2>
 __device__ __forceinline__ bool produce_tile(const CUtensorMap* tmQ, const CUtensorMap* tmK,
                                              const CUtensorMap* tmV, uint8_t* stage_ptr,
                                              uint32_t stage, uint32_t full_bar, uint32_t tail_bar,
                                              uint32_t& n_tail, int t, int z, int valid,
-                                             bool packed, uint64_t pol, int lane,
-                                             volatile int* abort_flag) {
-    constexpr uint32_t kBytes = (kLoadQ ? 3 : 2) * kTileBytes;
+                                             bool packed, uint64_t q_pol, uint64_t pol, int lane,
+                                             volatile int* abort_flag, int v_x = 0) {
+    constexpr uint32_t kBytes = (kLoadQ ? 2 : 1) * kTileBytes + kVHalves * kHalfBytes;
     const bool tail = packed && valid < kTileRows;
     if (lane == 0) {
         const uint32_t b = tail ? tail_bar : full_bar;
         ptx::mbar_arrive_expect_tx(b, kBytes);
         uint32_t dst = stage;
         if (kLoadQ) {
-            ptx::tma_load_3d(dst, tmQ, b, 0, t, z, pol);
-            ptx::tma_load_3d(dst + kHalfBytes, tmQ, b, 64, t, z, pol);
+            ptx::tma_load_3d(dst, tmQ, b, 0, t, z, q_pol);
+            ptx::tma_load_3d(dst + kHalfBytes, tmQ, b, 64, t, z, q_pol);
             dst += kTileBytes;
         }
         ptx::tma_load_3d(dst, tmK, b, 0, t, z, pol);
         ptx::tma_load_3d(dst + kHalfBytes, tmK, b, 64, t, z, pol);
-        ptx::tma_load_3d(dst + kTileBytes, tmV, b, 0, t, z, pol);
-        ptx::tma_load_3d(dst + kTileBytes + kHalfBytes, tmV, b, 64, t, z, pol);
+#pragma unroll
+        for (int hv = 0; hv < kVHalves; ++hv)
+            ptx::tma_load_3d(dst + kTileBytes + hv * kHalfBytes, tmV, b, v_x + 64 * hv, t, z, pol);
     }
     if (!tail) return true;
     int ok = 1;
@@ -193,7 +237,7 @@ __device__ __forceinline__ bool produce_tile(const CUtensorMap* tmQ, const CUten
     ok = __shfl_sync(0xffffffffu, ok, 0);
     ++n_tail;
     if (!ok) return false;
-    zero_tail_rows(stage_ptr + (kLoadQ ? 2 : 1) * kTileBytes, valid, lane);
+    zero_tail_rows(stage_ptr + (kLoadQ ? 2 : 1) * kTileBytes, valid, lane, kVHalves);
     ptx::fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(full_bar);
@@ -202,16 +246,44 @@ __device__ __forceinline__ bool produce_tile(const CUtensorMap* tmQ, const CUten
 
 // ============================================================================
 // Main kernel: outputs of every chunk from its starting state.
+//
+// Three-pass schedule (p.fused == 0): the starting state of chunk c > 0 is
+// the exclusive prefix p.prefix[ws] written by chunk_state + chunk_scan.
+//
+// Single pass (p.fused == 1), per work item (z, c):
+//   phase A  a chunk with a successor accumulates its increment K_c^T V_c in
+//            TMEM (columns kColDelta);
+//   phase B  the epilogue waits for the inclusive prefix of chunk c-1, which
+//            the CTA owning it publishes in global memory, publishes its own
+//            inclusive prefix for chunk c+1, and loads the exclusive prefix
+//            as the starting state;
+//   phase C  outputs, as in the three-pass schedule.
+// A CTA runs phase A of its next item before phase C of the current one, so
+// the K/V stream of that phase A overlaps the epilogue's phase B.  Items are
+// visited in chunk-major order and every CTA walks its items in increasing
+// order, so the smallest unfinished item never waits (the predecessor it
+// needs has a smaller index).  Every wait is bounded; a consumed prefix is
+// dropped from L2 without write-back (it has exactly one reader).
 // ============================================================================
+// kNV: value columns handled by one CTA (128, or 64 when the columns of every
+// head are split over p.vparts = 2 CTAs).  Columns of S and O are independent
+// (S[:, v] = sum k^T v[v], O[:, v] = Q S[:, v] + P V[:, v]), so a split needs
+// no exchange; both parts compute the scores Q K^T.
+template <int kNV>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const Params p) {
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const Params p) {
+    static_assert(kNV == 64 || kNV == 128, "value part width");
+    constexpr int kVHalves = kNV / 64;
+    constexpr int kStageB = stage_bytes(kNV);
+    constexpr int kSbarOffT = sbar_offset(kNV);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + kCtrlOff);
+    Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + ctrl_offset(kNV));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t sbase = ptx::smem_u32(smem);
-    const uint32_t sSbar = sbase + kSbarOff;
+    const uint32_t sSbar = sbase + kSbarOffT;
     auto bar = [&](uint64_t& b) { return ptx::smem_u32(&b); };
 
     if (threadIdx.x == 0) {
@@ -226,6 +298,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         ptx::mbar_init(bar(ctrl->state_done), 1);
         ptx::mbar_init(bar(ctrl->o_full), 1);
         ptx::mbar_init(bar(ctrl->o_free), kEpiWarps);
+        ptx::mbar_init(bar(ctrl->delta_done), 1);
+        ptx::mbar_init(bar(ctrl->delta_free), kChainWarps);
+        ptx::mbar_init(bar(ctrl->state_free), kEpiWarps);
+        ptx::mbar_init(bar(ctrl->o_staged), kEpiWarps);
+        for (int s = 0; s < kStages; ++s) ptx::mbar_init(bar(ctrl->o_stored[s]), 1);
         ctrl->abort = 0;
         ptx::fence_mbar_init();
     }
@@ -237,6 +314,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         ptx::prefetch_tmap(&tmQ);
         ptx::prefetch_tmap(&tmK);
         ptx::prefetch_tmap(&tmV);
+        ptx::prefetch_tmap(&tmO);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -245,54 +323,131 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     volatile int* abort_flag = &ctrl->abort;
     const int n_items = num_items(p);
     const bool packed = p.mode == kModeVarlen;
+    const bool fused = p.fused != 0;
+    const int stride = gridDim.x;
+    // phase A is run for chunks that have a successor (single pass only)
+    auto has_phase_a = [&](const Item& it) { return fused && !it.last; };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        const uint64_t pol = ptx::policy_evict_first();
+        const uint64_t pol_first = ptx::policy_evict_first();
+        const uint64_t pol_last = ptx::policy_evict_last();
         uint32_t g = 0, n_tail = 0;
         bool ok = true;
-        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+        auto next_stage = [&](int& s) -> bool {
+            s = g & 1;
+            if (g >= 2) {
+                int w = 1;
+                if (lane == 0) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
+                if (!__shfl_sync(0xffffffffu, w, 0)) return false;
+            }
+            return true;
+        };
+        auto load_phase_a = [&](const Item& it) {
+            // K and V only, kept in L2 for phase C
+            for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
+                int s;
+                if (!next_stage(s) ||
+                    !produce_tile<false, kVHalves>(nullptr, &tmK, &tmV, smem + s * kStageB + kTileBytes,
+                                                   sbase + s * kStageB + kTileBytes, bar(ctrl->full[s]),
+                                                   bar(ctrl->tail_ld), n_tail, t, it.z, it.t1 - t, packed,
+                                                   pol_last, pol_last, lane, abort_flag, it.vp * kNV))
+                    ok = false;
+            }
+        };
+        if ((int)blockIdx.x < n_items) {
+            const Item first = get_item(p, blockIdx.x);
+            if (has_phase_a(first)) load_phase_a(first);
+        }
+        uint32_t c_uses[kStages] = {0, 0};   // phase-C uses of each stage so far
+        for (int item = blockIdx.x; ok && item < n_items; item += stride) {
             const Item it = get_item(p, item);
-            for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
-                const int s = g & 1;
-                if (g >= 2) {
+            if (item + stride < n_items) {
+                const Item nx = get_item(p, item + stride);
+                if (has_phase_a(nx)) load_phase_a(nx);
+            }
+            for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
+                int s;
+                if (!next_stage(s)) { ok = false; break; }
+                if (c_uses[s] > 0) {
+                    // the Q slot also staged the O tile of that stage's last phase-C block
                     int w = 1;
-                    if (lane == 0) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
+                    if (lane == 0) w = ptx::mbar_wait(bar(ctrl->o_stored[s]), (c_uses[s] - 1) & 1, abort_flag);
                     if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
                 }
-                if (!produce_tile<true>(&tmQ, &tmK, &tmV, smem + s * kStageBytes, sbase + s * kStageBytes,
-                                        bar(ctrl->full[s]), bar(ctrl->tail_ld), n_tail, t, it.z,
-                                        it.t1 - t, packed, pol, lane, abort_flag)) {
+                ++c_uses[s];
+                if (!produce_tile<true, kVHalves>(&tmQ, &tmK, &tmV, smem + s * kStageB, sbase + s * kStageB,
+                                                  bar(ctrl->full[s]), bar(ctrl->tail_ld), n_tail, t, it.z,
+                                                  it.t1 - t, packed, pol_first, pol_first, lane, abort_flag,
+                                                  it.vp * kNV))
                     ok = false;
-                    break;
-                }
             }
         }
-        // Wait for the last stage releases so that no asynchronous arrive
-        // is still pending on this CTA's shared memory when it exits.
-        if (lane == 0)
+        // Wait for the last stage releases (MMA commits and O stores) so that no
+        // asynchronous arrive is still pending on this CTA's shared memory when
+        // it exits.
+        if (lane == 0) {
             for (uint32_t j = (g >= 2 ? g - 2 : 0); ok && j < g; ++j)
                 ok = ptx::mbar_wait(bar(ctrl->empty[j & 1]), (j >> 1) & 1, abort_flag);
+            for (int s = 0; ok && s < kStages; ++s)
+                if (c_uses[s] > 0) ok = ptx::mbar_wait(bar(ctrl->o_stored[s]), (c_uses[s] - 1) & 1, abort_flag);
+        }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t id_qk = ptx::idesc_bf16(128, 128, false, false);  // Q K^T
-            constexpr uint32_t id_qs = ptx::idesc_bf16(128, 128, false, true);   // Q S̄
-            constexpr uint32_t id_kv = ptx::idesc_bf16(128, 128, true, true);    // K^T V
-            constexpr uint32_t id_pv = ptx::idesc_bf16(128, 128, false, true);   // P V
-            uint32_t g = 0;
+            constexpr uint32_t id_qs = ptx::idesc_bf16(128, kNV, false, true);   // Q S̄
+            constexpr uint32_t id_kv = ptx::idesc_bf16(128, kNV, true, true);    // K^T V
+            constexpr uint32_t id_pv = ptx::idesc_bf16(128, kNV, false, true);   // P V
+            uint32_t g = 0, n_sb = 0, n_a = 0, n_blk = 0;
             bool ok = true;
-            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-                const Item it = get_item(p, item);
-                bool has_state = (p.prefix != nullptr) && it.c > 0;
+            // phase A: TMEM delta = K_c^T V_c over the chunk's blocks
+            auto run_phase_a = [&](const Item& it) {
+                if (n_a > 0 && !ptx::mbar_wait(bar(ctrl->delta_free), (n_a - 1) & 1, abort_flag)) {
+                    ok = false;
+                    return;
+                }
+                ptx::tc_fence_after();
+                bool first = true;
                 for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
+                    const int s = g & 1;
+                    if (!ptx::mbar_wait(bar(ctrl->full[s]), (g >> 1) & 1, abort_flag)) { ok = false; return; }
+                    ptx::tc_fence_after();
+                    const uint32_t sk = sbase + s * kStageB + kTileBytes;
+                    const uint32_t sv = sk + kTileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        ptx::mma_ss(tmem + kColDelta, ptx::sdesc_sw128(sk + kk * 2048, kHalfBytes, 1024),
+                                    ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_kv,
+                                    (kk > 0 || !first) ? 1u : 0u);
+                    ptx::mma_commit(bar(ctrl->empty[s]));
+                    first = false;
+                }
+                ptx::mma_commit(bar(ctrl->delta_done));
+                ++n_a;
+            };
+            if ((int)blockIdx.x < n_items) {
+                const Item first = get_item(p, blockIdx.x);
+                if (has_phase_a(first)) run_phase_a(first);
+            }
+            for (int item = blockIdx.x; ok && item < n_items; item += stride) {
+                const Item it = get_item(p, item);
+                if (item + stride < n_items) {
+                    const Item nx = get_item(p, item + stride);
+                    if (has_phase_a(nx)) run_phase_a(nx);
+                    if (!ok) break;
+                }
+                bool has_state = fused ? it.c > 0 : (p.prefix != nullptr && it.c > 0);
+                for (int t = it.t0; t < it.t1; t += kTileRows, ++g, ++n_blk) {
                     const int s = g & 1;
                     if (!ptx::mbar_wait(bar(ctrl->full[s]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
                     ptx::tc_fence_after();
-                    const uint32_t sq = sbase + s * kStageBytes;
+                    const uint32_t sq = sbase + s * kStageB;
                     const uint32_t sk = sq + kTileBytes;
                     const uint32_t sv = sq + 2 * kTileBytes;
-                    // MMA1: scores = Q K^T (both operands K-major, K = head dim)
+                    // MMA1: scores = Q K^T (both operands K-major, K = head dim).  It
+                    // overwrites the P of the previous block, whose MMA2 was issued
+                    // earlier by this thread (tcgen05 MMAs run in issue order).
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
@@ -300,8 +455,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                                     ptx::sdesc_sw128(sk + off, 16, 1024), id_qk, kk > 0);
                     }
                     ptx::mma_commit(bar(ctrl->s_full));
-                    if (!ptx::mbar_wait(bar(ctrl->sbar_ready), g & 1, abort_flag)) { ok = false; break; }
-                    if (g > 0 && !ptx::mbar_wait(bar(ctrl->o_free), (g - 1) & 1, abort_flag)) { ok = false; break; }
+                    if (!ptx::mbar_wait(bar(ctrl->sbar_ready), n_sb++ & 1, abort_flag)) { ok = false; break; }
+                    if (n_blk > 0 && !ptx::mbar_wait(bar(ctrl->o_free), (n_blk - 1) & 1, abort_flag)) { ok = false; break; }
                     ptx::tc_fence_after();
                     // MMA3: O = Q S̄ (inter-block, right product); S̄ is MN-major
                     if (has_state) {
@@ -321,12 +476,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                                     (kk > 0 || has_state) ? 1u : 0u);
                     }
                     ptx::mma_commit(bar(ctrl->state_done));
-                    if (!ptx::mbar_wait(bar(ctrl->p_ready), g & 1, abort_flag)) { ok = false; break; }
+                    if (!ptx::mbar_wait(bar(ctrl->p_ready), n_blk & 1, abort_flag)) { ok = false; break; }
                     ptx::tc_fence_after();
                     // MMA2: O += P V (intra-block, left product); P from TMEM
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
-                        ptx::mma_ts(tmem + kColO, tmem + kColP + kk * 8,
+                        ptx::mma_ts(tmem + kColO, tmem + p_col(kk),
                                     ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_pv,
                                     (kk > 0 || has_state) ? 1u : 0u);
                     }
@@ -336,68 +491,60 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 }
             }
         }
-    } else {
+    } else if (warp < kFirstChainWarp) {
         // ------------------------------------------------------------ epilogue
-        const int ew = warp - 2;             // 0..7
-        const int h = ew >> 2;               // column half owned by this warpgroup
+        const int ew = warp - kFirstEpiWarp; // 0..7
         const int sp = warp & 3;             // TMEM sub-partition this warp may access
         const int r = sp * 32 + lane;        // tile row owned by this thread
-        const int c0 = 64 * h;               // first owned column
+        const int k0 = 64 * (ew >> 2);       // score columns (keys) [k0, k0 + 64) of that row
+        constexpr int kCols = kNV / 2;       // value columns per thread
+        const int c0 = kCols * (ew >> 2);    // value columns [c0, c0 + kCols) of this part
         const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
-        uint8_t* sbar_tile = smem + kSbarOff;
+        uint8_t* sbar_tile = smem + kSbarOffT;
+        const bool store_leader = (ew == 0 && lane == 0);
+        uint32_t n_blk = 0;
+        // tile counter of the producer (phase A and phase C tiles), to know the
+        // stage a phase-C block occupies
         uint32_t g = 0;
+        auto n_tiles = [&](const Item& x) { return (uint32_t)((x.t1 - x.t0 + kTileRows - 1) / kTileRows); };
+        if ((int)blockIdx.x < n_items) {
+            const Item first = get_item(p, blockIdx.x);
+            if (has_phase_a(first)) g += n_tiles(first);
+        }
         bool ok = true;
-        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+        for (int item = blockIdx.x; ok && item < n_items; item += stride) {
             const Item it = get_item(p, item);
-            // ---- initial state of the chunk: TMEM S and its bf16 copy S̄
-            if (p.prefix != nullptr && it.c > 0) {
-                const float4* src = reinterpret_cast<const float4*>(
-                    p.prefix + (size_t)it.ws * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim + c0);
-                uint32_t f[64];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float4 x = __ldg(src + j);
-                    f[4 * j + 0] = __float_as_uint(x.x);
-                    f[4 * j + 1] = __float_as_uint(x.y);
-                    f[4 * j + 2] = __float_as_uint(x.z);
-                    f[4 * j + 3] = __float_as_uint(x.w);
-                }
-                ptx::tmem_st32(tl + kColState + c0, *reinterpret_cast<uint32_t(*)[32]>(f));
-                ptx::tmem_st32(tl + kColState + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(f + 32));
-                store_row32_bf16_sw128(sbar_tile, r, c0, f);
-                store_row32_bf16_sw128(sbar_tile, r, c0 + 32, f + 32);
-                ptx::tmem_st_wait();
-                ptx::fence_proxy_async_smem();
+            if (item + stride < n_items) {
+                const Item nx = get_item(p, item + stride);
+                if (has_phase_a(nx)) g += n_tiles(nx);
             }
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready));
-
-            for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
+            for (int t = it.t0; t < it.t1; t += kTileRows, ++n_blk, ++g) {
                 const bool last_block = t + kTileRows >= it.t1;
-                // ---- 1. P = tril(scores) as bf16 pairs into TMEM (columns c0..c0+63)
-                if (!ptx::mbar_wait(bar(ctrl->s_full), g & 1, abort_flag)) { ok = false; break; }
+                const int s = g & 1;
+                // ---- 1. P = tril(scores) as bf16 pairs over the first half of the
+                //         score columns this thread reads (keys c0..c0+63)
+                if (!ptx::mbar_wait(bar(ctrl->s_full), n_blk & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
                 {
                     uint32_t pk[32];
-                    if (c0 > sp * 32 + 31) {
+                    if (k0 > sp * 32 + 31) {
                         // every key of this half lies above the diagonal for these rows
 #pragma unroll
                         for (int j = 0; j < 32; ++j) pk[j] = 0u;
                     } else {
                         uint32_t v[64];
-                        ptx::tmem_ld32(tl + kColS + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
-                        ptx::tmem_ld32(tl + kColS + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                        ptx::tmem_ld32(tl + kColS + k0, *reinterpret_cast<uint32_t(*)[32]>(v));
+                        ptx::tmem_ld32(tl + kColS + k0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
                         ptx::tmem_ld_wait();
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
-                            const int key = c0 + 2 * j;
+                            const int key = k0 + 2 * j;
                             const float a = (key <= r) ? __uint_as_float(v[2 * j]) : 0.0f;
                             const float b = (key + 1 <= r) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
                             pk[j] = ptx::pack_bf16x2(a, b);
                         }
                     }
-                    ptx::tmem_st32(tl + kColP + (c0 >> 1), pk);
+                    ptx::tmem_st32(tl + kColS + k0, pk);
                 }
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
@@ -405,46 +552,68 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 if (lane == 0) ptx::mbar_arrive(bar(ctrl->p_ready));
 
                 // ---- 2. state: bf16 copy for the next block, or the final state
-                if (!ptx::mbar_wait(bar(ctrl->state_done), g & 1, abort_flag)) { ok = false; break; }
+                if (!ptx::mbar_wait(bar(ctrl->state_done), n_blk & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
-                if (!last_block || p.state_out != nullptr) {
-                    uint32_t v[64];
-                    ptx::tmem_ld32(tl + kColState + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
-                    ptx::tmem_ld32(tl + kColState + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                float* final_dst = nullptr;
+                if (last_block && p.state_out != nullptr && (!fused || it.last))
+                    final_dst = p.state_out + (size_t)it.sidx * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim +
+                                it.vp * kNV + c0;
+                if (!last_block || final_dst != nullptr) {
+                    uint32_t v[kCols];
+#pragma unroll
+                    for (int q = 0; q < kCols / 32; ++q)
+                        ptx::tmem_ld32(tl + kColState + c0 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * q));
                     ptx::tmem_ld_wait();
                     if (!last_block) {
-                        store_row32_bf16_sw128(sbar_tile, r, c0, v);
-                        store_row32_bf16_sw128(sbar_tile, r, c0 + 32, v + 32);
-                        ptx::fence_proxy_async_smem();
-                        ptx::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready));
-                    } else {
-                        float4* dst = reinterpret_cast<float4*>(
-                            p.state_out + (size_t)it.z * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim + c0);
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
+                        for (int q = 0; q < kCols / 32; ++q) store_row32_bf16_sw128(sbar_tile, r, c0 + 32 * q, v + 32 * q);
+                    } else {
+                        float4* dst = reinterpret_cast<float4*>(final_dst);
+#pragma unroll
+                        for (int j = 0; j < kCols / 4; ++j)
                             dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                                                  __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
                     }
                 }
+                ptx::tc_fence_before();
+                if (!last_block) {
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready));
+                } else {
+                    // TMEM S and S̄ are no longer read for this item: the chain warps
+                    // may write the next item's starting state
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->state_free));
+                }
 
-                // ---- 3. O -> bf16 -> global (columns c0..c0+63 of row t + r)
-                if (!ptx::mbar_wait(bar(ctrl->o_full), g & 1, abort_flag)) { ok = false; break; }
+                // ---- 3. O: load to registers, release the accumulator, convert to
+                //         bf16 into the Q slot of this block's stage (free: MMA1 and
+                //         MMA3 have completed), then one thread stores the tile with
+                //         TMA.  The last block of a packed sequence is stored row by
+                //         row instead, so that the next sequence's rows are untouched.
+                if (!ptx::mbar_wait(bar(ctrl->o_full), n_blk & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
+                const bool rowwise = packed && t + kTileRows > it.t1;
+                uint8_t* ostage = smem + s * kStageB;
                 {
-                    uint32_t v[64];
-                    ptx::tmem_ld32(tl + kColO + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
-                    ptx::tmem_ld32(tl + kColO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                    uint32_t v[kCols];
+#pragma unroll
+                    for (int q = 0; q < kCols / 32; ++q)
+                        ptx::tmem_ld32(tl + kColO + c0 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * q));
                     ptx::tmem_ld_wait();
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_free));
-                    if (t + r < it.t1) {
-                        uint4* orow = reinterpret_cast<uint4*>(
-                            p.o + ((size_t)it.z * p.rows + t + r) * kHeadDim + c0);
+                    if (!rowwise) {
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
+                        for (int q = 0; q < kCols / 32; ++q) store_row32_bf16_sw128(ostage, r, c0 + 32 * q, v + 32 * q);
+                        ptx::fence_proxy_async_smem();
+                    } else if (t + r < it.t1) {
+                        uint4* orow = reinterpret_cast<uint4*>(
+                            p.o + ((size_t)it.z * p.rows + t + r) * kHeadDim + it.vp * kNV + c0);
+#pragma unroll
+                        for (int j = 0; j < kCols / 8; ++j) {
                             uint4 w;
                             w.x = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
                             w.y = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
@@ -453,8 +622,149 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                             orow[j] = w;
                         }
                     }
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_staged));
                 }
+                if (store_leader) {
+                    if (!ptx::mbar_wait(bar(ctrl->o_staged), n_blk & 1, abort_flag)) { ok = false; }
+                    if (ok && !rowwise) {
+                        const uint32_t src = sbase + s * kStageB;
+#pragma unroll
+                        for (int hv = 0; hv < kVHalves; ++hv)
+                            ptx::tma_store_3d(&tmO, src + hv * kHalfBytes, it.vp * kNV + 64 * hv, t, it.z);
+                        ptx::bulk_commit_group();
+                        ptx::bulk_wait_group_read0();
+                    }
+                    ptx::mbar_arrive(bar(ctrl->o_stored[s]));
+                }
+                __syncwarp();
+                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             }
+        }
+        if (store_leader) ptx::bulk_wait_group0();
+    } else {
+        // ------------------------------------------------------------ chain warps
+        // Starting state of every item; in the single pass also phase B.  Each
+        // chain warp owns rows [32 sp, 32 sp + 32) of the state (a 16 KiB slice
+        // with its own "published" flag), so the slices advance independently.
+        // Phase B of an item runs while the epilogue is still on the previous
+        // item; only writing the starting state waits for that item to finish.
+        const int cw = warp - kFirstChainWarp;  // 0..3
+        const int sp = warp & 3;
+        const int r = sp * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
+        uint8_t* sbar_tile = smem + kSbarOffT;
+        uint32_t n_delta = 0, n_sf = 0;
+        bool ok = true;
+        bool first_item = true;
+        for (int item = blockIdx.x; ok && item < n_items; item += stride) {
+            const Item it = get_item(p, item);
+            const bool phase_a = has_phase_a(it);
+            const bool look = fused && it.c > 0;
+            const bool from_prefix = !fused && p.prefix != nullptr && it.c > 0;
+            const size_t roff = (size_t)r * kHeadDim + it.vp * kNV;   // row r, this value part
+            const float* src = nullptr;          // exclusive prefix
+            if (look) src = p.chain + (size_t)(it.ws - 1) * (kHeadDim * kHeadDim) + roff;
+            if (from_prefix) src = p.prefix + (size_t)it.ws * (kHeadDim * kHeadDim) + roff;
+            const size_t fl = ((size_t)it.ws * p.vparts + it.vp) * kChainWarps + cw;   // own flag
+            const size_t fl_prev = fl - (size_t)p.vparts * kChainWarps;               // chunk c-1's
+            if (phase_a) {
+                if (!ptx::mbar_wait(bar(ctrl->delta_done), n_delta++ & 1, abort_flag)) { ok = false; break; }
+                ptx::tc_fence_after();
+            }
+            if (look) {
+                // ---- wait for this slice of chunk c-1's inclusive prefix
+                const int* f = p.flags + fl_prev;
+                const unsigned long long t0 = globaltimer_ns();
+                bool seen = false;
+                while (true) {
+                    const int v = ptx::ld_acquire_gpu(f);
+                    if (__all_sync(0xffffffffu, v != 0)) { seen = true; break; }
+                    if (*abort_flag) break;
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        record_device_error(LA_ERR_TIMEOUT);
+                        break;
+                    }
+                }
+                if (!__all_sync(0xffffffffu, seen)) { ok = false; break; }
+            }
+            if (phase_a) {
+                // ---- publish this slice of chunk c's inclusive prefix, 64 columns
+                //      per round trip to L2
+                float4* dst = reinterpret_cast<float4*>(p.chain + (size_t)it.ws * (kHeadDim * kHeadDim) + roff);
+#pragma unroll
+                for (int hh = 0; hh < kVHalves; ++hh) {
+                    float pr[64];
+                    if (src != nullptr) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float4 x = __ldcg(reinterpret_cast<const float4*>(src + 64 * hh) + j);
+                            pr[4 * j + 0] = x.x;
+                            pr[4 * j + 1] = x.y;
+                            pr[4 * j + 2] = x.z;
+                            pr[4 * j + 3] = x.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) pr[j] = 0.f;
+                    }
+#pragma unroll
+                    for (int q2 = 0; q2 < 2; ++q2) {
+                        uint32_t d[32];
+                        ptx::tmem_ld32(tl + kColDelta + 64 * hh + 32 * q2, d);
+                        ptx::tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            __stcg(dst + 16 * hh + 8 * q2 + j,
+                                   make_float4(pr[32 * q2 + 4 * j + 0] + __uint_as_float(d[4 * j + 0]),
+                                               pr[32 * q2 + 4 * j + 1] + __uint_as_float(d[4 * j + 1]),
+                                               pr[32 * q2 + 4 * j + 2] + __uint_as_float(d[4 * j + 2]),
+                                               pr[32 * q2 + 4 * j + 3] + __uint_as_float(d[4 * j + 3])));
+                    }
+                }
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) ptx::st_release_gpu(p.flags + fl, 1);
+                // the increment has been read: TMEM is free for the next phase A
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(ctrl->delta_free));
+            }
+            // ---- starting state of phase C, once the previous item is done with it
+            if (!first_item && !ptx::mbar_wait(bar(ctrl->state_free), n_sf++ & 1, abort_flag)) { ok = false; break; }
+            first_item = false;
+            ptx::tc_fence_after();
+            if (src != nullptr) {
+#pragma unroll
+                for (int hh = 0; hh < kVHalves; ++hh) {
+                    uint32_t f[64];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float4 x = look ? __ldcg(reinterpret_cast<const float4*>(src + 64 * hh) + j)
+                                              : __ldg(reinterpret_cast<const float4*>(src + 64 * hh) + j);
+                        f[4 * j + 0] = __float_as_uint(x.x);
+                        f[4 * j + 1] = __float_as_uint(x.y);
+                        f[4 * j + 2] = __float_as_uint(x.z);
+                        f[4 * j + 3] = __float_as_uint(x.w);
+                    }
+                    ptx::tmem_st32(tl + kColState + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(f));
+                    ptx::tmem_st32(tl + kColState + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(f + 32));
+                    store_row32_bf16_sw128(sbar_tile, r, 64 * hh, f);
+                    store_row32_bf16_sw128(sbar_tile, r, 64 * hh + 32, f + 32);
+                }
+                if (look) {
+                    // this slice of chunk c-1's prefix has exactly one reader: drop it
+#pragma unroll
+                    for (int j = 0; j < kNV / 32; ++j) ptx::discard_l2_line(src + 32 * j);
+                }
+                ptx::tmem_st_wait();
+                ptx::fence_proxy_async_smem();
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            // sbar_ready counts epilogue warps: each chain warp stands for two
+            if (lane == 0) ptx::mbar_arrive_cnt(bar(ctrl->sbar_ready), kEpiWarps / kChainWarps);
         }
     }
 
@@ -463,6 +773,361 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     if (warp == 1) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ============================================================================
+// Sequential kernel for split value columns (64 per CTA).
+//
+// One work item is a whole sequence (or a chunk of the three-pass schedule)
+// for one half of the value columns.  The block loop is pipelined so that the
+// tensor cores never wait for the epilogue:
+//   * the state increment of each block, dS_i = K_i^T V_i, goes to one of two
+//     TMEM buffers; the running state S (fp32) lives in the epilogue's
+//     registers (32 values per thread), which add dS_i and write the bf16 copy
+//     S̄_i for the next block's Q S̄ into one of two shared-memory buffers;
+//   * scores / P and the output accumulator are double-buffered in TMEM.
+// MMA order per block i: QK^T -> K^T V -> Q S̄_{i-1} -> P V.  TMEM: scores
+// 2 x 128, O 2 x 64, dS 2 x 64 columns.  Shared memory: two stages of
+// Q, K (128 x 128) and V (128 x 64), S̄ 2 x 16 KiB.
+// ============================================================================
+namespace sq {
+constexpr int kNV = 64;
+constexpr int kStageB = 2 * kTileBytes + kHalfBytes;        // 80 KiB
+constexpr int kSbarOff = kStages * kStageB;                 // S̄[2], 16 KiB each
+constexpr int kCtrlOff = kSbarOff + 2 * kHalfBytes;
+constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
+constexpr uint32_t kColSP = 0;      // scores / P: 2 x 128
+constexpr uint32_t kColO = 256;     // output: 2 x 64
+constexpr uint32_t kColDS = 384;    // state increment: 2 x 64
+constexpr uint32_t kTmemCols = 512;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
+
+struct Ctrl {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tail_ld;
+    uint64_t s_full;        // MMA1 complete
+    uint64_t p_ready;       // P written (8 warps)
+    uint64_t ds_full;       // MMA4 complete
+    uint64_t ds_free[2];    // dS buffer read (8 warps)
+    uint64_t sbar_ready;    // S̄ written (8 warps)
+    uint64_t o_full;        // MMA2 complete
+    uint64_t o_free[2];     // O buffer read (8 warps)
+    uint64_t o_staged;      // O staged in shared memory (8 warps)
+    uint64_t o_stored[kStages];
+    uint32_t tmem_base;
+    int abort;
+};
+}  // namespace sq
+
+__global__ void __launch_bounds__(sq::kThreads, 1)
+prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    sq::Ctrl* ctrl = reinterpret_cast<sq::Ctrl*>(smem + sq::kCtrlOff);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t sbase = ptx::smem_u32(smem);
+    const uint32_t sSbar = sbase + sq::kSbarOff;
+    auto bar = [&](uint64_t& b) { return ptx::smem_u32(&b); };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(bar(ctrl->full[s]), 1);
+            ptx::mbar_init(bar(ctrl->empty[s]), 1);
+            ptx::mbar_init(bar(ctrl->o_stored[s]), 1);
+        }
+        ptx::mbar_init(bar(ctrl->tail_ld), 1);
+        ptx::mbar_init(bar(ctrl->s_full), 1);
+        ptx::mbar_init(bar(ctrl->p_ready), sq::kEpiWarps);
+        ptx::mbar_init(bar(ctrl->ds_full), 1);
+        ptx::mbar_init(bar(ctrl->sbar_ready), sq::kEpiWarps);
+        ptx::mbar_init(bar(ctrl->o_full), 1);
+        ptx::mbar_init(bar(ctrl->o_staged), sq::kEpiWarps);
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(bar(ctrl->ds_free[b]), sq::kEpiWarps);
+            ptx::mbar_init(bar(ctrl->o_free[b]), sq::kEpiWarps);
+        }
+        ctrl->abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(ptx::smem_u32(&ctrl->tmem_base), sq::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&tmQ);
+        ptx::prefetch_tmap(&tmK);
+        ptx::prefetch_tmap(&tmV);
+        ptx::prefetch_tmap(&tmO);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = ctrl->tmem_base;
+    volatile int* abort_flag = &ctrl->abort;
+    const int n_items = num_items(p);
+    const bool packed = p.mode == kModeVarlen;
+    const int stride = gridDim.x;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        const uint64_t pol = ptx::policy_evict_first();
+        uint32_t g = 0, n_tail = 0;
+        uint32_t c_uses[kStages] = {0, 0};
+        bool ok = true;
+        for (int item = blockIdx.x; ok && item < n_items; item += stride) {
+            const Item it = get_item(p, item);
+            for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
+                const int s = g & 1;
+                if (g >= 2) {
+                    int w = 1;
+                    if (lane == 0) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
+                    if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+                }
+                if (c_uses[s] > 0) {
+                    // the Q slot also staged the O tile of that stage's previous block
+                    int w = 1;
+                    if (lane == 0) w = ptx::mbar_wait(bar(ctrl->o_stored[s]), (c_uses[s] - 1) & 1, abort_flag);
+                    if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+                }
+                ++c_uses[s];
+                if (!produce_tile<true, 1>(&tmQ, &tmK, &tmV, smem + s * sq::kStageB, sbase + s * sq::kStageB,
+                                           bar(ctrl->full[s]), bar(ctrl->tail_ld), n_tail, t, it.z,
+                                           it.t1 - t, packed, pol, pol, lane, abort_flag, it.vp * sq::kNV))
+                    ok = false;
+            }
+        }
+        if (lane == 0) {
+            for (uint32_t j = (g >= 2 ? g - 2 : 0); ok && j < g; ++j)
+                ok = ptx::mbar_wait(bar(ctrl->empty[j & 1]), (j >> 1) & 1, abort_flag);
+            for (int s = 0; ok && s < kStages; ++s)
+                if (c_uses[s] > 0) ok = ptx::mbar_wait(bar(ctrl->o_stored[s]), (c_uses[s] - 1) & 1, abort_flag);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_qk = ptx::idesc_bf16(128, 128, false, false);  // Q K^T
+            constexpr uint32_t id_qs = ptx::idesc_bf16(128, sq::kNV, false, true);   // Q S̄
+            constexpr uint32_t id_kv = ptx::idesc_bf16(128, sq::kNV, true, true);    // K^T V
+            constexpr uint32_t id_pv = ptx::idesc_bf16(128, sq::kNV, false, true);   // P V
+            uint32_t g = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < n_items; item += stride) {
+                const Item it = get_item(p, item);
+                bool has_state = p.prefix != nullptr && it.c > 0;
+                for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
+                    const int s = g & 1;
+                    const uint32_t b = g & 1;
+                    if (!ptx::mbar_wait(bar(ctrl->full[s]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t sq_ = sbase + s * sq::kStageB;
+                    const uint32_t sk = sq_ + kTileBytes;
+                    const uint32_t sv = sq_ + 2 * kTileBytes;
+                    const uint32_t sp_cols = tmem + sq::kColSP + b * 128;
+                    // MMA1: scores = Q K^T into buffer b (its previous P, of block g-2,
+                    // was consumed by an MMA issued earlier by this thread)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+                        ptx::mma_ss(sp_cols, ptx::sdesc_sw128(sq_ + off, 16, 1024),
+                                    ptx::sdesc_sw128(sk + off, 16, 1024), id_qk, kk > 0);
+                    }
+                    ptx::mma_commit(bar(ctrl->s_full));
+                    // MMA4: dS = K^T V into buffer b, once block g-2's dS has been read
+                    if (g >= 2 && !ptx::mbar_wait(bar(ctrl->ds_free[b]), ((g >> 1) + 1) & 1, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        ptx::mma_ss(tmem + sq::kColDS + b * sq::kNV, ptx::sdesc_sw128(sk + kk * 2048, kHalfBytes, 1024),
+                                    ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_kv, kk > 0);
+                    ptx::mma_commit(bar(ctrl->ds_full));
+                    // MMA3: O = Q S̄_{g-1} into buffer b (S̄ buffer (g-1) & 1)
+                    if (!ptx::mbar_wait(bar(ctrl->sbar_ready), g & 1, abort_flag)) { ok = false; break; }
+                    if (g >= 2 && !ptx::mbar_wait(bar(ctrl->o_free[b]), ((g >> 1) + 1) & 1, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t o_cols = tmem + sq::kColO + b * sq::kNV;
+                    if (has_state) {
+                        const uint32_t sb = sSbar + ((g + 1) & 1) * kHalfBytes;
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+                            ptx::mma_ss(o_cols, ptx::sdesc_sw128(sq_ + off, 16, 1024),
+                                        ptx::sdesc_sw128(sb + kk * 2048, kHalfBytes, 1024), id_qs, kk > 0);
+                        }
+                    }
+                    // MMA2: O += P V (P in TMEM buffer b)
+                    if (!ptx::mbar_wait(bar(ctrl->p_ready), g & 1, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        ptx::mma_ts(o_cols, tmem + sq::kColSP + b * 128 + p_col(kk) - kColS,
+                                    ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_pv,
+                                    (kk > 0 || has_state) ? 1u : 0u);
+                    ptx::mma_commit(bar(ctrl->o_full));
+                    ptx::mma_commit(bar(ctrl->empty[s]));
+                    has_state = true;
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - 2;             // 0..7
+        const int sp = warp & 3;             // TMEM sub-partition of this warp
+        const int r = sp * 32 + lane;        // tile row owned by this thread
+        const int k0 = 64 * (ew >> 2);       // keys [k0, k0 + 64) for P
+        const int c0 = 32 * (ew >> 2);       // value columns [c0, c0 + 32) of this part
+        const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
+        const bool store_leader = (ew == 0 && lane == 0);
+        uint32_t g = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; ok && item < n_items; item += stride) {
+            const Item it = get_item(p, item);
+            const int vcol = it.vp * sq::kNV + c0;  // first owned column of the 128
+            // ---- running state S (row r, columns vcol..vcol+31) and S̄ for block 0
+            float srun[32];
+            if (p.prefix != nullptr && it.c > 0) {
+                const float4* src = reinterpret_cast<const float4*>(
+                    p.prefix + (size_t)it.ws * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim + vcol);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 x = __ldg(src + j);
+                    srun[4 * j + 0] = x.x;
+                    srun[4 * j + 1] = x.y;
+                    srun[4 * j + 2] = x.z;
+                    srun[4 * j + 3] = x.w;
+                }
+                uint32_t f[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
+                // S̄ buffer read by this item's first block g: (g - 1) & 1
+                store_row32_bf16_sw128(smem + sq::kSbarOff + ((g + 1) & 1) * kHalfBytes - 0, r, c0, f);
+                ptx::fence_proxy_async_smem();
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) srun[j] = 0.f;
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready));
+
+            for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
+                const bool last_block = t + kTileRows >= it.t1;
+                const int s = g & 1;
+                const uint32_t b = g & 1;
+                // ---- 1. P = tril(scores) as bf16 pairs, in place in buffer b
+                if (!ptx::mbar_wait(bar(ctrl->s_full), g & 1, abort_flag)) { ok = false; break; }
+                ptx::tc_fence_after();
+                {
+                    const uint32_t scol = tl + sq::kColSP + b * 128 + k0;
+                    uint32_t pk[32];
+                    if (k0 > sp * 32 + 31) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) pk[j] = 0u;
+                    } else {
+                        uint32_t v[64];
+                        ptx::tmem_ld32(scol, *reinterpret_cast<uint32_t(*)[32]>(v));
+                        ptx::tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                        ptx::tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int key = k0 + 2 * j;
+                            const float a = (key <= r) ? __uint_as_float(v[2 * j]) : 0.0f;
+                            const float bb = (key + 1 <= r) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
+                            pk[j] = ptx::pack_bf16x2(a, bb);
+                        }
+                    }
+                    ptx::tmem_st32(scol, pk);
+                }
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(ctrl->p_ready));
+
+                // ---- 2. S += dS_g; S̄_g for the next block, or the final state
+                if (!ptx::mbar_wait(bar(ctrl->ds_full), g & 1, abort_flag)) { ok = false; break; }
+                ptx::tc_fence_after();
+                {
+                    uint32_t d[32];
+                    ptx::tmem_ld32(tl + sq::kColDS + b * sq::kNV + c0, d);
+                    ptx::tmem_ld_wait();
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->ds_free[b]));
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) srun[j] += __uint_as_float(d[j]);
+                }
+                if (!last_block) {
+                    // buffer g & 1 was last read by MMA3 of block g-1, complete
+                    // since its o_full was observed below in the previous block
+                    uint32_t f[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
+                    store_row32_bf16_sw128(smem + sq::kSbarOff + (g & 1) * kHalfBytes, r, c0, f);
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready));
+                } else if (p.state_out != nullptr) {
+                    float4* dst = reinterpret_cast<float4*>(
+                        p.state_out + (size_t)it.sidx * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim + vcol);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        dst[j] = make_float4(srun[4 * j], srun[4 * j + 1], srun[4 * j + 2], srun[4 * j + 3]);
+                }
+
+                // ---- 3. O: registers, release buffer b, stage as bf16, TMA store
+                if (!ptx::mbar_wait(bar(ctrl->o_full), g & 1, abort_flag)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const bool rowwise = packed && t + kTileRows > it.t1;
+                uint8_t* ostage = smem + s * sq::kStageB;
+                {
+                    uint32_t v[32];
+                    ptx::tmem_ld32(tl + sq::kColO + b * sq::kNV + c0, v);
+                    ptx::tmem_ld_wait();
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_free[b]));
+                    if (!rowwise) {
+                        store_row32_bf16_sw128(ostage, r, c0, v);
+                        ptx::fence_proxy_async_smem();
+                    } else if (t + r < it.t1) {
+                        uint4* orow = reinterpret_cast<uint4*>(p.o + ((size_t)it.z * p.rows + t + r) * kHeadDim + vcol);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint4 w;
+                            w.x = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+                            w.y = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+                            w.z = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+                            w.w = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+                            orow[j] = w;
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_staged));
+                }
+                if (store_leader) {
+                    if (!ptx::mbar_wait(bar(ctrl->o_staged), g & 1, abort_flag)) ok = false;
+                    if (ok && !rowwise) {
+                        ptx::tma_store_3d(&tmO, sbase + s * sq::kStageB, it.vp * sq::kNV, t, it.z);
+                        ptx::bulk_commit_group();
+                        ptx::bulk_wait_group_read0();
+                    }
+                    ptx::mbar_arrive(bar(ctrl->o_stored[s]));
+                }
+                __syncwarp();
+                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+            }
+        }
+        if (store_leader) ptx::bulk_wait_group0();
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, sq::kTmemCols);
     }
 }
 
@@ -545,7 +1210,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                 if (!produce_tile<false>(nullptr, &tmK, &tmV, smem + s * cs::kStageBytes,
                                          sbase + s * cs::kStageBytes, bar(ctrl->full[s]),
                                          bar(ctrl->tail_ld), n_tail, t, it.z, it.t1 - t, packed, pol,
-                                         lane, abort_flag)) {
+                                         pol, lane, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -671,6 +1336,18 @@ chunk_scan_varlen_kernel(float* ws, float* state_out, const int32_t* chunk_off, 
         if (state_out != nullptr)
             reinterpret_cast<float4*>(state_out + ((size_t)j * H + hh) * (kHeadDim * kHeadDim))[e4] = acc;
     }
+}
+
+// Single pass over packed sequences: an empty sequence owns no work item, so
+// its final state is cleared here.  Grid (num_seqs, H).
+__global__ void __launch_bounds__(256)
+zero_empty_states_kernel(float* state_out, const int32_t* cu, const int* seq_ok, int H) {
+    if (*seq_ok == 0) return;
+    const int j = blockIdx.x;
+    if (cu[j + 1] != cu[j]) return;
+    float4* dst = reinterpret_cast<float4*>(state_out + ((size_t)j * H + blockIdx.y) * (kHeadDim * kHeadDim));
+    for (int e = threadIdx.x; e < kHeadDim * kHeadDim / 4; e += blockDim.x)
+        dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // cu_seqlens check and chunk offsets of packed sequences (one CTA): verdict in

@@ -52,11 +52,21 @@ def test_fp32_ternary_exact():
     assert np.array_equal(host64(st), s_ref)
 
 
+SCHEDULES = [
+    pytest.param(0, id="default"),
+    pytest.param(la.LA_FLAG_FUSED | la.LA_FLAG_NO_SPLIT_V, id="single-pass"),
+    pytest.param(la.LA_FLAG_FUSED | la.LA_FLAG_SPLIT_V, id="single-pass-splitv"),
+    pytest.param(la.LA_FLAG_THREE_PASS | la.LA_FLAG_NO_SPLIT_V, id="three-pass"),
+    pytest.param(la.LA_FLAG_THREE_PASS | la.LA_FLAG_SPLIT_V, id="three-pass-splitv"),
+]
+
+
+@pytest.mark.parametrize("flags", SCHEDULES)
 @pytest.mark.parametrize("N", [1, 2, 127, 128, 129, 255, 300, 1000, 2049])
 @pytest.mark.parametrize("chunk", [0, 128, 384])
-def test_bf16_ragged_lengths_and_chunks(N, chunk):
+def test_bf16_ragged_lengths_and_chunks(N, chunk, flags):
     q, k, v = inputs.qkv((2, 3, N, 128), dtype=torch.bfloat16, device=DEV, seed=N + chunk)
-    o, st = _run(q, k, v, 128, chunk_tokens=chunk)
+    o, st = _run(q, k, v, 128, chunk_tokens=chunk, flags=flags)
     o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
     assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16
     assert per_head_rel_err(host64(st), s_ref) <= TOL_STATE
@@ -74,12 +84,13 @@ def test_bf16_ternary_bit_exact(N, chunk):
     assert np.array_equal(host64(st), s_ref)
 
 
-@pytest.mark.parametrize("chunk", [0, 1024, 8192])
-def test_bf16_onehot_long_bit_exact(chunk):
+@pytest.mark.parametrize("flags", SCHEDULES)
+@pytest.mark.parametrize("chunk", [0, 128, 1024, 8192])
+def test_bf16_onehot_long_bit_exact(chunk, flags):
     # one nonzero per key row keeps every state entry a small integer, so even
-    # the multi-chunk path (chunk states, scan, prefix start) is exact.
+    # the multi-chunk paths (look-back chain, or chunk states + scan) are exact.
     q, k, v = inputs.onehot_k_qkv((1, 4, 8192, 128), dtype=torch.bfloat16, device=DEV, seed=11)
-    o, st = _run(q, k, v, 128, chunk_tokens=chunk)
+    o, st = _run(q, k, v, 128, chunk_tokens=chunk, flags=flags)
     o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
     assert np.max(np.abs(s_ref)) <= 256
     assert np.array_equal(host64(o), round_like(o_ref, torch.bfloat16))
@@ -141,3 +152,36 @@ def test_without_state_output():
     assert st is None and la.la_get_last_error() == la.LA_OK
     o_ref, _ = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
     assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16
+
+
+@pytest.mark.parametrize("split", [la.LA_FLAG_NO_SPLIT_V, la.LA_FLAG_SPLIT_V])
+@pytest.mark.parametrize("BH,N", [(1, 16384), (3, 5000), (200, 1000)])
+def test_bf16_single_pass_long_chains(BH, N, split):
+    # 128-token chunks: every chunk waits for its predecessor's published
+    # prefix, the chains run through many CTAs (one head: 128 links).
+    q, k, v = inputs.onehot_k_qkv((1, BH, N, 128), dtype=torch.bfloat16, device=DEV, seed=BH)
+    o, st = _run(q, k, v, 128, chunk_tokens=128, flags=la.LA_FLAG_FUSED | split)
+    o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert np.array_equal(host64(o), round_like(o_ref, torch.bfloat16))
+    assert np.array_equal(host64(st), s_ref)
+
+
+def test_bf16_schedules_agree():
+    q, k, v = inputs.qkv((2, 8, 6000, 128), dtype=torch.bfloat16, device=DEV, seed=17)
+    o1, s1 = _run(q, k, v, 128, chunk_tokens=1024, flags=la.LA_FLAG_THREE_PASS | la.LA_FLAG_NO_SPLIT_V)
+    for fl in (la.LA_FLAG_FUSED | la.LA_FLAG_NO_SPLIT_V, la.LA_FLAG_FUSED | la.LA_FLAG_SPLIT_V,
+               la.LA_FLAG_THREE_PASS | la.LA_FLAG_SPLIT_V):
+        o2, s2 = _run(q, k, v, 128, chunk_tokens=1024, flags=fl)
+        # same chunking: the starting states agree up to fp32 summation order
+        assert per_head_rel_err(host64(o2), host64(o1)) <= 1e-2
+        assert per_head_rel_err(host64(s2), host64(s1)) <= 1e-5
+
+
+@pytest.mark.parametrize("flags", SCHEDULES)
+def test_bf16_prefill_config_all_heads_schedules(flags):
+    # B=4, H=16, N=8192 in every schedule, all heads
+    q, k, v = inputs.qkv((4, 16, 8192, 128), dtype=torch.bfloat16, device=DEV, seed=3)
+    o, st = _run(q, k, v, 128, flags=flags)
+    o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16
+    assert per_head_rel_err(host64(st), s_ref) <= TOL_STATE

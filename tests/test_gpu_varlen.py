@@ -48,17 +48,25 @@ def test_bad_seqlens_detected_on_device(bad):
 from _util import TOL_O_BF16, round_like  # noqa: E402
 
 
+SCHEDULES = [pytest.param(0, id="single-pass"), pytest.param(la.LA_FLAG_THREE_PASS, id="three-pass")]
+
+
+@pytest.mark.parametrize("flags", SCHEDULES)
+@pytest.mark.parametrize("chunk", [0, 256])
 @pytest.mark.parametrize("lens", [
     [5, 0, 130, 1, 64, 257],
     [128, 127, 129, 1, 0, 0, 1000],
     [3000, 1, 2049, 5000],
+    [0, 0, 7],
 ])
-def test_varlen_bf16(lens):
+def test_varlen_bf16(lens, chunk, flags):
     cu = _cu(lens)
     H, T = 3, sum(lens)
     q, k, v = inputs.qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=len(lens))
     o = torch.full_like(q, 5.0)
-    o, st = la.prefill_varlen(q, k, v, cu, blk=128, out=o)
+    st = torch.full((len(lens), H, 128, 128), 5.0, device=DEV)
+    o, st = la.prefill_varlen(q, k, v, cu, blk=128, out=o, state_out=st, chunk_tokens=chunk,
+                              flags=flags)
     assert la.la_get_last_error() == la.LA_OK
     o_ref, s_ref = oracle.prefill_varlen(host64(q), host64(k), host64(v), cu.cpu().numpy())
     assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16
@@ -68,14 +76,16 @@ def test_varlen_bf16(lens):
             assert not torch.any(st[j])
 
 
-def test_varlen_bf16_onehot_bit_exact():
+@pytest.mark.parametrize("flags", SCHEDULES)
+@pytest.mark.parametrize("chunk", [0, 128, 640])
+def test_varlen_bf16_onehot_bit_exact(chunk, flags):
     # one-hot keys keep all intermediates small integers: the packed path,
     # including sequences longer than one chunk and ragged tails, is exact.
     lens = [2500, 1, 4097, 0, 1300, 128, 9000]
     cu = _cu(lens)
     H, T = 2, sum(lens)
     q, k, v = inputs.onehot_k_qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=21)
-    o, st = la.prefill_varlen(q, k, v, cu, blk=128)
+    o, st = la.prefill_varlen(q, k, v, cu, blk=128, chunk_tokens=chunk, flags=flags)
     assert la.la_get_last_error() == la.LA_OK
     o_ref, s_ref = oracle.prefill_varlen(host64(q), host64(k), host64(v), cu.cpu().numpy())
     assert np.array_equal(host64(o), round_like(o_ref, torch.bfloat16))
