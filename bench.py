@@ -326,6 +326,27 @@ def bench_secondary(args, device, stream, peaks):
     solo = _Solo()
     out = {}
 
+    # -- the headline prefill with 64-token blocks (B=4 H=16 N=8192 d=128 blk=64)
+    q, k, v = inputs.qkv((B, H, N, D), dtype=torch.bfloat16, device=device, seed=0)
+    o = torch.empty_like(q)
+    st = torch.empty((B, H, D, D), dtype=torch.float32, device=device)
+    n64 = 200
+    la.la_timing_enable(n64 * 4 + 64)
+    ms = timed(stream, lambda: la.prefill(q, k, v, blk=64, out=o, state_out=st), n64, 5, solo, device)
+    kt = kernel_times(la)
+    la.la_timing_enable(0)
+    main64 = kt.get("prefill_tc_kernel", {"total_ms": float("nan"), "launches": 1})
+    k_ms = main64["total_ms"] / max(main64["launches"], 1)
+    out["prefill_blk64"] = {
+        "workload": f"prefill bf16 B={B} H={H} N={N} d={D} blk=64",
+        "tokens_per_s": round(B * N / (ms / n64 / 1e3), 1), "ms_per_step": round(ms / n64, 5),
+        "hbm_frac": round(B * H * N * BYTES_PER_TOKEN_HEAD / (k_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+        "tensor_frac": round(B * H * N * (4 * 64 * D + 4 * D * D) / (ms / n64 / 1e3) / 1e12 /
+                             peaks["bf16_tflops"], 4),
+        "kernels": {k_: round(v_["total_ms"] / max(v_["launches"], 1), 5) for k_, v_ in kt.items()}}
+    del q, k, v, o, st
+    torch.cuda.empty_cache()
+
     # -- decode: 128 sequences x 64 heads, d=128; state from a 4096-token prefill
     n_seq, Hd, N0, steps = 128, 64, 4096, 256
     q0, k0, v0 = inputs.qkv((n_seq, Hd, N0, D), dtype=torch.bfloat16, device=device, seed=0)

@@ -84,7 +84,8 @@ int la_prefill(const void* q, const void* k, const void* v, void* o, float* stat
                                   default): each chunk publishes its inclusive
                                   state prefix for the next one              */
 #define LA_FLAG_SPLIT_V    4   /* split the value columns of every head over two
-                                  CTAs (independent halves of S and O)        */
+                                  CTAs (independent halves of S and O); blk 128
+                                  only, ignored with blk 64                    */
 #define LA_FLAG_NO_SPLIT_V 8   /* never split the value columns               */
 int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* state_out,
                   int B, int H, int N, int d, int blk, la_dtype dt, void* stream,

@@ -61,6 +61,8 @@ int device_setup(int* dev_out, int* sms_out) {
                                  tc::smem_bytes(128)) != cudaSuccess ||
             cudaFuncSetAttribute(tc::prefill_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tc::smem_bytes(64)) != cudaSuccess ||
+            cudaFuncSetAttribute(tc::prefill_tc_kernel<128, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::smem_bytes(128)) != cudaSuccess ||
             cudaFuncSetAttribute(tc::prefill_seq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tc::sq::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(tc::chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -192,10 +194,13 @@ int choose_chunk_tokens(int BH, int N, int ctas) {
 
 // Main kernel for p.vparts value parts per head (1: 128 columns per CTA, 2: 64).
 // Split value columns without a look-back chain run the sequential kernel
-// with the fully double-buffered block pipeline.
+// with the fully double-buffered block pipeline; 64-token blocks run the
+// 128-column kernel with two blocks per tile.
 void launch_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                  const CUtensorMap& to, const tc::Params& p, int grid, cudaStream_t stream) {
-    if (p.vparts == 2 && !p.fused)
+    if (p.blk == 64)
+        tc::prefill_tc_kernel<128, 64><<<grid, tc::kThreads, tc::smem_bytes(128), stream>>>(tq, tk, tv, to, p);
+    else if (p.vparts == 2 && !p.fused)
         tc::prefill_seq_kernel<<<grid, tc::sq::kThreads, tc::sq::kSmemBytes, stream>>>(tq, tk, tv, to, p);
     else if (p.vparts == 2)
         tc::prefill_tc_kernel<64><<<grid, tc::kThreads, tc::smem_bytes(64), stream>>>(tq, tk, tv, to, p);
@@ -214,6 +219,7 @@ tc::Params dense_params(int BH, int N, int chunk_tokens, void* o) {
     p.n_items = BH * p.n_chunks;
     p.o = reinterpret_cast<__nv_bfloat16*>(o);
     p.vparts = 1;
+    p.blk = 128;
     return p;
 }
 
@@ -311,18 +317,20 @@ int launch_fused(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
 int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, float* state_out,
                         int BH, int N, int blk, cudaStream_t stream, int sms, int chunk_tokens,
                         int flags) {
-    if (blk != 128) return LA_ERR_UNSUPPORTED;
+    if (blk != 128 && blk != 64) return LA_ERR_UNSUPPORTED;
     CUtensorMap tq, tk, tv, to;
     if (make_tmap_bf16(&tq, q, N, BH) || make_tmap_bf16(&tk, k, N, BH) ||
         make_tmap_bf16(&tv, v, N, BH) || make_tmap_bf16(&to, o, N, BH))
         return LA_ERR_CUDA;
     const bool three_pass = (flags & LA_FLAG_THREE_PASS) != 0;
-    const int vparts = want_split_v(BH, N, sms, flags) ? 2 : 1;
+    // 64-token blocks keep all 128 value columns in one CTA
+    const int vparts = (blk == 128 && want_split_v(BH, N, sms, flags)) ? 2 : 1;
     if (!three_pass) {
         if (chunk_tokens <= 0) chunk_tokens = choose_fused_chunk_tokens(BH * vparts, N, sms);
         chunk_tokens = ((chunk_tokens + kTileRows - 1) / kTileRows) * kTileRows;
         tc::Params p = dense_params(BH, N, chunk_tokens, o);
         p.vparts = vparts;
+        p.blk = blk;
         p.n_items *= vparts;
         const int grid = std::min(p.n_items, sms);
         return launch_fused(tq, tk, tv, to, p, p.n_chunks > 1 ? (long)BH * p.n_chunks : 0, state_out,
@@ -332,6 +340,7 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
     chunk_tokens = ((chunk_tokens + kTileRows - 1) / kTileRows) * kTileRows;
     tc::Params p = dense_params(BH, N, chunk_tokens, o);
     p.vparts = vparts;
+    p.blk = blk;
     p.n_items *= vparts;
     const int grid = std::min(p.n_items, sms);
 
@@ -377,7 +386,7 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
                                float* state_out, const int32_t* cu_seqlens, int num_seqs, int T,
                                int H, int blk, cudaStream_t stream, int sms, bool three_pass,
                                int chunk_tokens) {
-    if (blk != 128) return LA_ERR_UNSUPPORTED;
+    if (blk != 128 && blk != 64) return LA_ERR_UNSUPPORTED;
     if (chunk_tokens <= 0)
         chunk_tokens = three_pass ? choose_varlen_chunk_tokens(H, std::max(T, 1), sms)
                                   : choose_varlen_fused_chunk_tokens(H, std::max(T, 1), sms);
@@ -410,6 +419,7 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
     std::memset(&p, 0, sizeof(p));
     p.mode = tc::kModeVarlen;
     p.vparts = 1;
+    p.blk = blk;
     p.Z = H;
     p.rows = rows;
     p.chunk_tokens = chunk_tokens;
@@ -501,7 +511,7 @@ int noalloc_scratch(int dev, float** out) {
 int launch_prefill_bf16_noalloc(const void* q, const void* k, const void* v, void* o,
                                 float* state_out, int BH, int N, int blk, cudaStream_t stream,
                                 int dev, int sms) {
-    if (blk != 128) return LA_ERR_UNSUPPORTED;
+    if (blk != 128 && blk != 64) return LA_ERR_UNSUPPORTED;
     int chunk_tokens = choose_chunk_tokens(BH, N, sms);
     const int n_chunks = (N + chunk_tokens - 1) / chunk_tokens;
     const size_t ws_bytes = (size_t)BH * n_chunks * kHeadDim * kHeadDim * sizeof(float);
@@ -516,6 +526,7 @@ int launch_prefill_bf16_noalloc(const void* q, const void* k, const void* v, voi
         make_tmap_bf16(&tv, v, N, BH) || make_tmap_bf16(&to, o, N, BH))
         return LA_ERR_CUDA;
     tc::Params p = dense_params(BH, N, chunk_tokens, o);
+    p.blk = blk;
     const int grid = std::min(p.n_items, sms);
     if (n_chunks > 1) {
         launch_three_pass(tq, tk, tv, to, p, ws, state_out, grid, stream);

@@ -64,6 +64,12 @@ __host__ __device__ constexpr uint32_t p_col(int kk) {
     return kColS + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
 }
 
+// Same for 64-token blocks (scores 64 x 64): keys [32h, 32h+32) are packed
+// into columns [32h, 32h+16) of the score area.
+__host__ __device__ constexpr uint32_t p_col64(int kk) {
+    return kColS + (kk < 2 ? kk * 8 : 32 + (kk - 2) * 8);
+}
+
 // 14 warps: warp 0 producer, warp 1 MMA issuer, warps 2-9 epilogue, warps
 // 10-13 chain warps.
 constexpr int kEpiWarps = 8;       // P / S̄ / O / final state: 64 columns of one row per thread
@@ -116,6 +122,7 @@ struct Params {
     int* flags;                 // single pass: "prefix published" words, one per chunk,
                                 // value part and chain warp ([chunks][vparts][4], zeroed)
     int vparts;                 // value columns split over this many CTAs (1 or 2)
+    int blk;                    // block size of the intra/inter split: 128, or 64 (vparts 1)
 };
 
 // One work item: rows [t0, t1) of slice z, chunk c of its sequence, value
@@ -269,12 +276,19 @@ __device__ __forceinline__ bool produce_tile(const CUtensorMap* tmQ, const CUten
 // head are split over p.vparts = 2 CTAs).  Columns of S and O are independent
 // (S[:, v] = sum k^T v[v], O[:, v] = Q S[:, v] + P V[:, v]), so a split needs
 // no exchange; both parts compute the scores Q K^T.
-template <int kNV>
+//
+// kBlk: block size of the intra/inter split, 128 or 64.  With 64, each 128-row
+// tile is processed as two 64-token blocks: scores Q_b K_b^T (64 x 64), Q_b S̄
+// and P_b V_b run as M = 64 tcgen05 MMAs (rows in TMEM lanes 16 i .. 16 i + 15
+// of each 32-lane sub-partition i), and the state is updated every 64 tokens.
+template <int kNV, int kBlk = 128>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const Params p) {
     static_assert(kNV == 64 || kNV == 128, "value part width");
+    static_assert(kBlk == 128 || (kBlk == 64 && kNV == 128), "block size");
+    constexpr int kSub = kTileRows / kBlk;     // blocks per 128-row tile
     constexpr int kVHalves = kNV / 64;
     constexpr int kStageB = stage_bytes(kNV);
     constexpr int kSbarOffT = sbar_offset(kNV);
@@ -395,10 +409,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t id_qk = ptx::idesc_bf16(128, 128, false, false);  // Q K^T
-            constexpr uint32_t id_qs = ptx::idesc_bf16(128, kNV, false, true);   // Q S̄
-            constexpr uint32_t id_kv = ptx::idesc_bf16(128, kNV, true, true);    // K^T V
-            constexpr uint32_t id_pv = ptx::idesc_bf16(128, kNV, false, true);   // P V
+            constexpr uint32_t id_qk = ptx::idesc_bf16(kBlk, kBlk, false, false);  // Q K^T
+            constexpr uint32_t id_qs = ptx::idesc_bf16(kBlk, kNV, false, true);    // Q S̄
+            constexpr uint32_t id_kv = ptx::idesc_bf16(128, kNV, true, true);      // K^T V
+            constexpr uint32_t id_pv = ptx::idesc_bf16(kBlk, kNV, false, true);    // P V
             uint32_t g = 0, n_sb = 0, n_a = 0, n_blk = 0;
             bool ok = true;
             // phase A: TMEM delta = K_c^T V_c over the chunk's blocks
@@ -438,56 +452,63 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     if (!ok) break;
                 }
                 bool has_state = fused ? it.c > 0 : (p.prefix != nullptr && it.c > 0);
-                for (int t = it.t0; t < it.t1; t += kTileRows, ++g, ++n_blk) {
+                for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
                     const int s = g & 1;
                     if (!ptx::mbar_wait(bar(ctrl->full[s]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
                     ptx::tc_fence_after();
                     const uint32_t sq = sbase + s * kStageB;
                     const uint32_t sk = sq + kTileBytes;
                     const uint32_t sv = sq + 2 * kTileBytes;
-                    // MMA1: scores = Q K^T (both operands K-major, K = head dim).  It
-                    // overwrites the P of the previous block, whose MMA2 was issued
-                    // earlier by this thread (tcgen05 MMAs run in issue order).
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                        ptx::mma_ss(tmem + kColS, ptx::sdesc_sw128(sq + off, 16, 1024),
-                                    ptx::sdesc_sw128(sk + off, 16, 1024), id_qk, kk > 0);
-                    }
-                    ptx::mma_commit(bar(ctrl->s_full));
-                    if (!ptx::mbar_wait(bar(ctrl->sbar_ready), n_sb++ & 1, abort_flag)) { ok = false; break; }
-                    if (n_blk > 0 && !ptx::mbar_wait(bar(ctrl->o_free), (n_blk - 1) & 1, abort_flag)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    // MMA3: O = Q S̄ (inter-block, right product); S̄ is MN-major
-                    if (has_state) {
+                    const int nsub = (kSub == 1 || it.t1 - t > kBlk) ? kSub : 1;
+                    for (int sb = 0; sb < nsub; ++sb, ++n_blk) {
+                        // rows [sb * kBlk, (sb + 1) * kBlk) of the tile: kBlk rows of
+                        // 128 bytes into each 64-column half
+                        const uint32_t roff = (uint32_t)sb * kBlk * 128;
+                        // MMA1: scores = Q K^T (both operands K-major, K = head dim).
+                        // It overwrites the P of the previous block, whose MMA2 was
+                        // issued earlier by this thread (tcgen05 MMAs run in order).
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                            ptx::mma_ss(tmem + kColO, ptx::sdesc_sw128(sq + off, 16, 1024),
-                                        ptx::sdesc_sw128(sSbar + kk * 2048, kHalfBytes, 1024), id_qs,
-                                        kk > 0);
+                            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32 + roff;
+                            ptx::mma_ss(tmem + kColS, ptx::sdesc_sw128(sq + off, 16, 1024),
+                                        ptx::sdesc_sw128(sk + off, 16, 1024), id_qk, kk > 0);
                         }
-                    }
-                    // MMA4: S += K^T V (K = tokens; both operands MN-major)
+                        ptx::mma_commit(bar(ctrl->s_full));
+                        if (!ptx::mbar_wait(bar(ctrl->sbar_ready), n_sb++ & 1, abort_flag)) { ok = false; break; }
+                        if (n_blk > 0 && !ptx::mbar_wait(bar(ctrl->o_free), (n_blk - 1) & 1, abort_flag)) { ok = false; break; }
+                        ptx::tc_fence_after();
+                        // MMA3: O = Q S̄ (inter-block, right product); S̄ is MN-major
+                        if (has_state) {
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        ptx::mma_ss(tmem + kColState, ptx::sdesc_sw128(sk + kk * 2048, kHalfBytes, 1024),
-                                    ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_kv,
-                                    (kk > 0 || has_state) ? 1u : 0u);
-                    }
-                    ptx::mma_commit(bar(ctrl->state_done));
-                    if (!ptx::mbar_wait(bar(ctrl->p_ready), n_blk & 1, abort_flag)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    // MMA2: O += P V (intra-block, left product); P from TMEM
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32 + roff;
+                                ptx::mma_ss(tmem + kColO, ptx::sdesc_sw128(sq + off, 16, 1024),
+                                            ptx::sdesc_sw128(sSbar + kk * 2048, kHalfBytes, 1024), id_qs,
+                                            kk > 0);
+                            }
+                        }
+                        // MMA4: S += K^T V (K = the block's tokens; both operands MN-major)
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        ptx::mma_ts(tmem + kColO, tmem + p_col(kk),
-                                    ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_pv,
-                                    (kk > 0 || has_state) ? 1u : 0u);
+                        for (int kk = 0; kk < kBlk / 16; ++kk) {
+                            ptx::mma_ss(tmem + kColState, ptx::sdesc_sw128(sk + roff + kk * 2048, kHalfBytes, 1024),
+                                        ptx::sdesc_sw128(sv + roff + kk * 2048, kHalfBytes, 1024), id_kv,
+                                        (kk > 0 || has_state) ? 1u : 0u);
+                        }
+                        ptx::mma_commit(bar(ctrl->state_done));
+                        if (!ptx::mbar_wait(bar(ctrl->p_ready), n_blk & 1, abort_flag)) { ok = false; break; }
+                        ptx::tc_fence_after();
+                        // MMA2: O += P V (intra-block, left product); P from TMEM
+#pragma unroll
+                        for (int kk = 0; kk < kBlk / 16; ++kk) {
+                            ptx::mma_ts(tmem + kColO, tmem + (kBlk == 128 ? p_col(kk) : p_col64(kk)),
+                                        ptx::sdesc_sw128(sv + roff + kk * 2048, kHalfBytes, 1024), id_pv,
+                                        (kk > 0 || has_state) ? 1u : 0u);
+                        }
+                        ptx::mma_commit(bar(ctrl->o_full));
+                        has_state = true;
                     }
-                    ptx::mma_commit(bar(ctrl->o_full));
+                    if (!ok) break;
                     ptx::mma_commit(bar(ctrl->empty[s]));
-                    has_state = true;
                 }
             }
         }
@@ -502,7 +523,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
         uint8_t* sbar_tile = smem + kSbarOffT;
         const bool store_leader = (ew == 0 && lane == 0);
-        uint32_t n_blk = 0;
+        uint32_t n_blk = 0, n_tile = 0;
         // tile counter of the producer (phase A and phase C tiles), to know the
         // stage a phase-C block occupies
         uint32_t g = 0;
@@ -518,115 +539,149 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 const Item nx = get_item(p, item + stride);
                 if (has_phase_a(nx)) g += n_tiles(nx);
             }
-            for (int t = it.t0; t < it.t1; t += kTileRows, ++n_blk, ++g) {
-                const bool last_block = t + kTileRows >= it.t1;
+            for (int t = it.t0; t < it.t1; t += kTileRows, ++g, ++n_tile) {
                 const int s = g & 1;
-                // ---- 1. P = tril(scores) as bf16 pairs over the first half of the
-                //         score columns this thread reads (keys c0..c0+63)
-                if (!ptx::mbar_wait(bar(ctrl->s_full), n_blk & 1, abort_flag)) { ok = false; break; }
-                ptx::tc_fence_after();
-                {
-                    uint32_t pk[32];
-                    if (k0 > sp * 32 + 31) {
-                        // every key of this half lies above the diagonal for these rows
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) pk[j] = 0u;
-                    } else {
-                        uint32_t v[64];
-                        ptx::tmem_ld32(tl + kColS + k0, *reinterpret_cast<uint32_t(*)[32]>(v));
-                        ptx::tmem_ld32(tl + kColS + k0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-                        ptx::tmem_ld_wait();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int key = k0 + 2 * j;
-                            const float a = (key <= r) ? __uint_as_float(v[2 * j]) : 0.0f;
-                            const float b = (key + 1 <= r) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
-                            pk[j] = ptx::pack_bf16x2(a, b);
-                        }
-                    }
-                    ptx::tmem_st32(tl + kColS + k0, pk);
-                }
-                ptx::tmem_st_wait();
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(ctrl->p_ready));
-
-                // ---- 2. state: bf16 copy for the next block, or the final state
-                if (!ptx::mbar_wait(bar(ctrl->state_done), n_blk & 1, abort_flag)) { ok = false; break; }
-                ptx::tc_fence_after();
-                float* final_dst = nullptr;
-                if (last_block && p.state_out != nullptr && (!fused || it.last))
-                    final_dst = p.state_out + (size_t)it.sidx * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim +
-                                it.vp * kNV + c0;
-                if (!last_block || final_dst != nullptr) {
-                    uint32_t v[kCols];
-#pragma unroll
-                    for (int q = 0; q < kCols / 32; ++q)
-                        ptx::tmem_ld32(tl + kColState + c0 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * q));
-                    ptx::tmem_ld_wait();
-                    if (!last_block) {
-#pragma unroll
-                        for (int q = 0; q < kCols / 32; ++q) store_row32_bf16_sw128(sbar_tile, r, c0 + 32 * q, v + 32 * q);
-                    } else {
-                        float4* dst = reinterpret_cast<float4*>(final_dst);
-#pragma unroll
-                        for (int j = 0; j < kCols / 4; ++j)
-                            dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-                    }
-                }
-                ptx::tc_fence_before();
-                if (!last_block) {
-                    ptx::fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready));
-                } else {
-                    // TMEM S and S̄ are no longer read for this item: the chain warps
-                    // may write the next item's starting state
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->state_free));
-                }
-
-                // ---- 3. O: load to registers, release the accumulator, convert to
-                //         bf16 into the Q slot of this block's stage (free: MMA1 and
-                //         MMA3 have completed), then one thread stores the tile with
-                //         TMA.  The last block of a packed sequence is stored row by
-                //         row instead, so that the next sequence's rows are untouched.
-                if (!ptx::mbar_wait(bar(ctrl->o_full), n_blk & 1, abort_flag)) { ok = false; break; }
-                ptx::tc_fence_after();
+                const int nsub = (kSub == 1 || it.t1 - t > kBlk) ? kSub : 1;
+                const bool last_tile = t + kTileRows >= it.t1;
+                // the last tile of a packed sequence is stored row by row, so that
+                // the next sequence's rows are untouched
                 const bool rowwise = packed && t + kTileRows > it.t1;
                 uint8_t* ostage = smem + s * kStageB;
-                {
-                    uint32_t v[kCols];
+                // this thread's row in a block's M = kBlk accumulators: row r for
+                // 128-token blocks; 16 sp + lane (lanes 0-15) for 64-token blocks
+                const int br = (kBlk == 128) ? r : 16 * sp + lane;
+                const bool row_ok = (kBlk == 128) || lane < 16;
+                for (int sb = 0; sb < nsub; ++sb, ++n_blk) {
+                    const bool last_block = last_tile && sb == nsub - 1;
+                    const int trow = sb * kBlk + br;       // row within the 128-row tile
+                    // ---- 1. P = tril(scores) as bf16 pairs over the first half of the
+                    //         score columns this thread reads
+                    if (!ptx::mbar_wait(bar(ctrl->s_full), n_blk & 1, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    if constexpr (kBlk == 128) {
+                        uint32_t pk[32];
+                        if (k0 > sp * 32 + 31) {
+                            // every key of this half lies above the diagonal for these rows
 #pragma unroll
-                    for (int q = 0; q < kCols / 32; ++q)
-                        ptx::tmem_ld32(tl + kColO + c0 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * q));
-                    ptx::tmem_ld_wait();
+                            for (int j = 0; j < 32; ++j) pk[j] = 0u;
+                        } else {
+                            uint32_t v[64];
+                            ptx::tmem_ld32(tl + kColS + k0, *reinterpret_cast<uint32_t(*)[32]>(v));
+                            ptx::tmem_ld32(tl + kColS + k0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                            ptx::tmem_ld_wait();
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                const int key = k0 + 2 * j;
+                                const float a = (key <= r) ? __uint_as_float(v[2 * j]) : 0.0f;
+                                const float b = (key + 1 <= r) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
+                                pk[j] = ptx::pack_bf16x2(a, b);
+                            }
+                        }
+                        ptx::tmem_st32(tl + kColS + k0, pk);
+                    } else {
+                        // 64 x 64 scores: warpgroup h takes keys [32h, 32h+32)
+                        const int kp0 = k0 >> 1;
+                        uint32_t pk[16];
+                        if (kp0 > 16 * sp + 15) {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                        } else {
+                            uint32_t v[32];
+                            ptx::tmem_ld32(tl + kColS + kp0, v);
+                            ptx::tmem_ld_wait();
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const int key = kp0 + 2 * j;
+                                const float a = (key <= br) ? __uint_as_float(v[2 * j]) : 0.0f;
+                                const float b = (key + 1 <= br) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
+                                pk[j] = ptx::pack_bf16x2(a, b);
+                            }
+                        }
+                        ptx::tmem_st16(tl + kColS + kp0, pk);
+                    }
+                    ptx::tmem_st_wait();
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_free));
-                    if (!rowwise) {
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->p_ready));
+
+                    // ---- 2. state: bf16 copy for the next block, or the final state
+                    if (!ptx::mbar_wait(bar(ctrl->state_done), n_blk & 1, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    float* final_dst = nullptr;
+                    if (last_block && p.state_out != nullptr && (!fused || it.last))
+                        final_dst = p.state_out + (size_t)it.sidx * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim +
+                                    it.vp * kNV + c0;
+                    if (!last_block || final_dst != nullptr) {
+                        uint32_t v[kCols];
 #pragma unroll
-                        for (int q = 0; q < kCols / 32; ++q) store_row32_bf16_sw128(ostage, r, c0 + 32 * q, v + 32 * q);
-                        ptx::fence_proxy_async_smem();
-                    } else if (t + r < it.t1) {
-                        uint4* orow = reinterpret_cast<uint4*>(
-                            p.o + ((size_t)it.z * p.rows + t + r) * kHeadDim + it.vp * kNV + c0);
+                        for (int q = 0; q < kCols / 32; ++q)
+                            ptx::tmem_ld32(tl + kColState + c0 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * q));
+                        ptx::tmem_ld_wait();
+                        if (!last_block) {
 #pragma unroll
-                        for (int j = 0; j < kCols / 8; ++j) {
-                            uint4 w;
-                            w.x = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
-                            w.y = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
-                            w.z = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
-                            w.w = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
-                            orow[j] = w;
+                            for (int q = 0; q < kCols / 32; ++q) store_row32_bf16_sw128(sbar_tile, r, c0 + 32 * q, v + 32 * q);
+                        } else {
+                            float4* dst = reinterpret_cast<float4*>(final_dst);
+#pragma unroll
+                            for (int j = 0; j < kCols / 4; ++j)
+                                dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                     __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
                         }
                     }
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_staged));
+                    ptx::tc_fence_before();
+                    if (!last_block) {
+                        ptx::fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready));
+                    } else {
+                        // TMEM S and S̄ are no longer read for this item: the chain
+                        // warps may write the next item's starting state
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(bar(ctrl->state_free));
+                    }
+
+                    // ---- 3. O: load to registers, release the accumulator, convert to
+                    //         bf16 into the Q slot of this tile's stage (the block's
+                    //         MMA1 and MMA3 have completed; a 64-token block's rows
+                    //         do not overlap the rows the other block still reads)
+                    if (!ptx::mbar_wait(bar(ctrl->o_full), n_blk & 1, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    {
+                        uint32_t v[kCols];
+#pragma unroll
+                        for (int q = 0; q < kCols / 32; ++q)
+                            ptx::tmem_ld32(tl + kColO + c0 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * q));
+                        ptx::tmem_ld_wait();
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_free));
+                        if (!rowwise) {
+                            if (row_ok) {
+#pragma unroll
+                                for (int q = 0; q < kCols / 32; ++q) store_row32_bf16_sw128(ostage, trow, c0 + 32 * q, v + 32 * q);
+                            }
+                            ptx::fence_proxy_async_smem();
+                        } else if (row_ok && t + trow < it.t1) {
+                            uint4* orow = reinterpret_cast<uint4*>(
+                                p.o + ((size_t)it.z * p.rows + t + trow) * kHeadDim + it.vp * kNV + c0);
+#pragma unroll
+                            for (int j = 0; j < kCols / 8; ++j) {
+                                uint4 w;
+                                w.x = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+                                w.y = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+                                w.z = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+                                w.w = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+                                orow[j] = w;
+                            }
+                        }
+                    }
                 }
+                if (!ok) break;
+                // ---- the tile's O rows are staged: one thread stores them with TMA
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_staged));
                 if (store_leader) {
-                    if (!ptx::mbar_wait(bar(ctrl->o_staged), n_blk & 1, abort_flag)) { ok = false; }
+                    if (!ptx::mbar_wait(bar(ctrl->o_staged), n_tile & 1, abort_flag)) { ok = false; }
                     if (ok && !rowwise) {
                         const uint32_t src = sbase + s * kStageB;
 #pragma unroll

@@ -97,7 +97,7 @@ def test_bf16_onehot_long_bit_exact(chunk, flags):
     assert np.array_equal(host64(st), s_ref)
 
 
-@pytest.mark.parametrize("blk", [128])
+@pytest.mark.parametrize("blk", [128, 64])
 def test_bf16_prefill_config_all_heads(blk):
     # B=4, H=16, N=8192, d=128: every head against the oracle, in the launch
     # configuration the benchmark times (library-chosen chunking).
@@ -119,6 +119,67 @@ def test_bf16_long_context_sampled_heads():
     o_ref, s_ref = oracle.prefill_recurrent(hq, hk, hv)
     assert per_head_rel_err(host64(o[0, heads]), o_ref) <= TOL_O_BF16
     assert per_head_rel_err(host64(st[0, heads]), s_ref) <= TOL_STATE
+
+
+# ---------------------------------------------------------------- 64-token blocks
+# blk = 64 runs each 128-row tile as two blocks of 64 tokens (M = 64 MMAs); the
+# split-value flags do not apply and are ignored.
+SCHEDULES_64 = [
+    pytest.param(0, id="default"),
+    pytest.param(la.LA_FLAG_FUSED, id="single-pass"),
+    pytest.param(la.LA_FLAG_THREE_PASS, id="three-pass"),
+]
+
+
+@pytest.mark.parametrize("flags", SCHEDULES_64)
+@pytest.mark.parametrize("N", [1, 63, 64, 65, 127, 128, 129, 191, 192, 193, 300, 1000, 2049])
+@pytest.mark.parametrize("chunk", [0, 128, 384])
+def test_bf16_blk64_ragged_lengths_and_chunks(N, chunk, flags):
+    q, k, v = inputs.qkv((2, 3, N, 128), dtype=torch.bfloat16, device=DEV, seed=N + chunk + 7)
+    o, st = _run(q, k, v, 64, chunk_tokens=chunk, flags=flags)
+    o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16
+    assert per_head_rel_err(host64(st), s_ref) <= TOL_STATE
+
+
+def test_bf16_blk64_is_its_own_rounding_path():
+    # The bf16 path rounds P and the state copy S̄ once per block: 64-token
+    # blocks take a different rounding path from 128-token blocks (so the
+    # block size is really honoured) and stay within the bf16 bar.
+    q, k, v = inputs.qkv((1, 8, 1024, 128), dtype=torch.bfloat16, device=DEV, seed=31)
+    o64, _ = _run(q, k, v, 64, chunk_tokens=1024)
+    o128, _ = _run(q, k, v, 128, chunk_tokens=1024)
+    o_ref, _ = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert per_head_rel_err(host64(o64), o_ref) <= TOL_O_BF16
+    # different block sizes give different rounding paths, not the same bits
+    assert not torch.equal(o64, o128)
+
+
+@pytest.mark.parametrize("N,chunk", [(100, 0), (256, 0), (256, 128), (200, 128), (65, 0)])
+def test_bf16_blk64_ternary_bit_exact(N, chunk):
+    q, k, v = inputs.ternary_qkv((1, 4, N, 128), dtype=torch.bfloat16, device=DEV, seed=N + 1)
+    o, st = _run(q, k, v, 64, chunk_tokens=chunk)
+    o_ref = oracle.prefill_quadratic(host64(q), host64(k), host64(v))
+    _, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert np.array_equal(host64(o), round_like(o_ref, torch.bfloat16))
+    assert np.array_equal(host64(st), s_ref)
+
+
+@pytest.mark.parametrize("flags", SCHEDULES_64)
+@pytest.mark.parametrize("chunk", [0, 128, 1024])
+def test_bf16_blk64_onehot_long_bit_exact(chunk, flags):
+    q, k, v = inputs.onehot_k_qkv((1, 4, 8192, 128), dtype=torch.bfloat16, device=DEV, seed=12)
+    o, st = _run(q, k, v, 64, chunk_tokens=chunk, flags=flags)
+    o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert np.array_equal(host64(o), round_like(o_ref, torch.bfloat16))
+    assert np.array_equal(host64(st), s_ref)
+
+
+def test_bf16_blk64_split_flags_ignored():
+    q, k, v = inputs.qkv((1, 2, 700, 128), dtype=torch.bfloat16, device=DEV, seed=8)
+    o1, s1 = _run(q, k, v, 64, chunk_tokens=256, flags=la.LA_FLAG_FUSED)
+    o2, s2 = _run(q, k, v, 64, chunk_tokens=256, flags=la.LA_FLAG_FUSED | la.LA_FLAG_SPLIT_V)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
 
 
 def test_bf16_scaling_is_exact():

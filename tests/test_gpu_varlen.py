@@ -51,6 +51,7 @@ from _util import TOL_O_BF16, round_like  # noqa: E402
 SCHEDULES = [pytest.param(0, id="single-pass"), pytest.param(la.LA_FLAG_THREE_PASS, id="three-pass")]
 
 
+@pytest.mark.parametrize("blk", [128, 64])
 @pytest.mark.parametrize("flags", SCHEDULES)
 @pytest.mark.parametrize("chunk", [0, 256])
 @pytest.mark.parametrize("lens", [
@@ -59,13 +60,13 @@ SCHEDULES = [pytest.param(0, id="single-pass"), pytest.param(la.LA_FLAG_THREE_PA
     [3000, 1, 2049, 5000],
     [0, 0, 7],
 ])
-def test_varlen_bf16(lens, chunk, flags):
+def test_varlen_bf16(lens, chunk, flags, blk):
     cu = _cu(lens)
     H, T = 3, sum(lens)
     q, k, v = inputs.qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=len(lens))
     o = torch.full_like(q, 5.0)
     st = torch.full((len(lens), H, 128, 128), 5.0, device=DEV)
-    o, st = la.prefill_varlen(q, k, v, cu, blk=128, out=o, state_out=st, chunk_tokens=chunk,
+    o, st = la.prefill_varlen(q, k, v, cu, blk=blk, out=o, state_out=st, chunk_tokens=chunk,
                               flags=flags)
     assert la.la_get_last_error() == la.LA_OK
     o_ref, s_ref = oracle.prefill_varlen(host64(q), host64(k), host64(v), cu.cpu().numpy())
@@ -76,16 +77,17 @@ def test_varlen_bf16(lens, chunk, flags):
             assert not torch.any(st[j])
 
 
+@pytest.mark.parametrize("blk", [128, 64])
 @pytest.mark.parametrize("flags", SCHEDULES)
 @pytest.mark.parametrize("chunk", [0, 128, 640])
-def test_varlen_bf16_onehot_bit_exact(chunk, flags):
+def test_varlen_bf16_onehot_bit_exact(chunk, flags, blk):
     # one-hot keys keep all intermediates small integers: the packed path,
     # including sequences longer than one chunk and ragged tails, is exact.
     lens = [2500, 1, 4097, 0, 1300, 128, 9000]
     cu = _cu(lens)
     H, T = 2, sum(lens)
     q, k, v = inputs.onehot_k_qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=21)
-    o, st = la.prefill_varlen(q, k, v, cu, blk=128, chunk_tokens=chunk, flags=flags)
+    o, st = la.prefill_varlen(q, k, v, cu, blk=blk, chunk_tokens=chunk, flags=flags)
     assert la.la_get_last_error() == la.LA_OK
     o_ref, s_ref = oracle.prefill_varlen(host64(q), host64(k), host64(v), cu.cpu().numpy())
     assert np.array_equal(host64(o), round_like(o_ref, torch.bfloat16))
