@@ -3,9 +3,9 @@
 
 Headline workload (the configuration the metric is quoted on): bf16 prefill,
 B=4, H=16, N=8192, d=128, blk=128, q,k ~ N(0,1/d), v ~ N(0,1), seed 0 (seed +
-rank under torchrun).  A step is one la_prefill call over that batch
-(chunk-state pass, scan over chunks, outputs).  Inputs (384 MiB) and outputs
-exceed the 126 MB L2, so no flush is needed between steps.
+rank under torchrun).  A step is one la_prefill call over that batch, in the
+schedule the library picks for it.  Inputs (384 MiB) and outputs exceed the
+126 MB L2, so no flush is needed between steps.
 
   value     tokens/s of the whole job with inputs resident in HBM (max over ranks)
   e2e       the same metric through the public API with the inputs copied from
@@ -18,6 +18,11 @@ exceed the 126 MB L2, so no flush is needed between steps.
 
 ``--impl reference`` times the fp64 CPU oracle (the reference arm of this
 build) on a bounded sample of the same workload.
+
+``--profile-case NAME`` runs one workload for --warmup + --steps calls with no
+timing and prints a one-line summary: the command the ncu summaries under
+profiles/ were captured with (prefill, prefill_blk64, decode, long_prefill_32k,
+varlen_32k).
 """
 from __future__ import annotations
 
@@ -436,6 +441,64 @@ def bench_secondary(args, device, stream, peaks):
     return out
 
 
+# ----------------------------------------------------------------------------- profiling
+PROFILE_CASES = {
+    "prefill": "prefill bf16 B=4 H=16 N=8192 d=128 blk=128 (the headline launch)",
+    "prefill_blk64": "prefill bf16 B=4 H=16 N=8192 d=128 blk=64",
+    "decode": "decode step, 128 seq x 64 heads, d=128, fp32 state (random state)",
+    "long_prefill_32k": "prefill bf16 B=1 H=64 N=32768 d=128 blk=128 (long-context shape, "
+                        "1/8 of the length)",
+    "varlen_32k": "packed prefill bf16 T=2^15, lengths U[1024,8192] seed 0, H=64, d=128",
+}
+
+
+def profile_case(args):
+    """Launch one workload --warmup + --steps times, untimed, for an ncu capture."""
+    import torch
+    import linear_attention_13_b200 as la
+    from linear_attention_13_b200 import inputs
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    name = args.profile_case
+    if name in ("prefill", "prefill_blk64", "long_prefill_32k"):
+        shape = (B, H, N, D) if name != "long_prefill_32k" else (1, 64, 32768, D)
+        blk = 64 if name == "prefill_blk64" else BLK
+        q, k, v = inputs.qkv(shape, dtype=torch.bfloat16, device=device, seed=0)
+        o = torch.empty_like(q)
+        st = torch.empty(shape[:2] + (D, D), dtype=torch.float32, device=device)
+
+        def call():
+            la.prefill(q, k, v, blk=blk, out=o, state_out=st)
+    elif name == "decode":
+        n_seq, Hd = 128, 64
+        S = torch.randn((n_seq, Hd, D, D), dtype=torch.float32, device=device)
+        qq, kk, vv = inputs.decode_step_inputs(n_seq, Hd, D, 1, device=device)
+        od = torch.empty((n_seq, Hd, D), dtype=torch.bfloat16, device=device)
+
+        def call():
+            la.decode_step(qq, kk, vv, S, out=od)
+    elif name == "varlen_32k":
+        Tv, Hv = 1 << 15, 64
+        lens = inputs.varlen_lengths(Tv, 1024, 8192, seed=0)
+        cu = torch.from_numpy(inputs.cu_seqlens_from_lengths(lens)).to(device)
+        q, k, v = inputs.qkv((Hv, Tv, D), dtype=torch.bfloat16, device=device, seed=0)
+        o = torch.empty_like(q)
+        st = torch.empty((len(lens), Hv, D, D), dtype=torch.float32, device=device)
+
+        def call():
+            la.prefill_varlen(q, k, v, cu, blk=BLK, out=o, state_out=st)
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    for _ in range(args.warmup + args.steps):
+        call()
+    torch.cuda.synchronize()
+    status = la.la_get_last_error()
+    print(json.dumps({"profile_case": name, "workload": PROFILE_CASES[name],
+                      "calls": args.warmup + args.steps, "status": status}), flush=True)
+    return 0 if status == la.LA_OK else 1
+
+
 # ----------------------------------------------------------------------------- oracle
 def cpu_baseline(budget_s: float = 15.0):
     """The fp64 oracle (recurrent form, OpenMP over heads) on a bounded sample
@@ -508,9 +571,12 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.profile_case is not None:
+        return profile_case(args)
     dist = Dist()
     if args.impl == "reference":
         if dist.rank != 0:

@@ -850,28 +850,34 @@ namespace sq {
 constexpr int kNV = 64;
 constexpr int kStageB = 2 * kTileBytes + kHalfBytes;        // 80 KiB
 constexpr int kSbarOff = kStages * kStageB;                 // S̄[2], 16 KiB each
-constexpr int kCtrlOff = kSbarOff + 2 * kHalfBytes;
+constexpr int kOstOff = kSbarOff + 2 * kHalfBytes;          // O staging, 16 KiB
+constexpr int kCtrlOff = kOstOff + kHalfBytes;
 constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
 constexpr uint32_t kColSP = 0;      // scores / P: 2 x 128
 constexpr uint32_t kColO = 256;     // output: 2 x 64
 constexpr uint32_t kColDS = 384;    // state increment: 2 x 64
 constexpr uint32_t kTmemCols = 512;
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr int kStoreWarp = 2 + kEpiWarps;   // TMA stores of the staged O tiles
+constexpr int kMmaBWarp = 3 + kEpiWarps;    // second MMA issuer
+constexpr int kThreads = 32 * (4 + kEpiWarps);
+constexpr int kL2Ahead = 3;                 // tiles prefetched into L2 ahead of the load
 
 struct Ctrl {
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t tail_ld;
-    uint64_t s_full;        // MMA1 complete
+    uint64_t s_full[2];     // MMA1 complete (scores buffer b)
     uint64_t p_ready;       // P written (8 warps)
-    uint64_t ds_full;       // MMA4 complete
+    uint64_t ds_full[2];    // MMA4 complete (dS buffer b)
+    uint64_t p_free[2];     // MMA2 complete: P buffer b consumed
+    uint64_t mma3_done[2];  // MMA3 (or, without a state, MMA1) of the block using buffer b
     uint64_t ds_free[2];    // dS buffer read (8 warps)
     uint64_t sbar_ready;    // S̄ written (8 warps)
     uint64_t o_full;        // MMA2 complete
     uint64_t o_free[2];     // O buffer read (8 warps)
     uint64_t o_staged;      // O staged in shared memory (8 warps)
-    uint64_t o_stored[kStages];
+    uint64_t ost_free;      // the O staging buffer has been read by its TMA store
     uint32_t tmem_base;
     int abort;
 };
@@ -892,17 +898,19 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(bar(ctrl->full[s]), 1);
-            ptx::mbar_init(bar(ctrl->empty[s]), 1);
-            ptx::mbar_init(bar(ctrl->o_stored[s]), 1);
+            ptx::mbar_init(bar(ctrl->empty[s]), 2);   // one commit from each MMA issuer
         }
+        ptx::mbar_init(bar(ctrl->ost_free), 1);
         ptx::mbar_init(bar(ctrl->tail_ld), 1);
-        ptx::mbar_init(bar(ctrl->s_full), 1);
         ptx::mbar_init(bar(ctrl->p_ready), sq::kEpiWarps);
-        ptx::mbar_init(bar(ctrl->ds_full), 1);
         ptx::mbar_init(bar(ctrl->sbar_ready), sq::kEpiWarps);
         ptx::mbar_init(bar(ctrl->o_full), 1);
         ptx::mbar_init(bar(ctrl->o_staged), sq::kEpiWarps);
         for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(bar(ctrl->s_full[b]), 1);
+            ptx::mbar_init(bar(ctrl->ds_full[b]), 1);
+            ptx::mbar_init(bar(ctrl->p_free[b]), 1);
+            ptx::mbar_init(bar(ctrl->mma3_done[b]), 1);
             ptx::mbar_init(bar(ctrl->ds_free[b]), sq::kEpiWarps);
             ptx::mbar_init(bar(ctrl->o_free[b]), sq::kEpiWarps);
         }
@@ -932,24 +940,30 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         // ------------------------------------------------------------ producer
         const uint64_t pol = ptx::policy_evict_first();
         uint32_t g = 0, n_tail = 0;
-        uint32_t c_uses[kStages] = {0, 0};
         bool ok = true;
+        // L2 prefetch of the tile `ahead` tiles after row t of the item (the
+        // loads into shared memory then find it there)
+        auto prefetch = [&](const Item& it, int t, int ahead) {
+            const int tp = t + ahead * kTileRows;
+            if (lane == 0 && tp < it.t1) {
+                ptx::tma_prefetch_3d(&tmQ, 0, tp, it.z);
+                ptx::tma_prefetch_3d(&tmQ, 64, tp, it.z);
+                ptx::tma_prefetch_3d(&tmK, 0, tp, it.z);
+                ptx::tma_prefetch_3d(&tmK, 64, tp, it.z);
+                ptx::tma_prefetch_3d(&tmV, it.vp * sq::kNV, tp, it.z);
+            }
+        };
         for (int item = blockIdx.x; ok && item < n_items; item += stride) {
             const Item it = get_item(p, item);
+            for (int j = 1; j < sq::kL2Ahead; ++j) prefetch(it, it.t0, j);
             for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
                 const int s = g & 1;
+                prefetch(it, t, sq::kL2Ahead);
                 if (g >= 2) {
                     int w = 1;
                     if (lane == 0) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
                     if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
                 }
-                if (c_uses[s] > 0) {
-                    // the Q slot also staged the O tile of that stage's previous block
-                    int w = 1;
-                    if (lane == 0) w = ptx::mbar_wait(bar(ctrl->o_stored[s]), (c_uses[s] - 1) & 1, abort_flag);
-                    if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-                }
-                ++c_uses[s];
                 if (!produce_tile<true, 1>(&tmQ, &tmK, &tmV, smem + s * sq::kStageB, sbase + s * sq::kStageB,
                                            bar(ctrl->full[s]), bar(ctrl->tail_ld), n_tail, t, it.z,
                                            it.t1 - t, packed, pol, pol, lane, abort_flag, it.vp * sq::kNV))
@@ -959,12 +973,17 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (lane == 0) {
             for (uint32_t j = (g >= 2 ? g - 2 : 0); ok && j < g; ++j)
                 ok = ptx::mbar_wait(bar(ctrl->empty[j & 1]), (j >> 1) & 1, abort_flag);
-            for (int s = 0; ok && s < kStages; ++s)
-                if (c_uses[s] > 0) ok = ptx::mbar_wait(bar(ctrl->o_stored[s]), (c_uses[s] - 1) & 1, abort_flag);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == sq::kMmaBWarp) {
+        // ------------------------------------------------------------ MMA issuers
+        // One thread issues tcgen05 MMAs at about half the tensor core's rate for
+        // these shapes, so two warps issue: A the products with Q (MMA1 scores,
+        // MMA3 inter-block), B those with V (MMA4 state increment, MMA2 P V).
+        // Every resource either one reuses is double-buffered by block parity b
+        // and guarded by a barrier of that buffer, so neither can run two blocks
+        // ahead of the other.  Both release a stage (empty[s] counts 2).
         if (lane == 0) {
+            const bool is_a = warp == 1;
             constexpr uint32_t id_qk = ptx::idesc_bf16(128, 128, false, false);  // Q K^T
             constexpr uint32_t id_qs = ptx::idesc_bf16(128, sq::kNV, false, true);   // Q S̄
             constexpr uint32_t id_kv = ptx::idesc_bf16(128, sq::kNV, true, true);    // K^T V
@@ -977,56 +996,87 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
                     const int s = g & 1;
                     const uint32_t b = g & 1;
-                    if (!ptx::mbar_wait(bar(ctrl->full[s]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
+                    const uint32_t par = (g >> 1) & 1;           // phase parity of buffer b's barriers
+                    const uint32_t prev = ((g >> 1) + 1) & 1;    // ... for block g - 2
+                    if (!ptx::mbar_wait(bar(ctrl->full[s]), par, abort_flag)) { ok = false; break; }
                     ptx::tc_fence_after();
                     const uint32_t sq_ = sbase + s * sq::kStageB;
                     const uint32_t sk = sq_ + kTileBytes;
                     const uint32_t sv = sq_ + 2 * kTileBytes;
                     const uint32_t sp_cols = tmem + sq::kColSP + b * 128;
-                    // MMA1: scores = Q K^T into buffer b (its previous P, of block g-2,
-                    // was consumed by an MMA issued earlier by this thread)
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                        ptx::mma_ss(sp_cols, ptx::sdesc_sw128(sq_ + off, 16, 1024),
-                                    ptx::sdesc_sw128(sk + off, 16, 1024), id_qk, kk > 0);
-                    }
-                    ptx::mma_commit(bar(ctrl->s_full));
-                    // MMA4: dS = K^T V into buffer b, once block g-2's dS has been read
-                    if (g >= 2 && !ptx::mbar_wait(bar(ctrl->ds_free[b]), ((g >> 1) + 1) & 1, abort_flag)) { ok = false; break; }
-                    ptx::tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        ptx::mma_ss(tmem + sq::kColDS + b * sq::kNV, ptx::sdesc_sw128(sk + kk * 2048, kHalfBytes, 1024),
-                                    ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_kv, kk > 0);
-                    ptx::mma_commit(bar(ctrl->ds_full));
-                    // MMA3: O = Q S̄_{g-1} into buffer b (S̄ buffer (g-1) & 1)
-                    if (!ptx::mbar_wait(bar(ctrl->sbar_ready), g & 1, abort_flag)) { ok = false; break; }
-                    if (g >= 2 && !ptx::mbar_wait(bar(ctrl->o_free[b]), ((g >> 1) + 1) & 1, abort_flag)) { ok = false; break; }
-                    ptx::tc_fence_after();
                     const uint32_t o_cols = tmem + sq::kColO + b * sq::kNV;
-                    if (has_state) {
-                        const uint32_t sb = sSbar + ((g + 1) & 1) * kHalfBytes;
+                    if (is_a) {
+                        // MMA1: scores = Q K^T into buffer b, once MMA2 of block g-2
+                        // has consumed the P there
+                        if (g >= 2 && !ptx::mbar_wait(bar(ctrl->p_free[b]), prev, abort_flag)) { ok = false; break; }
+                        ptx::tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
                             const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                            ptx::mma_ss(o_cols, ptx::sdesc_sw128(sq_ + off, 16, 1024),
-                                        ptx::sdesc_sw128(sb + kk * 2048, kHalfBytes, 1024), id_qs, kk > 0);
+                            ptx::mma_ss(sp_cols, ptx::sdesc_sw128(sq_ + off, 16, 1024),
+                                        ptx::sdesc_sw128(sk + off, 16, 1024), id_qk, kk > 0);
                         }
-                    }
-                    // MMA2: O += P V (P in TMEM buffer b)
-                    if (!ptx::mbar_wait(bar(ctrl->p_ready), g & 1, abort_flag)) { ok = false; break; }
-                    ptx::tc_fence_after();
+                        ptx::mma_commit(bar(ctrl->s_full[b]));
+                        // MMA3: O = Q S̄_{g-1} into buffer b (S̄ buffer (g-1) & 1), once
+                        // the epilogue has read block g-2's O there
+                        if (!ptx::mbar_wait(bar(ctrl->sbar_ready), g & 1, abort_flag)) { ok = false; break; }
+                        if (g >= 2 && !ptx::mbar_wait(bar(ctrl->o_free[b]), prev, abort_flag)) { ok = false; break; }
+                        ptx::tc_fence_after();
+                        if (has_state) {
+                            const uint32_t sb = sSbar + ((g + 1) & 1) * kHalfBytes;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        ptx::mma_ts(o_cols, tmem + sq::kColSP + b * 128 + p_col(kk) - kColS,
-                                    ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_pv,
-                                    (kk > 0 || has_state) ? 1u : 0u);
-                    ptx::mma_commit(bar(ctrl->o_full));
-                    ptx::mma_commit(bar(ctrl->empty[s]));
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+                                ptx::mma_ss(o_cols, ptx::sdesc_sw128(sq_ + off, 16, 1024),
+                                            ptx::sdesc_sw128(sb + kk * 2048, kHalfBytes, 1024), id_qs, kk > 0);
+                            }
+                        }
+                        ptx::mma_commit(bar(ctrl->mma3_done[b]));
+                        ptx::mma_commit(bar(ctrl->empty[s]));
+                    } else {
+                        // MMA4: dS = K^T V into buffer b, once block g-2's dS has been read
+                        if (g >= 2 && !ptx::mbar_wait(bar(ctrl->ds_free[b]), prev, abort_flag)) { ok = false; break; }
+                        ptx::tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            ptx::mma_ss(tmem + sq::kColDS + b * sq::kNV, ptx::sdesc_sw128(sk + kk * 2048, kHalfBytes, 1024),
+                                        ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_kv, kk > 0);
+                        ptx::mma_commit(bar(ctrl->ds_full[b]));
+                        // MMA2: O += P V (P in TMEM buffer b), after MMA3 wrote O
+                        if (!ptx::mbar_wait(bar(ctrl->p_ready), g & 1, abort_flag)) { ok = false; break; }
+                        if (!ptx::mbar_wait(bar(ctrl->mma3_done[b]), par, abort_flag)) { ok = false; break; }
+                        ptx::tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            ptx::mma_ts(o_cols, tmem + sq::kColSP + b * 128 + p_col(kk) - kColS,
+                                        ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_pv,
+                                        (kk > 0 || has_state) ? 1u : 0u);
+                        ptx::mma_commit(bar(ctrl->o_full));
+                        ptx::mma_commit(bar(ctrl->p_free[b]));
+                        ptx::mma_commit(bar(ctrl->empty[s]));
+                    }
                     has_state = true;
                 }
             }
+        }
+    } else if (warp == sq::kStoreWarp) {
+        // ------------------------------------------------------------ O stores
+        if (lane == 0) {
+            uint32_t g = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < n_items; item += stride) {
+                const Item it = get_item(p, item);
+                for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
+                    if (!ptx::mbar_wait(bar(ctrl->o_staged), g & 1, abort_flag)) { ok = false; break; }
+                    if (!(packed && t + kTileRows > it.t1)) {
+                        ptx::tma_store_3d(&tmO, sbase + sq::kOstOff, it.vp * sq::kNV, t, it.z);
+                        ptx::bulk_commit_group();
+                        ptx::bulk_wait_group_read0();
+                    }
+                    ptx::mbar_arrive(bar(ctrl->ost_free));
+                }
+            }
+            ptx::bulk_wait_group0();
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -1036,7 +1086,6 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int k0 = 64 * (ew >> 2);       // keys [k0, k0 + 64) for P
         const int c0 = 32 * (ew >> 2);       // value columns [c0, c0 + 32) of this part
         const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
-        const bool store_leader = (ew == 0 && lane == 0);
         uint32_t g = 0;
         bool ok = true;
         for (int item = blockIdx.x; ok && item < n_items; item += stride) {
@@ -1070,10 +1119,9 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
             for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
                 const bool last_block = t + kTileRows >= it.t1;
-                const int s = g & 1;
                 const uint32_t b = g & 1;
                 // ---- 1. P = tril(scores) as bf16 pairs, in place in buffer b
-                if (!ptx::mbar_wait(bar(ctrl->s_full), g & 1, abort_flag)) { ok = false; break; }
+                if (!ptx::mbar_wait(bar(ctrl->s_full[b]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
                 {
                     const uint32_t scol = tl + sq::kColSP + b * 128 + k0;
@@ -1102,7 +1150,7 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 if (lane == 0) ptx::mbar_arrive(bar(ctrl->p_ready));
 
                 // ---- 2. S += dS_g; S̄_g for the next block, or the final state
-                if (!ptx::mbar_wait(bar(ctrl->ds_full), g & 1, abort_flag)) { ok = false; break; }
+                if (!ptx::mbar_wait(bar(ctrl->ds_full[b]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
                 {
                     uint32_t d[32];
@@ -1132,11 +1180,12 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         dst[j] = make_float4(srun[4 * j], srun[4 * j + 1], srun[4 * j + 2], srun[4 * j + 3]);
                 }
 
-                // ---- 3. O: registers, release buffer b, stage as bf16, TMA store
+                // ---- 3. O: registers, release buffer b, stage as bf16 for the
+                //         store warp once it has stored the previous tile
                 if (!ptx::mbar_wait(bar(ctrl->o_full), g & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const bool rowwise = packed && t + kTileRows > it.t1;
-                uint8_t* ostage = smem + s * sq::kStageB;
+                uint8_t* ostage = smem + sq::kOstOff;
                 {
                     uint32_t v[32];
                     ptx::tmem_ld32(tl + sq::kColO + b * sq::kNV + c0, v);
@@ -1144,6 +1193,7 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_free[b]));
+                    if (g >= 1 && !ptx::mbar_wait(bar(ctrl->ost_free), (g - 1) & 1, abort_flag)) { ok = false; break; }
                     if (!rowwise) {
                         store_row32_bf16_sw128(ostage, r, c0, v);
                         ptx::fence_proxy_async_smem();
@@ -1162,20 +1212,8 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_staged));
                 }
-                if (store_leader) {
-                    if (!ptx::mbar_wait(bar(ctrl->o_staged), g & 1, abort_flag)) ok = false;
-                    if (ok && !rowwise) {
-                        ptx::tma_store_3d(&tmO, sbase + s * sq::kStageB, it.vp * sq::kNV, t, it.z);
-                        ptx::bulk_commit_group();
-                        ptx::bulk_wait_group_read0();
-                    }
-                    ptx::mbar_arrive(bar(ctrl->o_stored[s]));
-                }
-                __syncwarp();
-                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             }
         }
-        if (store_leader) ptx::bulk_wait_group0();
     }
 
     ptx::tc_fence_before();

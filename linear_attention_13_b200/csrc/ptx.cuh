@@ -133,6 +133,15 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, uint32_t src,
         : "memory");
 }
 
+// 3-D tiled prefetch global -> L2 (no shared memory, no completion).  Same
+// coordinate rules as tma_load_3d; rows outside the tensor are ignored.
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* m, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -145,6 +154,11 @@ __device__ __forceinline__ void bulk_wait_group0() {
 // Wait until every committed bulk store has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_group_read0() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Wait until at most one committed bulk store is still reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
 // ----------------------------------------------------------------- tcgen05
