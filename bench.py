@@ -60,9 +60,13 @@ def load_peaks():
 
 
 class Dist:
-    """One process per GPU (torchrun env); a no-op when WORLD_SIZE is 1."""
+    """One process per GPU (torchrun env); a no-op when WORLD_SIZE is 1.
 
-    def __init__(self, backend="nccl"):
+    The backend is NCCL on GPUs; LA_DIST_BACKEND=gloo runs the same host
+    logic (barrier, max over ranks) on CPU processes."""
+
+    def __init__(self, backend=None):
+        backend = backend or os.environ.get("LA_DIST_BACKEND", "nccl")
         self.rank = int(os.environ.get("RANK", "0"))
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -169,23 +173,37 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- ours
 def timed(stream, fn, steps, warmup, dist, device):
     """W untimed steps, then exactly `steps` timed between CUDA events on
-    `stream`, bracketed by barrier + synchronize; returns max-over-ranks ms."""
+    `stream`, bracketed by barrier + synchronize; returns max-over-ranks ms.
+    (On a CPU device -- the multi-rank host tests -- a host clock stands in
+    for the events.)"""
     import torch
+    on_gpu = getattr(device, "type", str(device)) == "cuda"
+    sync = torch.cuda.synchronize if on_gpu else (lambda: None)
     for _ in range(warmup):
         fn()
-    torch.cuda.synchronize()
+    sync()
     dist.barrier()
-    torch.cuda.synchronize()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
+    sync()
+    if on_gpu:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+    else:
+        t0 = time.perf_counter()
     for _ in range(steps):
         fn()
-    end.record(stream)
-    torch.cuda.synchronize()
+    if on_gpu:
+        end.record(stream)
+    sync()
+    ms = start.elapsed_time(end) if on_gpu else (time.perf_counter() - t0) * 1e3
     dist.barrier()
-    ms = start.elapsed_time(end)
     return dist.max(ms, device)
+
+
+def job_throughput(units_per_rank_step: float, steps: int, max_ms: float, world: int) -> float:
+    """Whole-job throughput under weak scaling: every rank processes the same
+    number of units per step; the job takes the slowest rank's time."""
+    return world * units_per_rank_step * steps / (max_ms / 1e3)
 
 
 def kernel_times(la):
@@ -234,7 +252,7 @@ def bench_ours(args, dist):
 
     ms_step = ms / args.steps
     tokens_step = B * N
-    value = dist.world * tokens_step * args.steps / (ms / 1e3)
+    value = job_throughput(tokens_step, args.steps, ms, dist.world)
     flops_step = B * H * N * FLOPS_PER_TOKEN_HEAD
     bytes_step = B * H * N * BYTES_PER_TOKEN_HEAD
     # launches during the timed region = totals minus warm-up launches (the
@@ -309,7 +327,7 @@ def bench_e2e(args, dist, device, stream, qd, kd, vd):
     ms = timed(stream, step, steps, 2, dist, device)
     h2d = 3 * qd.numel() * qd.element_size()
     d2h = do.numel() * do.element_size() + ds.numel() * 4
-    return {"value": round(dist.world * B * N * steps / (ms / 1e3), 1), "unit": UNIT,
+    return {"value": round(job_throughput(B * N, steps, ms, dist.world), 1), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 4)}
 
@@ -532,7 +550,7 @@ def bench_reference(args, dist):
     from linear_attention_13_b200 import inputs
     cores = oracle.num_threads()
     # size one step so that warm-up + timed steps stay within ~2 minutes
-    step_budget = max(0.05, 120.0 / max(args.steps + args.warmup, 1))
+    step_budget = max(0.05, args.ref_budget / max(args.steps + args.warmup, 1))
     q, k, v = inputs.qkv((1, cores, N, D), dtype=torch.bfloat16, device="cpu", seed=0)
     q, k, v = (t.to(torch.float64).numpy() for t in (q, k, v))
     t0 = time.perf_counter()
@@ -569,6 +587,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=120.0,
+                    help="seconds of oracle work for the whole --impl reference run")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None)
