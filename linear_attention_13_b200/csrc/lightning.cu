@@ -158,6 +158,20 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // 3-D bf16 tensor map over [outer][rows][128] with a {64, 128, 1} box and the
 // 128-byte swizzle; rows past `rows` read as zero.
+// [outer][rows][128] bf16 as {64 columns, rows, 2 halves, outer}: a
+// {64, 128, 2, 1} box is one whole tile in two 128B-swizzled halves.
+int make_tmap_bf16_tile(CUtensorMap* m, const void* base, uint64_t rows, uint64_t outer) {
+    cuuint64_t dims[4] = {64, (cuuint64_t)rows, 2, (cuuint64_t)outer};
+    cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, 128, (cuuint64_t)rows * kHeadDim * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)kTileRows, 2, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LA_OK : LA_ERR_CUDA;
+}
+
 int make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t outer) {
     cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows, (cuuint64_t)outer};
     cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)rows * kHeadDim * 2};
@@ -168,6 +182,15 @@ int make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t out
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? LA_OK : LA_ERR_CUDA;
+}
+
+int make_tile_maps(tc::TileMaps* m, const void* q, const void* k, const void* v, const void* o,
+                   uint64_t rows, uint64_t outer) {
+    if (make_tmap_bf16_tile(&m->q, q, rows, outer) || make_tmap_bf16_tile(&m->k, k, rows, outer) ||
+        make_tmap_bf16_tile(&m->v, v, rows, outer) || make_tmap_bf16(&m->v_half, v, rows, outer) ||
+        make_tmap_bf16(&m->o, o, rows, outer))
+        return LA_ERR_CUDA;
+    return LA_OK;
 }
 
 // Chunk length (tokens, multiple of 128) for the bf16 dense path: the
@@ -196,16 +219,15 @@ int choose_chunk_tokens(int BH, int N, int ctas) {
 // Split value columns without a look-back chain run the sequential kernel
 // with the fully double-buffered block pipeline; 64-token blocks run the
 // 128-column kernel with two blocks per tile.
-void launch_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                 const CUtensorMap& to, const tc::Params& p, int grid, cudaStream_t stream) {
+void launch_main(const tc::TileMaps& m, const tc::Params& p, int grid, cudaStream_t stream) {
     if (p.blk == 64)
-        tc::prefill_tc_kernel<128, 64><<<grid, tc::kThreads, tc::smem_bytes(128), stream>>>(tq, tk, tv, to, p);
+        tc::prefill_tc_kernel<128, 64><<<grid, tc::kThreads, tc::smem_bytes(128), stream>>>(m, p);
     else if (p.vparts == 2 && !p.fused)
-        tc::prefill_seq_kernel<<<grid, tc::sq::kThreads, tc::sq::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+        tc::prefill_seq_kernel<<<grid, tc::sq::kThreads, tc::sq::kSmemBytes, stream>>>(m, p);
     else if (p.vparts == 2)
-        tc::prefill_tc_kernel<64><<<grid, tc::kThreads, tc::smem_bytes(64), stream>>>(tq, tk, tv, to, p);
+        tc::prefill_tc_kernel<64><<<grid, tc::kThreads, tc::smem_bytes(64), stream>>>(m, p);
     else
-        tc::prefill_tc_kernel<128><<<grid, tc::kThreads, tc::smem_bytes(128), stream>>>(tq, tk, tv, to, p);
+        tc::prefill_tc_kernel<128><<<grid, tc::kThreads, tc::smem_bytes(128), stream>>>(m, p);
 }
 
 tc::Params dense_params(int BH, int N, int chunk_tokens, void* o) {
@@ -234,8 +256,8 @@ bool want_split_v(long slices, long N, int sms, int flags) {
 }
 
 // chunk states -> scan -> outputs, with the chunk states in `ws`
-void launch_three_pass(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& to, tc::Params p, float* ws, float* state_out, int grid, cudaStream_t stream) {
+void launch_three_pass(const tc::TileMaps& m, tc::Params p, float* ws, float* state_out, int grid,
+                       cudaStream_t stream) {
     p.chunk_delta = ws;
     {
         // chunk states are computed once per chunk over all value columns
@@ -244,7 +266,7 @@ void launch_three_pass(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
         pc.n_items = p.Z * p.n_chunks;
         TimedLaunch tl(LA_KERNEL_CHUNK_STATE, stream);
         tc::chunk_state_kernel<<<std::min(grid, pc.n_items), tc::cs::kThreads, tc::cs::kSmemBytes,
-                                 stream>>>(tk, tv, pc);
+                                 stream>>>(m, pc);
     }
     {
         TimedLaunch tl(LA_KERNEL_CHUNK_SCAN, stream);
@@ -255,7 +277,7 @@ void launch_three_pass(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     p.state_out = nullptr;
     {
         TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
-        launch_main(tq, tk, tv, to, p, grid, stream);
+        launch_main(m, p, grid, stream);
     }
 }
 
@@ -280,8 +302,7 @@ int choose_fused_chunk_tokens(int Z, int N, int ctas) {
 }
 
 // Single pass with look-back: one launch (plus a memset of the chunk flags).
-int launch_fused(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                 const CUtensorMap& to, tc::Params p,
+int launch_fused(const tc::TileMaps& m, tc::Params p,
                  long n_chunk_slots, float* state_out, int grid, cudaStream_t stream) {
     p.state_out = state_out;
     if (n_chunk_slots > 0) {
@@ -300,7 +321,7 @@ int launch_fused(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
         cudaMemsetAsync(p.flags, 0, flag_words * sizeof(int), stream);
         {
             TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
-            launch_main(tq, tk, tv, to, p, grid, stream);
+            launch_main(m, p, grid, stream);
         }
         const int st = note_cuda(cudaGetLastError());
         cudaFreeAsync(buf, stream);
@@ -309,7 +330,7 @@ int launch_fused(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
     p.fused = 0;
     {
         TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
-        launch_main(tq, tk, tv, to, p, grid, stream);
+        launch_main(m, p, grid, stream);
     }
     return note_cuda(cudaGetLastError());
 }
@@ -318,10 +339,8 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
                         int BH, int N, int blk, cudaStream_t stream, int sms, int chunk_tokens,
                         int flags) {
     if (blk != 128 && blk != 64) return LA_ERR_UNSUPPORTED;
-    CUtensorMap tq, tk, tv, to;
-    if (make_tmap_bf16(&tq, q, N, BH) || make_tmap_bf16(&tk, k, N, BH) ||
-        make_tmap_bf16(&tv, v, N, BH) || make_tmap_bf16(&to, o, N, BH))
-        return LA_ERR_CUDA;
+    tc::TileMaps m;
+    if (make_tile_maps(&m, q, k, v, o, N, BH)) return LA_ERR_CUDA;
     const bool three_pass = (flags & LA_FLAG_THREE_PASS) != 0;
     // 64-token blocks keep all 128 value columns in one CTA
     const int vparts = (blk == 128 && want_split_v(BH, N, sms, flags)) ? 2 : 1;
@@ -333,7 +352,7 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
         p.blk = blk;
         p.n_items *= vparts;
         const int grid = std::min(p.n_items, sms);
-        return launch_fused(tq, tk, tv, to, p, p.n_chunks > 1 ? (long)BH * p.n_chunks : 0, state_out,
+        return launch_fused(m, p, p.n_chunks > 1 ? (long)BH * p.n_chunks : 0, state_out,
                             grid, stream);
     }
     if (chunk_tokens <= 0) chunk_tokens = choose_chunk_tokens(BH * vparts, N, sms);
@@ -348,7 +367,7 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
         p.state_out = state_out;
         {
             TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
-            launch_main(tq, tk, tv, to, p, grid, stream);
+            launch_main(m, p, grid, stream);
         }
         return note_cuda(cudaGetLastError());
     }
@@ -358,7 +377,7 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
         cudaGetLastError();
         return LA_ERR_ALLOC;
     }
-    launch_three_pass(tq, tk, tv, to, p, ws, state_out, grid, stream);
+    launch_three_pass(m, p, ws, state_out, grid, stream);
     int st = note_cuda(cudaGetLastError());
     cudaFreeAsync(ws, stream);
     return st;
@@ -393,11 +412,9 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
     chunk_tokens = ((chunk_tokens + kTileRows - 1) / kTileRows) * kTileRows;
     const long max_chunks = (long)(T + chunk_tokens - 1) / chunk_tokens + num_seqs;
     if ((long)H * max_chunks > (1L << 30)) return LA_ERR_UNSUPPORTED;
-    CUtensorMap tq, tk, tv, to;
+    tc::TileMaps m;
     const int rows = std::max(T, 1);
-    if (make_tmap_bf16(&tq, q, rows, H) || make_tmap_bf16(&tk, k, rows, H) ||
-        make_tmap_bf16(&tv, v, rows, H) || make_tmap_bf16(&to, o, rows, H))
-        return LA_ERR_CUDA;
+    if (make_tile_maps(&m, q, k, v, o, rows, H)) return LA_ERR_CUDA;
     const size_t aux_bytes = ((size_t)(num_seqs + 2) * sizeof(int32_t) + 255) / 256 * 256;
     const size_t ws_bytes = (size_t)H * max_chunks * kHeadDim * kHeadDim * sizeof(float);
     const size_t flag_bytes = three_pass ? 0 : (size_t)H * max_chunks * tc::kChainWarps * sizeof(int);
@@ -445,7 +462,7 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
         p.state_out = state_out;
         {
             TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
-            launch_main(tq, tk, tv, to, p, grid, stream);
+            launch_main(m, p, grid, stream);
         }
         const int st = note_cuda(cudaGetLastError());
         cudaFreeAsync(buf, stream);
@@ -454,7 +471,7 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
     p.chunk_delta = ws;
     {
         TimedLaunch tl(LA_KERNEL_CHUNK_STATE, stream);
-        tc::chunk_state_kernel<<<grid, tc::cs::kThreads, tc::cs::kSmemBytes, stream>>>(tk, tv, p);
+        tc::chunk_state_kernel<<<grid, tc::cs::kThreads, tc::cs::kSmemBytes, stream>>>(m, p);
     }
     {
         TimedLaunch tl(LA_KERNEL_CHUNK_SCAN, stream);
@@ -465,7 +482,7 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
     p.prefix = ws;
     {
         TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
-        launch_main(tq, tk, tv, to, p, grid, stream);
+        launch_main(m, p, grid, stream);
     }
     const int st = note_cuda(cudaGetLastError());
     cudaFreeAsync(buf, stream);
@@ -521,19 +538,17 @@ int launch_prefill_bf16_noalloc(const void* q, const void* k, const void* v, voi
         const int st = noalloc_scratch(dev, &ws);
         if (st != LA_OK) return st;
     }
-    CUtensorMap tq, tk, tv, to;
-    if (make_tmap_bf16(&tq, q, N, BH) || make_tmap_bf16(&tk, k, N, BH) ||
-        make_tmap_bf16(&tv, v, N, BH) || make_tmap_bf16(&to, o, N, BH))
-        return LA_ERR_CUDA;
+    tc::TileMaps m;
+    if (make_tile_maps(&m, q, k, v, o, N, BH)) return LA_ERR_CUDA;
     tc::Params p = dense_params(BH, N, chunk_tokens, o);
     p.blk = blk;
     const int grid = std::min(p.n_items, sms);
     if (n_chunks > 1) {
-        launch_three_pass(tq, tk, tv, to, p, ws, state_out, grid, stream);
+        launch_three_pass(m, p, ws, state_out, grid, stream);
     } else {
         p.state_out = state_out;
         TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
-        launch_main(tq, tk, tv, to, p, grid, stream);
+        launch_main(m, p, grid, stream);
     }
     return note_cuda(cudaGetLastError());
 }

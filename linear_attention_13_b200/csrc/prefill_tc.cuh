@@ -209,14 +209,24 @@ __device__ __forceinline__ void zero_tail_rows(uint8_t* vtile, int valid, int la
     }
 }
 
+// Tensor maps of one call.  q, k, v describe [Z][rows][128] bf16 as
+// {64 columns, rows, 2 column halves, Z} with a {64, 128, 2, 1} box: one TMA
+// operation moves a whole 128-row tile, both 64-column halves (128B swizzle),
+// into two consecutive 16 KiB halves.  A TMA engine moves about one operation
+// per 200 ns per issuing thread, so whole-tile operations double what one
+// producer thread loads.  v_half and o are {128, rows, Z} maps with a
+// {64, 128, 1} box: one half tile of V (split value columns) or of O.
+struct TileMaps {
+    CUtensorMap q, k, v, v_half, o;
+};
+
 // Warp-wide producer step: wait until stage `s` may be refilled, then load Q
 // (optional), K and V tiles of rows [t, t+128) of slice z.  For a packed tail
 // (fewer than 128 valid rows) the load completes on `tail_ld`, the warp clears
 // the foreign rows of V and then releases `full`.  Returns false on abort.
 // The V tile holds kVHalves 64-column halves starting at column v_x.
 template <bool kLoadQ, int kVHalves = 2>
-__device__ __forceinline__ bool produce_tile(const CUtensorMap* tmQ, const CUtensorMap* tmK,
-                                             const CUtensorMap* tmV, uint8_t* stage_ptr,
+__device__ __forceinline__ bool produce_tile(const TileMaps& maps, uint8_t* stage_ptr,
                                              uint32_t stage, uint32_t full_bar, uint32_t tail_bar,
                                              uint32_t& n_tail, int t, int z, int valid,
                                              bool packed, uint64_t q_pol, uint64_t pol, int lane,
@@ -228,15 +238,14 @@ __device__ __forceinline__ bool produce_tile(const CUtensorMap* tmQ, const CUten
         ptx::mbar_arrive_expect_tx(b, kBytes);
         uint32_t dst = stage;
         if (kLoadQ) {
-            ptx::tma_load_3d(dst, tmQ, b, 0, t, z, q_pol);
-            ptx::tma_load_3d(dst + kHalfBytes, tmQ, b, 64, t, z, q_pol);
+            ptx::tma_load_4d(dst, &maps.q, b, 0, t, 0, z, q_pol);
             dst += kTileBytes;
         }
-        ptx::tma_load_3d(dst, tmK, b, 0, t, z, pol);
-        ptx::tma_load_3d(dst + kHalfBytes, tmK, b, 64, t, z, pol);
-#pragma unroll
-        for (int hv = 0; hv < kVHalves; ++hv)
-            ptx::tma_load_3d(dst + kTileBytes + hv * kHalfBytes, tmV, b, v_x + 64 * hv, t, z, pol);
+        ptx::tma_load_4d(dst, &maps.k, b, 0, t, 0, z, pol);
+        if (kVHalves == 2)
+            ptx::tma_load_4d(dst + kTileBytes, &maps.v, b, 0, t, 0, z, pol);
+        else
+            ptx::tma_load_3d(dst + kTileBytes, &maps.v_half, b, v_x, t, z, pol);
     }
     if (!tail) return true;
     int ok = 1;
@@ -283,8 +292,7 @@ __device__ __forceinline__ bool produce_tile(const CUtensorMap* tmQ, const CUten
 // of each 32-lane sub-partition i), and the state is updated every 64 tokens.
 template <int kNV, int kBlk = 128>
 __global__ void __launch_bounds__(kThreads, 1)
-prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+prefill_tc_kernel(const __grid_constant__ TileMaps maps,
                   const Params p) {
     static_assert(kNV == 64 || kNV == 128, "value part width");
     static_assert(kBlk == 128 || (kBlk == 64 && kNV == 128), "block size");
@@ -325,10 +333,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         ptx::tmem_relinquish();
     }
     if (warp == 0 && lane == 0) {
-        ptx::prefetch_tmap(&tmQ);
-        ptx::prefetch_tmap(&tmK);
-        ptx::prefetch_tmap(&tmV);
-        ptx::prefetch_tmap(&tmO);
+        ptx::prefetch_tmap(&maps.q);
+        ptx::prefetch_tmap(&maps.k);
+        ptx::prefetch_tmap(&maps.v);
+        ptx::prefetch_tmap(&maps.v_half);
+        ptx::prefetch_tmap(&maps.o);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -362,7 +371,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
                 int s;
                 if (!next_stage(s) ||
-                    !produce_tile<false, kVHalves>(nullptr, &tmK, &tmV, smem + s * kStageB + kTileBytes,
+                    !produce_tile<false, kVHalves>(maps, smem + s * kStageB + kTileBytes,
                                                    sbase + s * kStageB + kTileBytes, bar(ctrl->full[s]),
                                                    bar(ctrl->tail_ld), n_tail, t, it.z, it.t1 - t, packed,
                                                    pol_last, pol_last, lane, abort_flag, it.vp * kNV))
@@ -390,7 +399,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
                 }
                 ++c_uses[s];
-                if (!produce_tile<true, kVHalves>(&tmQ, &tmK, &tmV, smem + s * kStageB, sbase + s * kStageB,
+                if (!produce_tile<true, kVHalves>(maps, smem + s * kStageB, sbase + s * kStageB,
                                                   bar(ctrl->full[s]), bar(ctrl->tail_ld), n_tail, t, it.z,
                                                   it.t1 - t, packed, pol_first, pol_first, lane, abort_flag,
                                                   it.vp * kNV))
@@ -686,7 +695,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                         const uint32_t src = sbase + s * kStageB;
 #pragma unroll
                         for (int hv = 0; hv < kVHalves; ++hv)
-                            ptx::tma_store_3d(&tmO, src + hv * kHalfBytes, it.vp * kNV + 64 * hv, t, it.z);
+                            ptx::tma_store_3d(&maps.o, src + hv * kHalfBytes, it.vp * kNV + 64 * hv, t, it.z);
                         ptx::bulk_commit_group();
                         ptx::bulk_wait_group_read0();
                     }
@@ -884,8 +893,7 @@ struct Ctrl {
 }  // namespace sq
 
 __global__ void __launch_bounds__(sq::kThreads, 1)
-prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                    const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -922,10 +930,11 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         ptx::tmem_relinquish();
     }
     if (warp == 0 && lane == 0) {
-        ptx::prefetch_tmap(&tmQ);
-        ptx::prefetch_tmap(&tmK);
-        ptx::prefetch_tmap(&tmV);
-        ptx::prefetch_tmap(&tmO);
+        ptx::prefetch_tmap(&maps.q);
+        ptx::prefetch_tmap(&maps.k);
+        ptx::prefetch_tmap(&maps.v);
+        ptx::prefetch_tmap(&maps.v_half);
+        ptx::prefetch_tmap(&maps.o);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -946,11 +955,9 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         auto prefetch = [&](const Item& it, int t, int ahead) {
             const int tp = t + ahead * kTileRows;
             if (lane == 0 && tp < it.t1) {
-                ptx::tma_prefetch_3d(&tmQ, 0, tp, it.z);
-                ptx::tma_prefetch_3d(&tmQ, 64, tp, it.z);
-                ptx::tma_prefetch_3d(&tmK, 0, tp, it.z);
-                ptx::tma_prefetch_3d(&tmK, 64, tp, it.z);
-                ptx::tma_prefetch_3d(&tmV, it.vp * sq::kNV, tp, it.z);
+                ptx::tma_prefetch_4d(&maps.q, 0, tp, 0, it.z);
+                ptx::tma_prefetch_4d(&maps.k, 0, tp, 0, it.z);
+                ptx::tma_prefetch_3d(&maps.v_half, it.vp * sq::kNV, tp, it.z);
             }
         };
         for (int item = blockIdx.x; ok && item < n_items; item += stride) {
@@ -964,7 +971,7 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     if (lane == 0) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
                     if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
                 }
-                if (!produce_tile<true, 1>(&tmQ, &tmK, &tmV, smem + s * sq::kStageB, sbase + s * sq::kStageB,
+                if (!produce_tile<true, 1>(maps, smem + s * sq::kStageB, sbase + s * sq::kStageB,
                                            bar(ctrl->full[s]), bar(ctrl->tail_ld), n_tail, t, it.z,
                                            it.t1 - t, packed, pol, pol, lane, abort_flag, it.vp * sq::kNV))
                     ok = false;
@@ -1069,7 +1076,7 @@ prefill_seq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
                     if (!ptx::mbar_wait(bar(ctrl->o_staged), g & 1, abort_flag)) { ok = false; break; }
                     if (!(packed && t + kTileRows > it.t1)) {
-                        ptx::tma_store_3d(&tmO, sbase + sq::kOstOff, it.vp * sq::kNV, t, it.z);
+                        ptx::tma_store_3d(&maps.o, sbase + sq::kOstOff, it.vp * sq::kNV, t, it.z);
                         ptx::bulk_commit_group();
                         ptx::bulk_wait_group_read0();
                     }
@@ -1247,7 +1254,7 @@ struct Ctrl {
 }  // namespace cs
 
 __global__ void __launch_bounds__(cs::kThreads, 1)
-chunk_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+chunk_state_kernel(const __grid_constant__ TileMaps maps,
                    const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -1274,8 +1281,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         ptx::tmem_relinquish();
     }
     if (warp == 0 && lane == 0) {
-        ptx::prefetch_tmap(&tmK);
-        ptx::prefetch_tmap(&tmV);
+        ptx::prefetch_tmap(&maps.k);
+        ptx::prefetch_tmap(&maps.v);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -1300,7 +1307,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                     if (lane == 0) w = ptx::mbar_wait(bar(ctrl->empty[s]), (use - 1) & 1, abort_flag);
                     if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
                 }
-                if (!produce_tile<false>(nullptr, &tmK, &tmV, smem + s * cs::kStageBytes,
+                if (!produce_tile<false>(maps, smem + s * cs::kStageBytes,
                                          sbase + s * cs::kStageBytes, bar(ctrl->full[s]),
                                          bar(ctrl->tail_ld), n_tail, t, it.z, it.t1 - t, packed, pol,
                                          pol, lane, abort_flag)) {
