@@ -10,7 +10,8 @@ schedule the library picks for it.  Inputs (384 MiB) and outputs exceed the
   value     tokens/s of the whole job with inputs resident in HBM (max over ranks)
   e2e       the same metric through the public API with the inputs copied from
             pinned host memory and o/state copied back inside the timed region
-  roofline  the dominant kernel (prefill_tc_kernel) against measured HBM
+  roofline  the dominant kernel (the prefill output pass; the variant the
+            library dispatched is named) against measured HBM
             bandwidth: algorithmic bytes per launch / CUDA-event launch time
   secondary decode GB/s (128 seq x 64 heads, 256 steps), long-context prefill
             (B=1, H=64, N=262144), the bf16 blk=64 prefill and the packed
@@ -48,6 +49,44 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"
 
 
 # ----------------------------------------------------------------------------- env
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "prefill_seq_kernel_b4h16n8192.md")
+
+
+def kernel_source_sha256() -> str:
+    """Hash of the CUDA sources (csrc/*.cu, *.cuh): identifies the kernel
+    version an ncu capture was taken of."""
+    import hashlib
+    csrc = os.path.join(ROOT, "linear_attention_13_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def captured_traffic(kernel: str, path: str = PROFILE_SUMMARY):
+    """DRAM bytes (read + write) per launch of the headline kernel from the
+    committed ncu summary, or None when the kernel sources changed since or
+    the summary is of another kernel."""
+    try:
+        with open(path) as f:
+            text = f.read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        if ":" in line and line.startswith("- "):
+            k, v = line[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("source_sha256") != kernel_source_sha256() or fields.get("kernel") != kernel:
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -260,12 +299,13 @@ def bench_ours(args, dist):
     launches_total = sum(v["launches"] for v in ktimes.values())
     launches_timed = launches_total * args.steps // (args.steps + args.warmup)
 
-    main = ktimes.get("prefill_tc_kernel", {"total_ms": float("nan"), "launches": 1})
+    main = ktimes.get("prefill_main", {"total_ms": float("nan"), "launches": 1})
+    main_kernel = la.la_prefill_main_kernel()
     main_ms = main["total_ms"] / max(main["launches"], 1)
     achieved = bytes_step / (main_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "prefill_tc_kernel", "achieved": round(achieved, 1),
+    roofline = {"bound": "hbm", "kernel": main_kernel, "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": captured_traffic(main_kernel),
                 "algorithmic_bytes_per_launch": bytes_step,
                 "launch_ms": round(main_ms, 5)}
     step_tflops = flops_step / (ms_step / 1e3) / 1e12
@@ -358,7 +398,7 @@ def bench_secondary(args, device, stream, peaks):
     ms = timed(stream, lambda: la.prefill(q, k, v, blk=64, out=o, state_out=st), n64, 5, solo, device)
     kt = kernel_times(la)
     la.la_timing_enable(0)
-    main64 = kt.get("prefill_tc_kernel", {"total_ms": float("nan"), "launches": 1})
+    main64 = kt.get("prefill_main", {"total_ms": float("nan"), "launches": 1})
     k_ms = main64["total_ms"] / max(main64["launches"], 1)
     out["prefill_blk64"] = {
         "workload": f"prefill bf16 B={B} H={H} N={N} d={D} blk=64",

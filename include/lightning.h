@@ -147,7 +147,8 @@ int la_device_sm_count(void);
  * library makes on the current device is bracketed by a pair of CUDA events
  * recorded on the launch's own stream, into a pool of `max_launches` pairs
  * (launches beyond the pool are counted but not timed).  Kernel ids:
- *   LA_KERNEL_PREFILL_TC  main tensor-core prefill kernel (outputs)
+ *   LA_KERNEL_PREFILL_TC  main tensor-core prefill pass (outputs), whichever
+ *                         kernel variant la_prefill_main_kernel() names
  *   LA_KERNEL_CHUNK_STATE per-chunk K^T V (first pass of the chunk scan)
  *   LA_KERNEL_CHUNK_SCAN  exclusive prefix over chunk states
  *   LA_KERNEL_PREFILL_F32 fp32 CUDA-core prefill (dense and varlen)
@@ -168,6 +169,16 @@ int la_device_sm_count(void);
 int la_timing_enable(int max_launches);
 int la_timing_read(int kernel_id, double* total_ms, int* launches);
 const char* la_kernel_name(int kernel_id);
+
+/*
+ * Name of the kernel the most recent bf16 prefill call (from any thread)
+ * launched for its output pass: "prefill_tc_kernel<128>" (whole value rows,
+ * chain warps), "prefill_tc_kernel<64>" (value columns split over two CTAs,
+ * single pass with look-back), "prefill_tc_kernel<128,64>" (64-token blocks)
+ * or "prefill_seq_kernel" (value columns split, no look-back); "" before the
+ * first call.  Informational: a static string, never freed.
+ */
+const char* la_prefill_main_kernel(void);
 
 /*
  * la_prefill_noalloc -- la_prefill (bf16, d = 128) that allocates no device

@@ -48,6 +48,7 @@ LA_NUM_KERNEL_IDS = 6
 EXPORTED = ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step",
             "la_status_string", "la_get_last_error", "la_device_sm_count",
             "la_timing_enable", "la_timing_read", "la_kernel_name", "la_prefill_noalloc",
+            "la_prefill_main_kernel",
             "la_prefill_varlen_ex")
 
 LA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -86,6 +87,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.la_kernel_name.argtypes = [i]
     lib.la_kernel_name.restype = ctypes.c_char_p
+    lib.la_prefill_main_kernel.argtypes = []
+    lib.la_prefill_main_kernel.restype = ctypes.c_char_p
     for name in ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_prefill_varlen_ex",
                  "la_decode_step",
                  "la_get_last_error", "la_device_sm_count", "la_timing_enable",
@@ -158,6 +161,11 @@ def la_timing_read(kernel_id):
 
 def la_kernel_name(kernel_id):
     return load_library().la_kernel_name(kernel_id).decode()
+
+
+def la_prefill_main_kernel():
+    """Kernel the most recent bf16 prefill launched for its output pass."""
+    return load_library().la_prefill_main_kernel().decode()
 
 
 # ---------------------------------------------------------------- tensor helpers

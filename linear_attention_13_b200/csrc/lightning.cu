@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -219,15 +220,22 @@ int choose_chunk_tokens(int BH, int N, int ctas) {
 // Split value columns without a look-back chain run the sequential kernel
 // with the fully double-buffered block pipeline; 64-token blocks run the
 // 128-column kernel with two blocks per tile.
+std::atomic<const char*> g_main_kernel{""};
+
 void launch_main(const tc::TileMaps& m, const tc::Params& p, int grid, cudaStream_t stream) {
-    if (p.blk == 64)
+    if (p.blk == 64) {
+        g_main_kernel = "prefill_tc_kernel<128,64>";
         tc::prefill_tc_kernel<128, 64><<<grid, tc::kThreads, tc::smem_bytes(128), stream>>>(m, p);
-    else if (p.vparts == 2 && !p.fused)
+    } else if (p.vparts == 2 && !p.fused) {
+        g_main_kernel = "prefill_seq_kernel";
         tc::prefill_seq_kernel<<<grid, tc::sq::kThreads, tc::sq::kSmemBytes, stream>>>(m, p);
-    else if (p.vparts == 2)
+    } else if (p.vparts == 2) {
+        g_main_kernel = "prefill_tc_kernel<64>";
         tc::prefill_tc_kernel<64><<<grid, tc::kThreads, tc::smem_bytes(64), stream>>>(m, p);
-    else
+    } else {
+        g_main_kernel = "prefill_tc_kernel<128>";
         tc::prefill_tc_kernel<128><<<grid, tc::kThreads, tc::smem_bytes(128), stream>>>(m, p);
+    }
 }
 
 tc::Params dense_params(int BH, int N, int chunk_tokens, void* o) {
@@ -790,9 +798,11 @@ int la_timing_read(int kernel_id, double* total_ms, int* launches) {
     return LA_OK;
 }
 
+const char* la_prefill_main_kernel(void) { return g_main_kernel.load(); }
+
 const char* la_kernel_name(int kernel_id) {
     switch (kernel_id) {
-        case LA_KERNEL_PREFILL_TC: return "prefill_tc_kernel";
+        case LA_KERNEL_PREFILL_TC: return "prefill_main";
         case LA_KERNEL_CHUNK_STATE: return "chunk_state_kernel";
         case LA_KERNEL_CHUNK_SCAN: return "chunk_scan_kernel";
         case LA_KERNEL_PREFILL_F32: return "prefill_simt_kernel";
