@@ -224,13 +224,14 @@ struct TileMaps {
 // (optional), K and V tiles of rows [t, t+128) of slice z.  For a packed tail
 // (fewer than 128 valid rows) the load completes on `tail_ld`, the warp clears
 // the foreign rows of V and then releases `full`.  Returns false on abort.
-// The V tile holds kVHalves 64-column halves starting at column v_x.
+// The V tile holds kVHalves 64-column halves starting at column v_x.  L2
+// policies: q_pol for Q, pol for K, v_pol (0: pol) for V.
 template <bool kLoadQ, int kVHalves = 2>
 __device__ __forceinline__ bool produce_tile(const TileMaps& maps, uint8_t* stage_ptr,
                                              uint32_t stage, uint32_t full_bar, uint32_t tail_bar,
                                              uint32_t& n_tail, int t, int z, int valid,
                                              bool packed, uint64_t q_pol, uint64_t pol, int lane,
-                                             volatile int* abort_flag, int v_x = 0) {
+                                             volatile int* abort_flag, int v_x = 0, uint64_t v_pol = 0) {
     constexpr uint32_t kBytes = (kLoadQ ? 2 : 1) * kTileBytes + kVHalves * kHalfBytes;
     const bool tail = packed && valid < kTileRows;
     if (lane == 0) {
@@ -243,9 +244,9 @@ __device__ __forceinline__ bool produce_tile(const TileMaps& maps, uint8_t* stag
         }
         ptx::tma_load_4d(dst, &maps.k, b, 0, t, 0, z, pol);
         if (kVHalves == 2)
-            ptx::tma_load_4d(dst + kTileBytes, &maps.v, b, 0, t, 0, z, pol);
+            ptx::tma_load_4d(dst + kTileBytes, &maps.v, b, 0, t, 0, z, v_pol ? v_pol : pol);
         else
-            ptx::tma_load_3d(dst + kTileBytes, &maps.v_half, b, v_x, t, z, pol);
+            ptx::tma_load_3d(dst + kTileBytes, &maps.v_half, b, v_x, t, z, v_pol ? v_pol : pol);
     }
     if (!tail) return true;
     int ok = 1;
@@ -355,6 +356,9 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
         // ------------------------------------------------------------ producer
         const uint64_t pol_first = ptx::policy_evict_first();
         const uint64_t pol_last = ptx::policy_evict_last();
+        // with split value columns the other CTA of the head reads the same Q
+        // and K: keep them at normal priority, evict only the private V half early
+        const uint64_t pol_qk = p.vparts > 1 ? ptx::policy_evict_normal() : pol_first;
         uint32_t g = 0, n_tail = 0;
         bool ok = true;
         auto next_stage = [&](int& s) -> bool {
@@ -401,8 +405,8 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
                 ++c_uses[s];
                 if (!produce_tile<true, kVHalves>(maps, smem + s * kStageB, sbase + s * kStageB,
                                                   bar(ctrl->full[s]), bar(ctrl->tail_ld), n_tail, t, it.z,
-                                                  it.t1 - t, packed, pol_first, pol_first, lane, abort_flag,
-                                                  it.vp * kNV))
+                                                  it.t1 - t, packed, pol_qk, pol_qk, lane, abort_flag,
+                                                  it.vp * kNV, pol_first))
                     ok = false;
             }
         }
@@ -947,7 +951,10 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        const uint64_t pol = ptx::policy_evict_first();
+        // the other CTA of the head reads the same Q and K: normal L2 priority
+        // for them, evict-first for this CTA's own V half
+        const uint64_t pol_qk = ptx::policy_evict_normal();
+        const uint64_t pol_v = ptx::policy_evict_first();
         uint32_t g = 0, n_tail = 0;
         bool ok = true;
         // L2 prefetch of the tile `ahead` tiles after row t of the item (the
@@ -973,7 +980,8 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 }
                 if (!produce_tile<true, 1>(maps, smem + s * sq::kStageB, sbase + s * sq::kStageB,
                                            bar(ctrl->full[s]), bar(ctrl->tail_ld), n_tail, t, it.z,
-                                           it.t1 - t, packed, pol, pol, lane, abort_flag, it.vp * sq::kNV))
+                                           it.t1 - t, packed, pol_qk, pol_qk, lane, abort_flag, it.vp * sq::kNV,
+                                           pol_v))
                     ok = false;
             }
         }
