@@ -878,7 +878,8 @@ constexpr int kL2Ahead = 3;                 // tiles prefetched into L2 ahead of
 
 struct Ctrl {
     uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t empty[kStages];    // Q and K slots of stage s read (MMA1, MMA3, MMA4)
+    uint64_t v_empty[kStages];  // V slot of stage s read (MMA2)
     uint64_t tail_ld;
     uint64_t s_full[2];     // MMA1 complete (scores buffer b)
     uint64_t p_ready;       // P written (8 warps)
@@ -911,6 +912,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(bar(ctrl->full[s]), 1);
             ptx::mbar_init(bar(ctrl->empty[s]), 2);   // one commit from each MMA issuer
+            ptx::mbar_init(bar(ctrl->v_empty[s]), 1);
         }
         ptx::mbar_init(bar(ctrl->ost_free), 1);
         ptx::mbar_init(bar(ctrl->tail_ld), 1);
@@ -972,22 +974,41 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
             for (int j = 1; j < sq::kL2Ahead; ++j) prefetch(it, it.t0, j);
             for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
                 const int s = g & 1;
+                const uint32_t stage = sbase + s * sq::kStageB;
                 prefetch(it, t, sq::kL2Ahead);
-                if (g >= 2) {
-                    int w = 1;
-                    if (lane == 0) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
-                    if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+                // Q and K of block g reuse slots that block g-2's MMA1, MMA3 and MMA4
+                // have finished with; V waits for its MMA2, which comes later
+                const bool tail = packed && it.t1 - t < kTileRows;
+                const uint32_t fb = tail ? bar(ctrl->tail_ld) : bar(ctrl->full[s]);
+                int w = 1;
+                if (lane == 0) {
+                    if (g >= 2) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
+                    if (w) {
+                        ptx::mbar_arrive_expect_tx(fb, 2 * kTileBytes + kHalfBytes);
+                        ptx::tma_load_4d(stage, &maps.q, fb, 0, t, 0, it.z, pol_qk);
+                        ptx::tma_load_4d(stage + kTileBytes, &maps.k, fb, 0, t, 0, it.z, pol_qk);
+                        if (g >= 2) w = ptx::mbar_wait(bar(ctrl->v_empty[s]), ((g >> 1) + 1) & 1, abort_flag);
+                        if (w) ptx::tma_load_3d(stage + 2 * kTileBytes, &maps.v_half, fb, it.vp * sq::kNV, t, it.z, pol_v);
+                    }
                 }
-                if (!produce_tile<true, 1>(maps, smem + s * sq::kStageB, sbase + s * sq::kStageB,
-                                           bar(ctrl->full[s]), bar(ctrl->tail_ld), n_tail, t, it.z,
-                                           it.t1 - t, packed, pol_qk, pol_qk, lane, abort_flag, it.vp * sq::kNV,
-                                           pol_v))
-                    ok = false;
+                if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+                if (tail) {
+                    // a packed tail: clear the next sequence's rows of V, then release
+                    if (lane == 0) w = ptx::mbar_wait(bar(ctrl->tail_ld), n_tail & 1, abort_flag);
+                    ++n_tail;
+                    if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+                    zero_tail_rows(smem + s * sq::kStageB + 2 * kTileBytes, it.t1 - t, lane, 1);
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->full[s]));
+                }
             }
         }
         if (lane == 0) {
-            for (uint32_t j = (g >= 2 ? g - 2 : 0); ok && j < g; ++j)
+            for (uint32_t j = (g >= 2 ? g - 2 : 0); ok && j < g; ++j) {
                 ok = ptx::mbar_wait(bar(ctrl->empty[j & 1]), (j >> 1) & 1, abort_flag);
+                if (ok) ok = ptx::mbar_wait(bar(ctrl->v_empty[j & 1]), (j >> 1) & 1, abort_flag);
+            }
         }
     } else if (warp == 1 || warp == sq::kMmaBWarp) {
         // ------------------------------------------------------------ MMA issuers
@@ -1057,6 +1078,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                             ptx::mma_ss(tmem + sq::kColDS + b * sq::kNV, ptx::sdesc_sw128(sk + kk * 2048, kHalfBytes, 1024),
                                         ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_kv, kk > 0);
                         ptx::mma_commit(bar(ctrl->ds_full[b]));
+                        ptx::mma_commit(bar(ctrl->empty[s]));    // K read
                         // MMA2: O += P V (P in TMEM buffer b), after MMA3 wrote O
                         if (!ptx::mbar_wait(bar(ctrl->p_ready), g & 1, abort_flag)) { ok = false; break; }
                         if (!ptx::mbar_wait(bar(ctrl->mma3_done[b]), par, abort_flag)) { ok = false; break; }
@@ -1068,7 +1090,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                                         (kk > 0 || has_state) ? 1u : 0u);
                         ptx::mma_commit(bar(ctrl->o_full));
                         ptx::mma_commit(bar(ctrl->p_free[b]));
-                        ptx::mma_commit(bar(ctrl->empty[s]));
+                        ptx::mma_commit(bar(ctrl->v_empty[s]));  // V read
                     }
                     has_state = true;
                 }
