@@ -109,9 +109,14 @@ int la_prefill_varlen(const void* q, const void* k, const void* v, void* o, floa
                       int H, int d, int blk, la_dtype dt, void* stream);
 
 /*
- * la_prefill_varlen_ex -- la_prefill_varlen with the scheduling controls of
- * la_prefill_ex (chunk_tokens: chunk length, a multiple of 128, 0 = library
- * choice; flags: LA_FLAG_THREE_PASS or LA_FLAG_FUSED, 0 = default).
+ * la_prefill_varlen_ex -- la_prefill_varlen with scheduling controls.
+ *   chunk_tokens: chunk length of the chunked schedules, a multiple of 128,
+ *                 0 = library choice (ignored by LA_FLAG_SPLIT_V).
+ *   flags: 0 = default; LA_FLAG_THREE_PASS or LA_FLAG_FUSED pick a chunked
+ *          schedule over whole value rows (optionally with LA_FLAG_NO_SPLIT_V);
+ *          LA_FLAG_SPLIT_V (alone; bf16, blk 128) runs every (sequence, head)
+ *          unchunked with its value columns split over two CTAs, longest
+ *          sequences first.  Other combinations return LA_ERR_INVALID_ARG.
  */
 int la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o, float* state_out,
                          const int32_t* cu_seqlens, int num_seqs, int total_tokens,

@@ -409,6 +409,62 @@ int choose_varlen_chunk_tokens(int H, int T, int ctas) {
     return (int)(((target + kTileRows - 1) / kTileRows) * kTileRows);
 }
 
+// Packed sequences with the value columns of every (sequence, head) split over
+// two CTAs and no chunking: one item per (sequence, head, half), longest
+// sequences first, run by the sequential kernel.  Nothing is read twice.
+int launch_prefill_varlen_split(const void* q, const void* k, const void* v, void* o,
+                                float* state_out, const int32_t* cu_seqlens, int num_seqs, int T,
+                                int H, cudaStream_t stream, int sms) {
+    const long max_items = (long)num_seqs * H * 2;
+    if (max_items > (1L << 30)) return LA_ERR_UNSUPPORTED;
+    tc::TileMaps m;
+    const int rows = std::max(T, 1);
+    if (make_tile_maps(&m, q, k, v, o, rows, H)) return LA_ERR_CUDA;
+    const int chunk_tokens = ((rows + kTileRows - 1) / kTileRows) * kTileRows;  // >= every length
+    const size_t aux_bytes = ((size_t)(2 * num_seqs + 2) * sizeof(int32_t) + 255) / 256 * 256;
+    uint8_t* buf = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&buf), aux_bytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_ALLOC;
+    }
+    int* ok = reinterpret_cast<int*>(buf);
+    int32_t* chunk_off = reinterpret_cast<int32_t*>(buf) + 1;
+    int32_t* order = chunk_off + num_seqs + 1;
+    {
+        TimedLaunch tl(LA_KERNEL_AUX, stream);
+        tc::varlen_prepare_kernel<<<1, 256, 0, stream>>>(cu_seqlens, num_seqs, T, chunk_tokens, ok,
+                                                        chunk_off, order);
+    }
+    if (state_out != nullptr) {
+        TimedLaunch tl(LA_KERNEL_AUX, stream);
+        tc::zero_empty_states_kernel<<<dim3(num_seqs, H), 256, 0, stream>>>(state_out, cu_seqlens, ok, H);
+    }
+    tc::Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.mode = tc::kModeVarlen;
+    p.vparts = 2;
+    p.blk = 128;
+    p.Z = H;
+    p.rows = rows;
+    p.chunk_tokens = chunk_tokens;
+    p.n_items = (int)max_items;
+    p.cu_seqlens = cu_seqlens;
+    p.chunk_off = chunk_off;
+    p.seq_ok = ok;
+    p.num_seqs = num_seqs;
+    p.seq_order = order;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.state_out = state_out;
+    const int grid = (int)std::min<long>(max_items, sms);
+    {
+        TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
+        launch_main(m, p, grid, stream);
+    }
+    const int st = note_cuda(cudaGetLastError());
+    cudaFreeAsync(buf, stream);
+    return st;
+}
+
 int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void* o,
                                float* state_out, const int32_t* cu_seqlens, int num_seqs, int T,
                                int H, int blk, cudaStream_t stream, int sms, bool three_pass,
@@ -438,7 +494,7 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
     {
         TimedLaunch tl(LA_KERNEL_AUX, stream);
         tc::varlen_prepare_kernel<<<1, 256, 0, stream>>>(cu_seqlens, num_seqs, T, chunk_tokens, ok,
-                                                        chunk_off);
+                                                        chunk_off, nullptr);
     }
     tc::Params p;
     std::memset(&p, 0, sizeof(p));
@@ -618,8 +674,11 @@ int la_prefill_varlen(const void* q, const void* k, const void* v, void* o, floa
 int la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o, float* state_out,
                          const int32_t* cu_seqlens, int num_seqs, int total_tokens, int H, int d,
                          int blk, la_dtype dt, void* stream, int chunk_tokens, int flags) {
-    if ((flags & ~(LA_FLAG_THREE_PASS | LA_FLAG_FUSED)) != 0 ||
-        flags == (LA_FLAG_THREE_PASS | LA_FLAG_FUSED) || chunk_tokens < 0)
+    constexpr int kAllFlags = LA_FLAG_THREE_PASS | LA_FLAG_FUSED | LA_FLAG_SPLIT_V | LA_FLAG_NO_SPLIT_V;
+    if ((flags & ~kAllFlags) != 0 ||
+        (flags & (LA_FLAG_THREE_PASS | LA_FLAG_FUSED)) == (LA_FLAG_THREE_PASS | LA_FLAG_FUSED) ||
+        (flags & (LA_FLAG_SPLIT_V | LA_FLAG_NO_SPLIT_V)) == (LA_FLAG_SPLIT_V | LA_FLAG_NO_SPLIT_V) ||
+        ((flags & LA_FLAG_SPLIT_V) && (flags & (LA_FLAG_THREE_PASS | LA_FLAG_FUSED))) || chunk_tokens < 0)
         return LA_ERR_INVALID_ARG;
     if (num_seqs < 1 || total_tokens < 0 || H < 1 || cu_seqlens == nullptr) return LA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return LA_ERR_INVALID_ARG;
@@ -630,6 +689,9 @@ int la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o, f
     st = device_setup(&dev, &sms);
     if (st != LA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dt == LA_BF16 && blk == 128 && (flags & LA_FLAG_SPLIT_V))
+        return launch_prefill_varlen_split(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens,
+                                           H, s, sms);
     if (dt == LA_BF16)
         return launch_prefill_varlen_bf16(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens,
                                           H, blk, s, sms, (flags & LA_FLAG_THREE_PASS) != 0,

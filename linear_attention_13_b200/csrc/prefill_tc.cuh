@@ -123,6 +123,8 @@ struct Params {
                                 // value part and chain warp ([chunks][vparts][4], zeroed)
     int vparts;                 // value columns split over this many CTAs (1 or 2)
     int blk;                    // block size of the intra/inter split: 128, or 64 (vparts 1)
+    const int32_t* seq_order;   // packed, one chunk per sequence: the sequence of chunk g
+                                // (non-empty sequences, longest first), or null
 };
 
 // One work item: rows [t0, t1) of slice z, chunk c of its sequence, value
@@ -156,6 +158,16 @@ __device__ __forceinline__ Item get_item(const Params& p, int item) {
         it.ws = it.z * p.n_chunks + g;
         it.sidx = it.z;
         it.last = g == p.n_chunks - 1;
+    } else if (p.seq_order != nullptr) {
+        // one chunk per sequence, longest sequences first (so that the work
+        // of a persistent grid is balanced)
+        const int j = p.seq_order[g];
+        it.c = 0;
+        it.t0 = p.cu_seqlens[j];
+        it.t1 = p.cu_seqlens[j + 1];
+        it.ws = it.z * p.chunk_off[p.num_seqs] + g;
+        it.sidx = j * p.Z + it.z;
+        it.last = true;
     } else {
         // sequence j with chunk_off[j] <= g < chunk_off[j+1] (empty sequences
         // own no chunk and are skipped by taking the largest such j)
@@ -1484,8 +1496,12 @@ zero_empty_states_kernel(float* state_out, const int32_t* cu, const int* seq_ok,
 // *ok, chunk_off[j] = sum over earlier sequences of ceil(len / chunk_tokens),
 // chunk_off[num_seqs] = chunks per head.  A malformed array records
 // LA_ERR_BAD_SEQLENS and yields zero chunks.
+// Check cu_seqlens and number the chunks of every sequence (chunk_off).  With
+// `order` non-null (one chunk per sequence: chunk_tokens >= every length) it
+// also lists the non-empty sequences longest first, ties by index: a
+// persistent grid that walks items in that order takes the long ones first.
 __global__ void varlen_prepare_kernel(const int32_t* cu, int num_seqs, int total, int chunk_tokens,
-                                      int* ok, int32_t* chunk_off) {
+                                      int* ok, int32_t* chunk_off, int32_t* order) {
     __shared__ int bad;
     if (threadIdx.x == 0) bad = 0;
     __syncthreads();
@@ -1509,6 +1525,19 @@ __global__ void varlen_prepare_kernel(const int32_t* cu, int num_seqs, int total
         }
         chunk_off[num_seqs] = acc;
         *ok = bad ? 0 : 1;
+    }
+    if (order == nullptr) return;
+    __syncthreads();
+    if (bad) return;
+    for (int j = threadIdx.x; j < num_seqs; j += blockDim.x) {
+        const int len = cu[j + 1] - cu[j];
+        if (len == 0) continue;
+        int rank = 0;
+        for (int i = 0; i < num_seqs; ++i) {
+            const int li = cu[i + 1] - cu[i];
+            rank += (li > len || (li == len && i < j)) ? 1 : 0;
+        }
+        order[rank] = j;   // empty sequences rank after every non-empty one
     }
 }
 

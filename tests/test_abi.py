@@ -84,6 +84,19 @@ def test_varlen_and_decode_argument_validation(lib):
                              None) == la.LA_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("flags", [
+    la.LA_FLAG_SPLIT_V | la.LA_FLAG_THREE_PASS,
+    la.LA_FLAG_SPLIT_V | la.LA_FLAG_FUSED,
+    la.LA_FLAG_SPLIT_V | la.LA_FLAG_NO_SPLIT_V,
+    la.LA_FLAG_THREE_PASS | la.LA_FLAG_FUSED,
+    64,
+])
+def test_varlen_schedule_flag_validation(lib, flags):
+    # rejected before anything touches the device
+    assert la.la_prefill_varlen_ex(FAKE, FAKE, FAKE, FAKE, None, FAKE, 1, 16, 1, 128, 128,
+                                   la.LA_BF16, None, 0, flags) == la.LA_ERR_INVALID_ARG
+
+
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="not built"):
         la.load_library(str(tmp_path / "nope.so"))

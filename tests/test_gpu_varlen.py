@@ -48,7 +48,9 @@ def test_bad_seqlens_detected_on_device(bad):
 from _util import TOL_O_BF16, round_like  # noqa: E402
 
 
-SCHEDULES = [pytest.param(0, id="single-pass"), pytest.param(la.LA_FLAG_THREE_PASS, id="three-pass")]
+SCHEDULES = [pytest.param(0, id="default"), pytest.param(la.LA_FLAG_FUSED, id="single-pass"),
+             pytest.param(la.LA_FLAG_THREE_PASS, id="three-pass"),
+             pytest.param(la.LA_FLAG_SPLIT_V, id="split-v")]
 
 
 @pytest.mark.parametrize("blk", [128, 64])
@@ -94,25 +96,48 @@ def test_varlen_bf16_onehot_bit_exact(chunk, flags, blk):
     assert np.array_equal(host64(st), s_ref)
 
 
-def test_varlen_bf16_bad_seqlens_detected():
+@pytest.mark.parametrize("lens", [
+    [300, 7000, 1, 0, 129, 5000, 0, 2048, 128, 4097, 77],
+    [0, 0, 0, 5],
+    [1] * 40 + [3000],
+])
+def test_varlen_bf16_split_longest_first_exact(lens):
+    # split value columns, longest sequence first: every sequence and head is
+    # produced exactly once with its own state (one-hot keys: exact)
+    cu = _cu(lens)
+    H, T = 3, sum(lens)
+    q, k, v = inputs.onehot_k_qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=len(lens))
+    o = torch.full_like(q, 3.0)
+    st = torch.full((len(lens), H, 128, 128), 3.0, device=DEV)
+    o, st = la.prefill_varlen(q, k, v, cu, blk=128, out=o, state_out=st, flags=la.LA_FLAG_SPLIT_V)
+    assert la.la_get_last_error() == la.LA_OK
+    assert la.la_prefill_main_kernel() == "prefill_seq_kernel"
+    o_ref, s_ref = oracle.prefill_varlen(host64(q), host64(k), host64(v), cu.cpu().numpy())
+    assert np.array_equal(host64(o), round_like(o_ref, torch.bfloat16))
+    assert np.array_equal(host64(st), s_ref)
+
+
+@pytest.mark.parametrize("flags", SCHEDULES)
+def test_varlen_bf16_bad_seqlens_detected(flags):
     H, T = 2, 300
     q, k, v = inputs.qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=1)
     cu = torch.tensor([0, 200, 100, 300], dtype=torch.int32, device=DEV)
     o = torch.full_like(q, 3.0)
     st = torch.full((3, H, 128, 128), 3.0, device=DEV)
-    la.prefill_varlen(q, k, v, cu, blk=128, out=o, state_out=st)
+    la.prefill_varlen(q, k, v, cu, blk=128, out=o, state_out=st, flags=flags)
     assert la.la_get_last_error() == la.LA_ERR_BAD_SEQLENS
     assert torch.all(o == 3.0) and torch.all(st == 3.0)
 
 
-def test_varlen_bf16_packed_config_sampled_heads():
+@pytest.mark.parametrize("flags", [pytest.param(0, id="default"), pytest.param(la.LA_FLAG_SPLIT_V, id="split-v")])
+def test_varlen_bf16_packed_config_sampled_heads(flags):
     # 2^20 packed tokens, lengths uniform in [1024, 65536] (seeded, last
     # trimmed), H = 64, d = 128: every sequence of 8 sampled heads.
     T, H = 1 << 20, 64
     lens = inputs.varlen_lengths(T, 1024, 65536, seed=0)
     cu = _cu(lens)
     q, k, v = inputs.qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=0)
-    o, st = la.prefill_varlen(q, k, v, cu, blk=128)
+    o, st = la.prefill_varlen(q, k, v, cu, blk=128, flags=flags)
     assert la.la_get_last_error() == la.LA_OK
     rng = np.random.default_rng(0)
     heads = [0, H - 1] + sorted(rng.choice(np.arange(1, H - 1), 6, replace=False).tolist())
