@@ -83,7 +83,8 @@ constexpr int kModeVarlen = 1;
 
 struct Ctrl {
     uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t empty[kStages];     // every MMA of the tile done (V and Q no longer read)
+    uint64_t k_empty[kStages];   // K no longer read (the tile's last MMA4 done)
     uint64_t tail_ld;      // TMA completion of a packed-sequence tail block
     uint64_t s_full;       // MMA1 complete (scores in TMEM)
     uint64_t p_ready;      // epilogue wrote P (one arrival per epilogue warp)
@@ -325,6 +326,7 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(bar(ctrl->full[s]), 1);
             ptx::mbar_init(bar(ctrl->empty[s]), 1);
+            ptx::mbar_init(bar(ctrl->k_empty[s]), 1);
         }
         ptx::mbar_init(bar(ctrl->tail_ld), 1);
         ptx::mbar_init(bar(ctrl->s_full), 1);
@@ -373,61 +375,76 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
         const uint64_t pol_qk = p.vparts > 1 ? ptx::policy_evict_normal() : pol_first;
         uint32_t g = 0, n_tail = 0;
         bool ok = true;
-        auto next_stage = [&](int& s) -> bool {
-            s = g & 1;
-            if (g >= 2) {
-                int w = 1;
-                if (lane == 0) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
+        uint32_t c_uses[kStages] = {0, 0};   // phase-C uses of each stage so far
+        // One tile (rows [t, t+128) of item it) into stage g & 1.  Each operand
+        // is loaded as soon as its slot is free: K once the stage's previous
+        // tile finished MMA4 (k_empty), V once it finished MMA2 (empty), and Q
+        // (phase C) once the O tile staged in the Q slot has been stored.
+        auto produce = [&](const Item& it, int t, bool phase_c) -> bool {
+            const int s = g & 1;
+            const uint32_t stage = sbase + s * kStageB;
+            const bool tail = packed && it.t1 - t < kTileRows;
+            const uint32_t fb = tail ? bar(ctrl->tail_ld) : bar(ctrl->full[s]);
+            const uint64_t pol_k = phase_c ? pol_qk : pol_last;
+            const uint64_t pol_v = phase_c ? pol_first : pol_last;
+            int w = 1;
+            if (lane == 0) {
+                if (g >= 2) w = ptx::mbar_wait(bar(ctrl->k_empty[s]), ((g >> 1) + 1) & 1, abort_flag);
+                if (w) {
+                    ptx::mbar_arrive_expect_tx(fb, (phase_c ? 2 : 1) * kTileBytes + kVHalves * kHalfBytes);
+                    ptx::tma_load_4d(stage + kTileBytes, &maps.k, fb, 0, t, 0, it.z, pol_k);
+                    if (g >= 2) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
+                }
+                if (w) {
+                    if (kVHalves == 2)
+                        ptx::tma_load_4d(stage + 2 * kTileBytes, &maps.v, fb, 0, t, 0, it.z, pol_v);
+                    else
+                        ptx::tma_load_3d(stage + 2 * kTileBytes, &maps.v_half, fb, it.vp * kNV, t, it.z, pol_v);
+                    if (phase_c && c_uses[s] > 0)
+                        w = ptx::mbar_wait(bar(ctrl->o_stored[s]), (c_uses[s] - 1) & 1, abort_flag);
+                    if (w && phase_c) ptx::tma_load_4d(stage, &maps.q, fb, 0, t, 0, it.z, pol_qk);
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, w, 0)) return false;
+            if (phase_c) ++c_uses[s];
+            if (tail) {
+                // a packed tail: clear the next sequence's rows of V, then release
+                if (lane == 0) w = ptx::mbar_wait(bar(ctrl->tail_ld), n_tail & 1, abort_flag);
+                ++n_tail;
                 if (!__shfl_sync(0xffffffffu, w, 0)) return false;
+                zero_tail_rows(smem + s * kStageB + 2 * kTileBytes, it.t1 - t, lane, kVHalves);
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(ctrl->full[s]));
             }
             return true;
         };
         auto load_phase_a = [&](const Item& it) {
             // K and V only, kept in L2 for phase C
-            for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
-                int s;
-                if (!next_stage(s) ||
-                    !produce_tile<false, kVHalves>(maps, smem + s * kStageB + kTileBytes,
-                                                   sbase + s * kStageB + kTileBytes, bar(ctrl->full[s]),
-                                                   bar(ctrl->tail_ld), n_tail, t, it.z, it.t1 - t, packed,
-                                                   pol_last, pol_last, lane, abort_flag, it.vp * kNV))
-                    ok = false;
-            }
+            for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g)
+                if (!produce(it, t, false)) ok = false;
         };
         if ((int)blockIdx.x < n_items) {
             const Item first = get_item(p, blockIdx.x);
             if (has_phase_a(first)) load_phase_a(first);
         }
-        uint32_t c_uses[kStages] = {0, 0};   // phase-C uses of each stage so far
         for (int item = blockIdx.x; ok && item < n_items; item += stride) {
             const Item it = get_item(p, item);
             if (item + stride < n_items) {
                 const Item nx = get_item(p, item + stride);
                 if (has_phase_a(nx)) load_phase_a(nx);
             }
-            for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
-                int s;
-                if (!next_stage(s)) { ok = false; break; }
-                if (c_uses[s] > 0) {
-                    // the Q slot also staged the O tile of that stage's last phase-C block
-                    int w = 1;
-                    if (lane == 0) w = ptx::mbar_wait(bar(ctrl->o_stored[s]), (c_uses[s] - 1) & 1, abort_flag);
-                    if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-                }
-                ++c_uses[s];
-                if (!produce_tile<true, kVHalves>(maps, smem + s * kStageB, sbase + s * kStageB,
-                                                  bar(ctrl->full[s]), bar(ctrl->tail_ld), n_tail, t, it.z,
-                                                  it.t1 - t, packed, pol_qk, pol_qk, lane, abort_flag,
-                                                  it.vp * kNV, pol_first))
-                    ok = false;
-            }
+            for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g)
+                if (!produce(it, t, true)) ok = false;
         }
         // Wait for the last stage releases (MMA commits and O stores) so that no
         // asynchronous arrive is still pending on this CTA's shared memory when
         // it exits.
         if (lane == 0) {
-            for (uint32_t j = (g >= 2 ? g - 2 : 0); ok && j < g; ++j)
-                ok = ptx::mbar_wait(bar(ctrl->empty[j & 1]), (j >> 1) & 1, abort_flag);
+            for (uint32_t j = (g >= 2 ? g - 2 : 0); ok && j < g; ++j) {
+                ok = ptx::mbar_wait(bar(ctrl->k_empty[j & 1]), (j >> 1) & 1, abort_flag);
+                if (ok) ok = ptx::mbar_wait(bar(ctrl->empty[j & 1]), (j >> 1) & 1, abort_flag);
+            }
             for (int s = 0; ok && s < kStages; ++s)
                 if (c_uses[s] > 0) ok = ptx::mbar_wait(bar(ctrl->o_stored[s]), (c_uses[s] - 1) & 1, abort_flag);
         }
@@ -459,6 +476,7 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
                         ptx::mma_ss(tmem + kColDelta, ptx::sdesc_sw128(sk + kk * 2048, kHalfBytes, 1024),
                                     ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_kv,
                                     (kk > 0 || !first) ? 1u : 0u);
+                    ptx::mma_commit(bar(ctrl->k_empty[s]));
                     ptx::mma_commit(bar(ctrl->empty[s]));
                     first = false;
                 }
@@ -520,6 +538,7 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
                                         (kk > 0 || has_state) ? 1u : 0u);
                         }
                         ptx::mma_commit(bar(ctrl->state_done));
+                        if (sb == nsub - 1) ptx::mma_commit(bar(ctrl->k_empty[s]));   // K read
                         if (!ptx::mbar_wait(bar(ctrl->p_ready), n_blk & 1, abort_flag)) { ok = false; break; }
                         ptx::tc_fence_after();
                         // MMA2: O += P V (intra-block, left product); P from TMEM
