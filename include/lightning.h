@@ -124,6 +124,32 @@ int la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o, f
                          int chunk_tokens, int flags);
 
 /*
+ * la_prefill_from_state / la_prefill_varlen_from_state -- the prefills above
+ * continued from a given state: S_{-1} = state_in instead of zero, so
+ *     o_t = q_t (state_in + sum_{s <= t} k_s^T v_s),  state_out = state_in + K^T V.
+ * A sequence processed in pieces (chunked prefill, a prompt extended after
+ * decoding) gives the same result as in one call: prefill(A) then
+ * prefill_from_state(B, state_out of A) equals prefill(A ++ B) on B.
+ *   state_in : dense [B, H, d, d] / packed [num_seqs, H, d, d] fp32, the
+ *              layout of state_out (read only; NULL = zero start, which is
+ *              la_prefill_ex / la_prefill_varlen_ex).  It may be the same
+ *              array as state_out (each head's state is read before its final
+ *              state is written).  An empty packed sequence gets
+ *              state_out = state_in.
+ * Every other argument, the flags and the errors are those of la_prefill_ex /
+ * la_prefill_varlen_ex.  The starting state of the block-wise form (section 1
+ * of the futurefh page) is the running state; the pages do not name this
+ * entry point.
+ */
+int la_prefill_from_state(const void* q, const void* k, const void* v, void* o, const float* state_in,
+                          float* state_out, int B, int H, int N, int d, int blk, la_dtype dt,
+                          void* stream, int chunk_tokens, int flags);
+int la_prefill_varlen_from_state(const void* q, const void* k, const void* v, void* o,
+                                 const float* state_in, float* state_out, const int32_t* cu_seqlens,
+                                 int num_seqs, int total_tokens, int H, int d, int blk, la_dtype dt,
+                                 void* stream, int chunk_tokens, int flags);
+
+/*
  * la_decode_step -- one token per sequence (prefill and decode are separate,
  * section 3 of the futurefh page):  S <- S + k^T v ;  o = q S  (the update
  * includes the current token, so prefill(N) + step == prefill(N+1)).

@@ -48,7 +48,7 @@ LA_NUM_KERNEL_IDS = 6
 EXPORTED = ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step",
             "la_status_string", "la_get_last_error", "la_device_sm_count",
             "la_timing_enable", "la_timing_read", "la_kernel_name", "la_prefill_noalloc",
-            "la_prefill_main_kernel",
+            "la_prefill_main_kernel", "la_prefill_from_state", "la_prefill_varlen_from_state",
             "la_prefill_varlen_ex")
 
 LA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -77,6 +77,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la_prefill_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
     lib.la_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.la_prefill_varlen_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
+    lib.la_prefill_from_state.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
+    lib.la_prefill_varlen_from_state.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
     lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, vp]
     lib.la_status_string.argtypes = [i]
     lib.la_status_string.restype = ctypes.c_char_p
@@ -92,7 +94,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_prefill_varlen_ex",
                  "la_decode_step",
                  "la_get_last_error", "la_device_sm_count", "la_timing_enable",
-                 "la_timing_read", "la_prefill_noalloc"):
+                 "la_timing_read", "la_prefill_noalloc", "la_prefill_from_state",
+                 "la_prefill_varlen_from_state"):
         getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -117,6 +120,19 @@ def la_prefill_varlen(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens,
                       stream):
     return load_library().la_prefill_varlen(q, k, v, o, state_out, cu_seqlens, num_seqs,
                                             total_tokens, H, d, blk, dt, stream)
+
+
+def la_prefill_from_state(q, k, v, o, state_in, state_out, B, H, N, d, blk, dt, stream,
+                          chunk_tokens, flags):
+    return load_library().la_prefill_from_state(q, k, v, o, state_in, state_out, B, H, N, d, blk,
+                                                dt, stream, chunk_tokens, flags)
+
+
+def la_prefill_varlen_from_state(q, k, v, o, state_in, state_out, cu_seqlens, num_seqs,
+                                 total_tokens, H, d, blk, dt, stream, chunk_tokens, flags):
+    return load_library().la_prefill_varlen_from_state(q, k, v, o, state_in, state_out, cu_seqlens,
+                                                       num_seqs, total_tokens, H, d, blk, dt,
+                                                       stream, chunk_tokens, flags)
 
 
 def la_prefill_noalloc(q, k, v, o, state_out, B, H, N, d, blk, dt, stream):
@@ -202,8 +218,9 @@ def _raise(status, where):
 
 
 def prefill(q, k, v, blk: int = 128, want_state: bool = True, chunk_tokens: int = 0,
-            flags: int = 0, out=None, state_out=None, stream=None):
-    """Causal linear attention prefill of [B,H,N,d] tensors.  Returns (o, state)."""
+            flags: int = 0, out=None, state_out=None, stream=None, state_in=None):
+    """Causal linear attention prefill of [B,H,N,d] tensors, from ``state_in``
+    ([B,H,d,d] fp32; None = zero).  Returns (o, state)."""
     torch = _torch()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, n)
@@ -214,16 +231,23 @@ def prefill(q, k, v, blk: int = 128, want_state: bool = True, chunk_tokens: int 
     st = state_out
     if st is None and want_state:
         st = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
-    status = la_prefill_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                           st.data_ptr() if st is not None else None, B, H, N, d, blk,
-                           _dtype_code(q), _stream_ptr(stream), chunk_tokens, flags)
+    if state_in is not None:
+        _check(state_in, "state_in")
+        if state_in.dtype != torch.float32 or tuple(state_in.shape) != (B, H, d, d):
+            raise ValueError("state_in must be float32 [B,H,d,d]")
+    status = la_prefill_from_state(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                   state_in.data_ptr() if state_in is not None else None,
+                                   st.data_ptr() if st is not None else None, B, H, N, d, blk,
+                                   _dtype_code(q), _stream_ptr(stream), chunk_tokens, flags)
     _raise(status, "la_prefill")
     return o, st
 
 
 def prefill_varlen(q, k, v, cu_seqlens, blk: int = 128, want_state: bool = True, out=None,
-                   state_out=None, stream=None, chunk_tokens: int = 0, flags: int = 0):
-    """Packed prefill of [H,T,d] tensors split by int32 device cu_seqlens.
+                   state_out=None, stream=None, chunk_tokens: int = 0, flags: int = 0,
+                   state_in=None):
+    """Packed prefill of [H,T,d] tensors split by int32 device cu_seqlens, each
+    sequence from its ``state_in`` ([num_seqs,H,d,d] fp32; None = zero).
 
     Returns (o, state [num_seqs,H,d,d])."""
     torch = _torch()
@@ -237,10 +261,15 @@ def prefill_varlen(q, k, v, cu_seqlens, blk: int = 128, want_state: bool = True,
     st = state_out
     if st is None and want_state:
         st = torch.empty((S, H, d, d), dtype=torch.float32, device=q.device)
-    status = la_prefill_varlen_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                  st.data_ptr() if st is not None else None, cu_seqlens.data_ptr(),
-                                  S, T, H, d, blk, _dtype_code(q), _stream_ptr(stream),
-                                  chunk_tokens, flags)
+    if state_in is not None:
+        _check(state_in, "state_in")
+        if state_in.dtype != torch.float32 or tuple(state_in.shape) != (S, H, d, d):
+            raise ValueError("state_in must be float32 [num_seqs,H,d,d]")
+    status = la_prefill_varlen_from_state(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                          state_in.data_ptr() if state_in is not None else None,
+                                          st.data_ptr() if st is not None else None,
+                                          cu_seqlens.data_ptr(), S, T, H, d, blk, _dtype_code(q),
+                                          _stream_ptr(stream), chunk_tokens, flags)
     _raise(status, "la_prefill_varlen")
     return o, st
 

@@ -279,7 +279,7 @@ void launch_three_pass(const tc::TileMaps& m, tc::Params p, float* ws, float* st
     {
         TimedLaunch tl(LA_KERNEL_CHUNK_SCAN, stream);
         dim3 sgrid(kHeadDim * kHeadDim / 4 / 256, p.Z);
-        tc::chunk_scan_kernel<<<sgrid, 256, 0, stream>>>(ws, state_out, p.n_chunks);
+        tc::chunk_scan_kernel<<<sgrid, 256, 0, stream>>>(ws, state_out, p.n_chunks, p.state_in);
     }
     p.prefix = ws;
     p.state_out = nullptr;
@@ -345,7 +345,7 @@ int launch_fused(const tc::TileMaps& m, tc::Params p,
 
 int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, float* state_out,
                         int BH, int N, int blk, cudaStream_t stream, int sms, int chunk_tokens,
-                        int flags) {
+                        int flags, const float* state_in) {
     if (blk != 128 && blk != 64) return LA_ERR_UNSUPPORTED;
     tc::TileMaps m;
     if (make_tile_maps(&m, q, k, v, o, N, BH)) return LA_ERR_CUDA;
@@ -358,6 +358,7 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
         tc::Params p = dense_params(BH, N, chunk_tokens, o);
         p.vparts = vparts;
         p.blk = blk;
+        p.state_in = state_in;
         p.n_items *= vparts;
         const int grid = std::min(p.n_items, sms);
         return launch_fused(m, p, p.n_chunks > 1 ? (long)BH * p.n_chunks : 0, state_out,
@@ -368,6 +369,7 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
     tc::Params p = dense_params(BH, N, chunk_tokens, o);
     p.vparts = vparts;
     p.blk = blk;
+    p.state_in = state_in;
     p.n_items *= vparts;
     const int grid = std::min(p.n_items, sms);
 
@@ -414,7 +416,7 @@ int choose_varlen_chunk_tokens(int H, int T, int ctas) {
 // sequences first, run by the sequential kernel.  Nothing is read twice.
 int launch_prefill_varlen_split(const void* q, const void* k, const void* v, void* o,
                                 float* state_out, const int32_t* cu_seqlens, int num_seqs, int T,
-                                int H, cudaStream_t stream, int sms) {
+                                int H, cudaStream_t stream, int sms, const float* state_in) {
     const long max_items = (long)num_seqs * H * 2;
     if (max_items > (1L << 30)) return LA_ERR_UNSUPPORTED;
     tc::TileMaps m;
@@ -437,7 +439,8 @@ int launch_prefill_varlen_split(const void* q, const void* k, const void* v, voi
     }
     if (state_out != nullptr) {
         TimedLaunch tl(LA_KERNEL_AUX, stream);
-        tc::zero_empty_states_kernel<<<dim3(num_seqs, H), 256, 0, stream>>>(state_out, cu_seqlens, ok, H);
+        tc::zero_empty_states_kernel<<<dim3(num_seqs, H), 256, 0, stream>>>(state_out, cu_seqlens, ok, H,
+                                                                          state_in);
     }
     tc::Params p;
     std::memset(&p, 0, sizeof(p));
@@ -453,6 +456,7 @@ int launch_prefill_varlen_split(const void* q, const void* k, const void* v, voi
     p.seq_ok = ok;
     p.num_seqs = num_seqs;
     p.seq_order = order;
+    p.state_in = state_in;
     p.o = reinterpret_cast<__nv_bfloat16*>(o);
     p.state_out = state_out;
     const int grid = (int)std::min<long>(max_items, sms);
@@ -468,7 +472,7 @@ int launch_prefill_varlen_split(const void* q, const void* k, const void* v, voi
 int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void* o,
                                float* state_out, const int32_t* cu_seqlens, int num_seqs, int T,
                                int H, int blk, cudaStream_t stream, int sms, bool three_pass,
-                               int chunk_tokens) {
+                               int chunk_tokens, const float* state_in) {
     if (blk != 128 && blk != 64) return LA_ERR_UNSUPPORTED;
     if (chunk_tokens <= 0)
         chunk_tokens = three_pass ? choose_varlen_chunk_tokens(H, std::max(T, 1), sms)
@@ -501,6 +505,7 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
     p.mode = tc::kModeVarlen;
     p.vparts = 1;
     p.blk = blk;
+    p.state_in = state_in;
     p.Z = H;
     p.rows = rows;
     p.chunk_tokens = chunk_tokens;
@@ -518,7 +523,7 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
         if (state_out != nullptr) {
             TimedLaunch tl(LA_KERNEL_AUX, stream);
             tc::zero_empty_states_kernel<<<dim3(num_seqs, H), 256, 0, stream>>>(state_out, cu_seqlens,
-                                                                              ok, H);
+                                                                              ok, H, state_in);
         }
         p.fused = 1;
         p.chain = ws;
@@ -541,7 +546,7 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
         TimedLaunch tl(LA_KERNEL_CHUNK_SCAN, stream);
         dim3 sgrid(num_seqs, H);
         tc::chunk_scan_varlen_kernel<<<sgrid, 256, 0, stream>>>(ws, state_out, chunk_off, ok, H,
-                                                               num_seqs);
+                                                               num_seqs, state_in);
     }
     p.prefix = ws;
     {
@@ -624,9 +629,10 @@ using namespace la;
 
 extern "C" {
 
-int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* state_out, int B,
-                  int H, int N, int d, int blk, la_dtype dt, void* stream, int chunk_tokens,
-                  int flags) {
+namespace {
+int prefill_impl(const void* q, const void* k, const void* v, void* o, const float* state_in,
+                 float* state_out, int B, int H, int N, int d, int blk, la_dtype dt, void* stream,
+                 int chunk_tokens, int flags) {
     if (B < 1 || H < 1 || N < 1) return LA_ERR_INVALID_ARG;
     constexpr int kAllFlags = LA_FLAG_THREE_PASS | LA_FLAG_FUSED | LA_FLAG_SPLIT_V | LA_FLAG_NO_SPLIT_V;
     if ((flags & ~kAllFlags) != 0 ||
@@ -635,7 +641,7 @@ int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* s
         return LA_ERR_INVALID_ARG;
     int st = validate_common(q, k, v, o, d, blk, dt);
     if (st != LA_OK) return st;
-    if (state_out && !aligned16(state_out)) return LA_ERR_INVALID_ARG;
+    if ((state_out && !aligned16(state_out)) || (state_in && !aligned16(state_in))) return LA_ERR_INVALID_ARG;
     if ((long long)B * H > (1ll << 30) || (long long)N > (1ll << 30)) return LA_ERR_INVALID_ARG;
     int dev = 0, sms = 0;
     st = device_setup(&dev, &sms);
@@ -650,14 +656,15 @@ int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* s
         TimedLaunch tl(LA_KERNEL_PREFILL_F32, s);
         if (d == 64)
             simt::prefill_simt_kernel<64><<<BH, simt::kThreads, simt::smem_bytes<64>(), s>>>(
-                qf, kf, vf, of, state_out, N, blk);
+                qf, kf, vf, of, state_out, state_in, N, blk);
         else
             simt::prefill_simt_kernel<128><<<BH, simt::kThreads, simt::smem_bytes<128>(), s>>>(
-                qf, kf, vf, of, state_out, N, blk);
+                qf, kf, vf, of, state_out, state_in, N, blk);
         return note_cuda(cudaGetLastError());
     }
-    return launch_prefill_bf16(q, k, v, o, state_out, BH, N, blk, s, sms, chunk_tokens, flags);
+    return launch_prefill_bf16(q, k, v, o, state_out, BH, N, blk, s, sms, chunk_tokens, flags, state_in);
 }
+}  // namespace
 
 int la_prefill(const void* q, const void* k, const void* v, void* o, float* state_out, int B, int H,
                int N, int d, int blk, la_dtype dt, void* stream) {
@@ -671,9 +678,10 @@ int la_prefill_varlen(const void* q, const void* k, const void* v, void* o, floa
                                 blk, dt, stream, 0, 0);
 }
 
-int la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o, float* state_out,
-                         const int32_t* cu_seqlens, int num_seqs, int total_tokens, int H, int d,
-                         int blk, la_dtype dt, void* stream, int chunk_tokens, int flags) {
+namespace {
+int varlen_impl(const void* q, const void* k, const void* v, void* o, const float* state_in,
+                float* state_out, const int32_t* cu_seqlens, int num_seqs, int total_tokens, int H,
+                int d, int blk, la_dtype dt, void* stream, int chunk_tokens, int flags) {
     constexpr int kAllFlags = LA_FLAG_THREE_PASS | LA_FLAG_FUSED | LA_FLAG_SPLIT_V | LA_FLAG_NO_SPLIT_V;
     if ((flags & ~kAllFlags) != 0 ||
         (flags & (LA_FLAG_THREE_PASS | LA_FLAG_FUSED)) == (LA_FLAG_THREE_PASS | LA_FLAG_FUSED) ||
@@ -684,18 +692,18 @@ int la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o, f
     if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return LA_ERR_INVALID_ARG;
     int st = validate_common(q, k, v, o, d, blk, dt);
     if (st != LA_OK) return st;
-    if (state_out && !aligned16(state_out)) return LA_ERR_INVALID_ARG;
+    if ((state_out && !aligned16(state_out)) || (state_in && !aligned16(state_in))) return LA_ERR_INVALID_ARG;
     int dev = 0, sms = 0;
     st = device_setup(&dev, &sms);
     if (st != LA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (dt == LA_BF16 && blk == 128 && (flags & LA_FLAG_SPLIT_V))
         return launch_prefill_varlen_split(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens,
-                                           H, s, sms);
+                                           H, s, sms, state_in);
     if (dt == LA_BF16)
         return launch_prefill_varlen_bf16(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens,
                                           H, blk, s, sms, (flags & LA_FLAG_THREE_PASS) != 0,
-                                          chunk_tokens);
+                                          chunk_tokens, state_in);
     int* ok = nullptr;
     if (cudaMallocAsync(reinterpret_cast<void**>(&ok), sizeof(int), s) != cudaSuccess) {
         cudaGetLastError();
@@ -714,14 +722,42 @@ int la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o, f
     TimedLaunch tl(LA_KERNEL_PREFILL_F32, s);
     if (d == 64)
         simt::prefill_simt_varlen_kernel<64><<<grid, simt::kThreads, simt::smem_bytes<64>(), s>>>(
-            qf, kf, vf, of, state_out, cu_seqlens, ok, num_seqs, H, total_tokens, blk);
+            qf, kf, vf, of, state_out, state_in, cu_seqlens, ok, num_seqs, H, total_tokens, blk);
     else
         simt::prefill_simt_varlen_kernel<128><<<grid, simt::kThreads, simt::smem_bytes<128>(), s>>>(
-            qf, kf, vf, of, state_out, cu_seqlens, ok, num_seqs, H, total_tokens, blk);
+            qf, kf, vf, of, state_out, state_in, cu_seqlens, ok, num_seqs, H, total_tokens, blk);
     }
     st = note_cuda(cudaGetLastError());
     cudaFreeAsync(ok, s);
     return st;
+}
+}  // namespace
+
+int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* state_out, int B,
+                  int H, int N, int d, int blk, la_dtype dt, void* stream, int chunk_tokens,
+                  int flags) {
+    return prefill_impl(q, k, v, o, nullptr, state_out, B, H, N, d, blk, dt, stream, chunk_tokens, flags);
+}
+
+int la_prefill_from_state(const void* q, const void* k, const void* v, void* o, const float* state_in,
+                          float* state_out, int B, int H, int N, int d, int blk, la_dtype dt,
+                          void* stream, int chunk_tokens, int flags) {
+    return prefill_impl(q, k, v, o, state_in, state_out, B, H, N, d, blk, dt, stream, chunk_tokens, flags);
+}
+
+int la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o, float* state_out,
+                         const int32_t* cu_seqlens, int num_seqs, int total_tokens, int H, int d,
+                         int blk, la_dtype dt, void* stream, int chunk_tokens, int flags) {
+    return varlen_impl(q, k, v, o, nullptr, state_out, cu_seqlens, num_seqs, total_tokens, H, d, blk,
+                       dt, stream, chunk_tokens, flags);
+}
+
+int la_prefill_varlen_from_state(const void* q, const void* k, const void* v, void* o,
+                                 const float* state_in, float* state_out, const int32_t* cu_seqlens,
+                                 int num_seqs, int total_tokens, int H, int d, int blk, la_dtype dt,
+                                 void* stream, int chunk_tokens, int flags) {
+    return varlen_impl(q, k, v, o, state_in, state_out, cu_seqlens, num_seqs, total_tokens, H, d, blk,
+                       dt, stream, chunk_tokens, flags);
 }
 
 int la_decode_step(const void* q, const void* k, const void* v, float* state, void* o, int B, int H,

@@ -33,6 +33,7 @@ struct Segment {
     size_t base;       // element offset of token row 0 of this head
     int t0, t1;        // token range [t0, t1)
     float* state;      // [D][D] destination or null
+    const float* state_in;  // [D][D] starting state, or null (zero)
 };
 
 template <int D>
@@ -46,7 +47,7 @@ __device__ void run_segment(const float* __restrict__ q, const float* __restrict
     float* P = Vs + kSub * D;            // [32][33]
     const int tid = threadIdx.x;
 
-    for (int i = tid; i < D * D; i += kThreads) S[i] = 0.f;
+    for (int i = tid; i < D * D; i += kThreads) S[i] = sg.state_in ? sg.state_in[i] : 0.f;
     __syncthreads();
 
     // thread -> (row i, columns j = jc + 8*m) of a 32 x D output sub-tile
@@ -133,7 +134,7 @@ __device__ void run_segment(const float* __restrict__ q, const float* __restrict
 template <int D>
 __global__ void __launch_bounds__(kThreads)
 prefill_simt_kernel(const float* q, const float* k, const float* v, float* o, float* state_out,
-                    int N, int blk) {
+                    const float* state_in, int N, int blk) {
     extern __shared__ float smem_f[];
     const int bh = blockIdx.x;
     Segment sg;
@@ -141,6 +142,7 @@ prefill_simt_kernel(const float* q, const float* k, const float* v, float* o, fl
     sg.t0 = 0;
     sg.t1 = N;
     sg.state = state_out ? state_out + (size_t)bh * D * D : nullptr;
+    sg.state_in = state_in ? state_in + (size_t)bh * D * D : nullptr;
     run_segment<D>(q, k, v, o, sg, blk, smem_f);
 }
 
@@ -149,8 +151,8 @@ prefill_simt_kernel(const float* q, const float* k, const float* v, float* o, fl
 template <int D>
 __global__ void __launch_bounds__(kThreads)
 prefill_simt_varlen_kernel(const float* q, const float* k, const float* v, float* o,
-                           float* state_out, const int32_t* cu_seqlens, const int* seqlens_ok,
-                           int num_seqs, int H, int T, int blk) {
+                           float* state_out, const float* state_in, const int32_t* cu_seqlens,
+                           const int* seqlens_ok, int num_seqs, int H, int T, int blk) {
     extern __shared__ float smem_f[];
     if (*seqlens_ok == 0) return;
     const int j = blockIdx.x;
@@ -160,6 +162,7 @@ prefill_simt_varlen_kernel(const float* q, const float* k, const float* v, float
     sg.t0 = cu_seqlens[j];
     sg.t1 = cu_seqlens[j + 1];
     sg.state = state_out ? state_out + ((size_t)j * H + h) * D * D : nullptr;
+    sg.state_in = state_in ? state_in + ((size_t)j * H + h) * D * D : nullptr;
     run_segment<D>(q, k, v, o, sg, blk, smem_f);
 }
 

@@ -126,6 +126,8 @@ struct Params {
     int blk;                    // block size of the intra/inter split: 128, or 64 (vparts 1)
     const int32_t* seq_order;   // packed, one chunk per sequence: the sequence of chunk g
                                 // (non-empty sequences, longest first), or null
+    const float* state_in;      // starting state of every sequence (layout of state_out),
+                                // or null (zero)
 };
 
 // One work item: rows [t0, t1) of slice z, chunk c of its sequence, value
@@ -185,6 +187,18 @@ __device__ __forceinline__ Item get_item(const Params& p, int item) {
         it.last = g == p.chunk_off[lo + 1] - 1;
     }
     return it;
+}
+
+// Starting state of an item that is not found by look-back, or null (zero).
+// With a prefix array (three-pass) it is the chunk's exclusive prefix, which
+// the scan starts from state_in, so chunk 0 reads it there too: state_out may
+// then alias state_in although the scan writes the final state before this
+// pass runs.  Without one, chunk 0 starts from the caller's state_in.  Points
+// at row 0, column 0 of the d x d state.
+__device__ __forceinline__ const float* start_state(const Params& p, const Item& it) {
+    if (it.c == 0 && p.state_in == nullptr) return nullptr;
+    if (p.prefix != nullptr) return p.prefix + (size_t)it.ws * (kHeadDim * kHeadDim);
+    return it.c == 0 ? p.state_in + (size_t)it.sidx * (kHeadDim * kHeadDim) : nullptr;
 }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -494,7 +508,7 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
                     if (has_phase_a(nx)) run_phase_a(nx);
                     if (!ok) break;
                 }
-                bool has_state = fused ? it.c > 0 : (p.prefix != nullptr && it.c > 0);
+                bool has_state = fused ? (it.c > 0 || p.state_in != nullptr) : start_state(p, it) != nullptr;
                 for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
                     const int s = g & 1;
                     if (!ptx::mbar_wait(bar(ctrl->full[s]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
@@ -760,11 +774,14 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
             const Item it = get_item(p, item);
             const bool phase_a = has_phase_a(it);
             const bool look = fused && it.c > 0;
-            const bool from_prefix = !fused && p.prefix != nullptr && it.c > 0;
             const size_t roff = (size_t)r * kHeadDim + it.vp * kNV;   // row r, this value part
-            const float* src = nullptr;          // exclusive prefix
-            if (look) src = p.chain + (size_t)(it.ws - 1) * (kHeadDim * kHeadDim) + roff;
-            if (from_prefix) src = p.prefix + (size_t)it.ws * (kHeadDim * kHeadDim) + roff;
+            const float* src = nullptr;          // exclusive prefix (with state_in)
+            if (look) {
+                src = p.chain + (size_t)(it.ws - 1) * (kHeadDim * kHeadDim) + roff;
+            } else {
+                const float* st0 = start_state(p, it);
+                if (st0 != nullptr) src = st0 + roff;
+            }
             const size_t fl = ((size_t)it.ws * p.vparts + it.vp) * kChainWarps + cw;   // own flag
             const size_t fl_prev = fl - (size_t)p.vparts * kChainWarps;               // chunk c-1's
             if (phase_a) {
@@ -1059,7 +1076,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
             bool ok = true;
             for (int item = blockIdx.x; ok && item < n_items; item += stride) {
                 const Item it = get_item(p, item);
-                bool has_state = p.prefix != nullptr && it.c > 0;
+                bool has_state = start_state(p, it) != nullptr;
                 for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
                     const int s = g & 1;
                     const uint32_t b = g & 1;
@@ -1161,9 +1178,8 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
             const int vcol = it.vp * sq::kNV + c0;  // first owned column of the 128
             // ---- running state S (row r, columns vcol..vcol+31) and S̄ for block 0
             float srun[32];
-            if (p.prefix != nullptr && it.c > 0) {
-                const float4* src = reinterpret_cast<const float4*>(
-                    p.prefix + (size_t)it.ws * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim + vcol);
+            if (const float* st0 = start_state(p, it)) {
+                const float4* src = reinterpret_cast<const float4*>(st0 + (size_t)r * kHeadDim + vcol);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const float4 x = __ldg(src + j);
@@ -1454,10 +1470,12 @@ chunk_state_kernel(const __grid_constant__ TileMaps maps,
 // Scans over chunks: exclusive prefix in place, inclusive total -> state_out.
 // ============================================================================
 __global__ void __launch_bounds__(256)
-chunk_scan_kernel(float* ws, float* state_out, int n_chunks) {
+chunk_scan_kernel(float* ws, float* state_out, int n_chunks, const float* state_in) {
     const int bh = blockIdx.y;
     const int e = (blockIdx.x * blockDim.x + threadIdx.x) * 4;   // < 128*128
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc = state_in != nullptr
+                     ? *reinterpret_cast<const float4*>(state_in + (size_t)bh * (kHeadDim * kHeadDim) + e)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
     float4* base = reinterpret_cast<float4*>(ws + (size_t)bh * n_chunks * (kHeadDim * kHeadDim) + e);
     constexpr int kStride4 = kHeadDim * kHeadDim / 4;
     for (int c = 0; c < n_chunks; ++c) {
@@ -1476,7 +1494,7 @@ chunk_scan_kernel(float* ws, float* state_out, int n_chunks) {
 // state_out is [num_seqs][H][128][128]; an empty sequence gets a zero state.
 __global__ void __launch_bounds__(256)
 chunk_scan_varlen_kernel(float* ws, float* state_out, const int32_t* chunk_off, const int* seq_ok,
-                         int H, int num_seqs) {
+                         int H, int num_seqs, const float* state_in) {
     if (*seq_ok == 0) return;
     const int j = blockIdx.x;
     const int hh = blockIdx.y;
@@ -1484,8 +1502,11 @@ chunk_scan_varlen_kernel(float* ws, float* state_out, const int32_t* chunk_off, 
     const int c0 = chunk_off[j], c1 = chunk_off[j + 1];
     constexpr int kStride4 = kHeadDim * kHeadDim / 4;
     float4* base = reinterpret_cast<float4*>(ws + (size_t)hh * total * (kHeadDim * kHeadDim));
+    const float4* in4 = state_in != nullptr
+                            ? reinterpret_cast<const float4*>(state_in + ((size_t)j * H + hh) * (kHeadDim * kHeadDim))
+                            : nullptr;
     for (int e4 = threadIdx.x; e4 < kStride4; e4 += blockDim.x) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 acc = in4 != nullptr ? in4[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
         for (int c = c0; c < c1; ++c) {
             const float4 x = base[(size_t)c * kStride4 + e4];
             base[(size_t)c * kStride4 + e4] = acc;
@@ -1500,22 +1521,25 @@ chunk_scan_varlen_kernel(float* ws, float* state_out, const int32_t* chunk_off, 
 }
 
 // Single pass over packed sequences: an empty sequence owns no work item, so
-// its final state is cleared here.  Grid (num_seqs, H).
+// its final state (its starting state, or zero) is written here.  Grid
+// (num_seqs, H).
 __global__ void __launch_bounds__(256)
-zero_empty_states_kernel(float* state_out, const int32_t* cu, const int* seq_ok, int H) {
+zero_empty_states_kernel(float* state_out, const int32_t* cu, const int* seq_ok, int H,
+                         const float* state_in) {
     if (*seq_ok == 0) return;
     const int j = blockIdx.x;
     if (cu[j + 1] != cu[j]) return;
-    float4* dst = reinterpret_cast<float4*>(state_out + ((size_t)j * H + blockIdx.y) * (kHeadDim * kHeadDim));
+    const size_t off = ((size_t)j * H + blockIdx.y) * (kHeadDim * kHeadDim);
+    float4* dst = reinterpret_cast<float4*>(state_out + off);
+    const float4* src = state_in != nullptr ? reinterpret_cast<const float4*>(state_in + off) : nullptr;
     for (int e = threadIdx.x; e < kHeadDim * kHeadDim / 4; e += blockDim.x)
-        dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        dst[e] = src != nullptr ? src[e] : make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // cu_seqlens check and chunk offsets of packed sequences (one CTA): verdict in
 // *ok, chunk_off[j] = sum over earlier sequences of ceil(len / chunk_tokens),
 // chunk_off[num_seqs] = chunks per head.  A malformed array records
-// LA_ERR_BAD_SEQLENS and yields zero chunks.
-// Check cu_seqlens and number the chunks of every sequence (chunk_off).  With
+// LA_ERR_BAD_SEQLENS and yields zero chunks.  Check cu_seqlens and number the chunks of every sequence (chunk_off).  With
 // `order` non-null (one chunk per sequence: chunk_tokens >= every length) it
 // also lists the non-empty sequences longest first, ties by index: a
 // persistent grid that walks items in that order takes the long ones first.
