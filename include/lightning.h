@@ -150,6 +150,29 @@ int la_prefill_varlen_from_state(const void* q, const void* k, const void* v, vo
                                  void* stream, int chunk_tokens, int flags);
 
 /*
+ * Sequence parallelism across GPUs (the improved linear-attention sequence
+ * parallelism, LASP, that section 2 of the futurefh page names for unbounded
+ * context windows; the pages give no algorithm, this is its plain reading).  A sequence split over R ranks, rank r
+ * holding tokens [r N/R, (r+1) N/R) of every (batch, head), is prefilled as
+ *   1. la_state_increment: dS_r = K_r^T V_r of the rank's tokens;
+ *   2. all-gather of dS over the ranks (the caller's collective, e.g. NCCL);
+ *   3. la_state_prefix: S_in,r = sum_{r' < r} dS_r';
+ *   4. la_prefill_from_state on the rank's tokens from S_in,r.
+ * The last rank's state_out is the whole sequence's final state.
+ *
+ * la_state_increment -- delta_out[B,H,d,d] (fp32, written) = K^T V over the
+ *   N tokens of k, v [B,H,N,d] (read only).  bf16 with d = 128 only
+ *   (LA_ERR_UNSUPPORTED otherwise).
+ * la_state_prefix -- prefix_out[B,H,d,d] = sum_{r < rank} states[r] (zero for
+ *   rank 0), summed in rank order; states is [R][B,H,d,d] fp32 (read only),
+ *   0 <= rank <= R, d in {64, 128}.
+ */
+int la_state_increment(const void* k, const void* v, float* delta_out, int B, int H, int N, int d,
+                       la_dtype dt, void* stream);
+int la_state_prefix(const float* states, int R, int rank, float* prefix_out, int B, int H, int d,
+                    void* stream);
+
+/*
  * la_decode_step -- one token per sequence (prefill and decode are separate,
  * section 3 of the futurefh page):  S <- S + k^T v ;  o = q S  (the update
  * includes the current token, so prefill(N) + step == prefill(N+1)).

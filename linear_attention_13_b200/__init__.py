@@ -49,6 +49,7 @@ EXPORTED = ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step"
             "la_status_string", "la_get_last_error", "la_device_sm_count",
             "la_timing_enable", "la_timing_read", "la_kernel_name", "la_prefill_noalloc",
             "la_prefill_main_kernel", "la_prefill_from_state", "la_prefill_varlen_from_state",
+            "la_state_increment", "la_state_prefix",
             "la_prefill_varlen_ex")
 
 LA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -78,6 +79,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.la_prefill_varlen_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
     lib.la_prefill_from_state.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
+    lib.la_state_increment.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
+    lib.la_state_prefix.argtypes = [vp, i, i, vp, i, i, i, vp]
     lib.la_prefill_varlen_from_state.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
     lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, vp]
     lib.la_status_string.argtypes = [i]
@@ -95,7 +98,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                  "la_decode_step",
                  "la_get_last_error", "la_device_sm_count", "la_timing_enable",
                  "la_timing_read", "la_prefill_noalloc", "la_prefill_from_state",
-                 "la_prefill_varlen_from_state"):
+                 "la_prefill_varlen_from_state", "la_state_increment", "la_state_prefix"):
         getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -133,6 +136,14 @@ def la_prefill_varlen_from_state(q, k, v, o, state_in, state_out, cu_seqlens, nu
     return load_library().la_prefill_varlen_from_state(q, k, v, o, state_in, state_out, cu_seqlens,
                                                        num_seqs, total_tokens, H, d, blk, dt,
                                                        stream, chunk_tokens, flags)
+
+
+def la_state_increment(k, v, delta_out, B, H, N, d, dt, stream):
+    return load_library().la_state_increment(k, v, delta_out, B, H, N, d, dt, stream)
+
+
+def la_state_prefix(states, R, rank, prefix_out, B, H, d, stream):
+    return load_library().la_state_prefix(states, R, rank, prefix_out, B, H, d, stream)
 
 
 def la_prefill_noalloc(q, k, v, o, state_out, B, H, N, d, blk, dt, stream):
@@ -272,6 +283,32 @@ def prefill_varlen(q, k, v, cu_seqlens, blk: int = 128, want_state: bool = True,
                                           _stream_ptr(stream), chunk_tokens, flags)
     _raise(status, "la_prefill_varlen")
     return o, st
+
+
+def state_increment(k, v, out=None, stream=None):
+    """K^T V over the tokens of [B,H,N,d] bf16 k, v: [B,H,d,d] fp32."""
+    torch = _torch()
+    for t, n in ((k, "k"), (v, "v")):
+        _check(t, n)
+    B, H, N, d = k.shape
+    o = out if out is not None else torch.empty((B, H, d, d), dtype=torch.float32, device=k.device)
+    status = la_state_increment(k.data_ptr(), v.data_ptr(), o.data_ptr(), B, H, N, d,
+                                _dtype_code(k), _stream_ptr(stream))
+    _raise(status, "la_state_increment")
+    return o
+
+
+def state_prefix(states, rank, out=None, stream=None):
+    """sum over r < rank of states[r] ([R,B,H,d,d] fp32): [B,H,d,d] fp32."""
+    torch = _torch()
+    _check(states, "states")
+    if states.dtype != torch.float32 or states.dim() != 5:
+        raise ValueError("states must be float32 [R,B,H,d,d]")
+    R, B, H, d, _ = states.shape
+    o = out if out is not None else torch.empty((B, H, d, d), dtype=torch.float32, device=states.device)
+    status = la_state_prefix(states.data_ptr(), R, rank, o.data_ptr(), B, H, d, _stream_ptr(stream))
+    _raise(status, "la_state_prefix")
+    return o
 
 
 def decode_step(q, k, v, state, out=None, stream=None):

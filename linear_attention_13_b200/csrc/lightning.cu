@@ -760,6 +760,49 @@ int la_prefill_varlen_from_state(const void* q, const void* k, const void* v, vo
                        dt, stream, chunk_tokens, flags);
 }
 
+int la_state_increment(const void* k, const void* v, float* delta_out, int B, int H, int N, int d,
+                       la_dtype dt, void* stream) {
+    if (B < 1 || H < 1 || N < 1 || !k || !v || !delta_out) return LA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(delta_out)) return LA_ERR_INVALID_ARG;
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (dt != LA_BF16 || d != 128) return LA_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1ll << 30) || (long long)N > (1ll << 30)) return LA_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    int st = device_setup(&dev, &sms);
+    if (st != LA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int BH = B * H;
+    // only the K and V maps are read; q and o name valid tensors of the same shape
+    tc::TileMaps m;
+    if (make_tile_maps(&m, k, k, v, v, N, BH)) return LA_ERR_CUDA;
+    tc::Params p = dense_params(BH, N, ((N + kTileRows - 1) / kTileRows) * kTileRows, nullptr);
+    p.chunk_delta = delta_out;   // one chunk per head: chunk index ws = head
+    {
+        TimedLaunch tl(LA_KERNEL_CHUNK_STATE, s);
+        tc::chunk_state_kernel<<<std::min(p.n_items, sms), tc::cs::kThreads, tc::cs::kSmemBytes, s>>>(m, p);
+    }
+    return note_cuda(cudaGetLastError());
+}
+
+int la_state_prefix(const float* states, int R, int rank, float* prefix_out, int B, int H, int d,
+                    void* stream) {
+    if (!states || !prefix_out || R < 1 || rank < 0 || rank > R || B < 1 || H < 1) return LA_ERR_INVALID_ARG;
+    if (!aligned16(states) || !aligned16(prefix_out)) return LA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
+    int dev = 0, sms = 0;
+    int st = device_setup(&dev, &sms);
+    if (st != LA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const long n4 = (long)B * H * d * d / 4;
+    {
+        TimedLaunch tl(LA_KERNEL_AUX, s);
+        const int grid = (int)std::min<long>((n4 + 255) / 256, 4L * sms);
+        tc::state_prefix_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(states), rank, n4,
+                                                     reinterpret_cast<float4*>(prefix_out));
+    }
+    return note_cuda(cudaGetLastError());
+}
+
 int la_decode_step(const void* q, const void* k, const void* v, float* state, void* o, int B, int H,
                    int d, la_dtype dt, void* stream) {
     if (B < 1 || H < 1) return LA_ERR_INVALID_ARG;

@@ -1520,6 +1520,23 @@ chunk_scan_varlen_kernel(float* ws, float* state_out, const int32_t* chunk_off, 
     }
 }
 
+// Exclusive prefix over ranks of per-rank states (sequence parallelism): out =
+// sum_{r < rank} states[r], summed in rank order.  states is [R][n4] float4.
+__global__ void __launch_bounds__(256)
+state_prefix_kernel(const float4* states, int rank, long n4, float4* out) {
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < rank; ++r) {
+            const float4 x = states[(size_t)r * n4 + i];
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
+        }
+        out[i] = acc;
+    }
+}
+
 // Single pass over packed sequences: an empty sequence owns no work item, so
 // its final state (its starting state, or zero) is written here.  Grid
 // (num_seqs, H).
