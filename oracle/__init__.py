@@ -88,6 +88,7 @@ class Oracle:
         lib.oracle_prefill_blockwise.argtypes = [dp, dp, dp, dp, dp, L, L, L, L]
         lib.oracle_decode_step.argtypes = [dp, dp, dp, dp, dp, L, L]
         lib.oracle_prefill_varlen.argtypes = [dp, dp, dp, ip, L, L, L, L, dp, dp, ip, L]
+        lib.oracle_prefill_backward.argtypes = [dp, dp, dp, dp, dp, dp, dp, L, L, L]
         for f in ("oracle_prefill_quadratic", "oracle_prefill_recurrent",
                   "oracle_prefill_blockwise", "oracle_decode_step", "oracle_prefill_varlen"):
             getattr(lib, f).restype = None
@@ -127,6 +128,15 @@ class Oracle:
         self.lib.oracle_prefill_blockwise(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(st),
                                           BH, N, d, blk)
         return o, st
+
+    def prefill_backward(self, q, k, v, do):
+        """Gradients (dq, dk, dv) of sum(dO * o) for the causal form (fp64)."""
+        BH, N, d = _shape_bhnd(q)
+        q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+        dq, dk, dv = (np.zeros(q.shape, dtype=np.float64) for _ in range(3))
+        self.lib.oracle_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk),
+                                         _ptr(dv), BH, N, d)
+        return dq, dk, dv
 
     def decode_step(self, q, k, v, state):
         """One decode step; returns (o, new_state), the input state untouched."""
@@ -190,6 +200,10 @@ def prefill_blockwise(q, k, v, blk: int):
 
 def decode_step(q, k, v, state):
     return _get().decode_step(q, k, v, state)
+
+
+def prefill_backward(q, k, v, do):
+    return _get().prefill_backward(q, k, v, do)
 
 
 def prefill_varlen(q, k, v, cu_seqlens, heads=None):

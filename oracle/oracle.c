@@ -117,6 +117,48 @@ void oracle_prefill_recurrent(const double* q, const double* k, const double* v,
 }
 
 /*
+ * Gradients of L = sum_t dO_t . o_t with respect to q, k, v, from the
+ * quadratic definition o_t = sum_{s <= t} (q_t . k_s) v_s differentiated term
+ * by term (the pages give no backward pass; training is the context of the
+ * LASP+ passage of the futurefh page, section 2):
+ *     dq_t = sum_{s <= t} (dO_t . v_s) k_s
+ *     dk_s = sum_{t >= s} (dO_t . v_s) q_t
+ *     dv_s = sum_{t >= s} (q_t . k_s) dO_t
+ * O(N^2 d).  Layout as the forward forms; do_ is dO.
+ */
+void oracle_prefill_backward(const double* q, const double* k, const double* v, const double* do_,
+                             double* dq, double* dk, double* dv, long BH, long N, long d) {
+    long bh;
+#pragma omp parallel for schedule(dynamic)
+    for (bh = 0; bh < BH; ++bh) {
+        const double* Q = q + bh * N * d;
+        const double* K = k + bh * N * d;
+        const double* V = v + bh * N * d;
+        const double* G = do_ + bh * N * d;
+        double* DQ = dq + bh * N * d;
+        double* DK = dk + bh * N * d;
+        double* DV = dv + bh * N * d;
+        memset(DQ, 0, (size_t)(N * d) * sizeof(double));
+        memset(DK, 0, (size_t)(N * d) * sizeof(double));
+        memset(DV, 0, (size_t)(N * d) * sizeof(double));
+        for (long t = 0; t < N; ++t) {
+            for (long s = 0; s <= t; s++) {
+                double gv = 0.0, qk = 0.0;
+                for (long c = 0; c < d; ++c) {
+                    gv += G[t * d + c] * V[s * d + c];
+                    qk += Q[t * d + c] * K[s * d + c];
+                }
+                for (long c = 0; c < d; ++c) {
+                    DQ[t * d + c] += gv * K[s * d + c];
+                    DK[s * d + c] += gv * Q[t * d + c];
+                    DV[s * d + c] += qk * G[t * d + c];
+                }
+            }
+        }
+    }
+}
+
+/*
  * Block form with block size blk, in the order section 1 of the futurefh page
  * describes: for block i (rows [i*blk, min((i+1)*blk, N)) ),
  *     O_i = tril(Q_i K_i^T) V_i   (intra-block, left product)

@@ -185,8 +185,46 @@ def pin_varlen(orc):
     assert np.array_equal(st2[:, 2], st[:, 2])
 
 
+def pin_backward_finite_differences(orc):
+    """The gradients of L = sum(dO * o) agree with central differences of the
+    forward (quadratic) form: a check that does not use the gradient formulas."""
+    rng = np.random.default_rng(17)
+    BH, N, d = 2, 5, 3
+    q, k, v, do = (rng.standard_normal((BH, N, d)) for _ in range(4))
+    dq, dk, dv = orc.prefill_backward(q, k, v, do)
+    h = 1e-6
+
+    def loss(qq, kk, vv):
+        return float(np.sum(do * orc.prefill_quadratic(qq, kk, vv)))
+
+    for x, g, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        assert np.allclose(g, num, rtol=0, atol=1e-6), which
+
+
+def pin_backward_d1_sums(orc):
+    """d = 1: dq_t = k-weighted prefix sum, dk_s and dv_s suffix sums (closed form)."""
+    rng = np.random.default_rng(3)
+    q, k, v, do = (rng.standard_normal((1, 7, 1)) for _ in range(4))
+    dq, dk, dv = orc.prefill_backward(q, k, v, do)
+    qf, kf, vf, gf = (x[0, :, 0] for x in (q, k, v, do))
+    assert np.allclose(dq[0, :, 0], gf * np.cumsum(vf * kf), atol=1e-12)
+    suffix_gq = np.cumsum((gf * qf)[::-1])[::-1]
+    assert np.allclose(dk[0, :, 0], vf * suffix_gq, atol=1e-12)
+    assert np.allclose(dv[0, :, 0], kf * suffix_gq, atol=1e-12)
+
+
 PINS = [pin_golden, pin_forms_agree, pin_state_is_KtV, pin_last_row, pin_d1_prefix_sum, pin_N1,
-        pin_ternary_bruteforce, pin_state_in, pin_decode, pin_varlen]
+        pin_ternary_bruteforce, pin_state_in, pin_decode, pin_varlen, pin_backward_finite_differences,
+        pin_backward_d1_sums]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -216,6 +254,9 @@ MUTANTS = {
         ""),
     "varlen_skips_first_token": ("long t0 = cu_seqlens[j], t1", "long t0 = cu_seqlens[j] + 1, t1"),
     "varlen_no_state_reset_shared_offset": ("O[t * d + c] = acc;", "O[t * d + c] = acc + (t == t0);"),
+    "backward_dq_uses_q": ("DQ[t * d + c] += gv * K[s * d + c];", "DQ[t * d + c] += gv * Q[s * d + c];"),
+    "backward_dk_wrong_token": ("DK[s * d + c] += gv * Q[t * d + c];", "DK[s * d + c] += gv * Q[s * d + c];"),
+    "backward_drops_diagonal": ("for (long s = 0; s <= t; s++) {", "for (long s = 0; s < t; s++) {"),
 }
 
 
