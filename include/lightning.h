@@ -150,6 +150,22 @@ int la_prefill_varlen_from_state(const void* q, const void* k, const void* v, vo
                                  void* stream, int chunk_tokens, int flags);
 
 /*
+ * la_prefill_backward -- gradients of L = sum_t dO_t . o_t for o = la_prefill
+ * (q, k, v) (zero starting state), the training direction:
+ *     dq_t = sum_{s <= t} (dO_t . v_s) k_s     (the causal form of (dO, v, k))
+ *     dk_s = sum_{t >= s} (dO_t . v_s) q_t     (anti-causal: the causal form
+ *     dv_s = sum_{t >= s} (q_t . k_s) dO_t      of the token-reversed sequence)
+ *   q, k, v, do_ : [B, H, N, d] of dt (read only); dq, dk, dv : [B, H, N, d]
+ *   of dt (written).  Same dtype, d, blk rules as la_prefill.  Scratch: five
+ *   tensors of the input size from the stream-ordered allocator.  The pages
+ *   give no backward pass (training is the context of section 2 of the
+ *   futurefh page); this is the derivative of the forward definition.
+ */
+int la_prefill_backward(const void* q, const void* k, const void* v, const void* do_, void* dq,
+                        void* dk, void* dv, int B, int H, int N, int d, int blk, la_dtype dt,
+                        void* stream);
+
+/*
  * Sequence parallelism across GPUs (the improved linear-attention sequence
  * parallelism, LASP, that section 2 of the futurefh page names for unbounded
  * context windows; the pages give no algorithm, this is its plain reading).  A sequence split over R ranks, rank r

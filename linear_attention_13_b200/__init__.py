@@ -49,7 +49,7 @@ EXPORTED = ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step"
             "la_status_string", "la_get_last_error", "la_device_sm_count",
             "la_timing_enable", "la_timing_read", "la_kernel_name", "la_prefill_noalloc",
             "la_prefill_main_kernel", "la_prefill_from_state", "la_prefill_varlen_from_state",
-            "la_state_increment", "la_state_prefix",
+            "la_state_increment", "la_state_prefix", "la_prefill_backward",
             "la_prefill_varlen_ex")
 
 LA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -80,6 +80,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la_prefill_varlen_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
     lib.la_prefill_from_state.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
     lib.la_state_increment.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
+    lib.la_prefill_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.la_state_prefix.argtypes = [vp, i, i, vp, i, i, i, vp]
     lib.la_prefill_varlen_from_state.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
     lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, vp]
@@ -98,7 +99,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                  "la_decode_step",
                  "la_get_last_error", "la_device_sm_count", "la_timing_enable",
                  "la_timing_read", "la_prefill_noalloc", "la_prefill_from_state",
-                 "la_prefill_varlen_from_state", "la_state_increment", "la_state_prefix"):
+                 "la_prefill_varlen_from_state", "la_state_increment", "la_state_prefix",
+                 "la_prefill_backward"):
         getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -136,6 +138,10 @@ def la_prefill_varlen_from_state(q, k, v, o, state_in, state_out, cu_seqlens, nu
     return load_library().la_prefill_varlen_from_state(q, k, v, o, state_in, state_out, cu_seqlens,
                                                        num_seqs, total_tokens, H, d, blk, dt,
                                                        stream, chunk_tokens, flags)
+
+
+def la_prefill_backward(q, k, v, do, dq, dk, dv, B, H, N, d, blk, dt, stream):
+    return load_library().la_prefill_backward(q, k, v, do, dq, dk, dv, B, H, N, d, blk, dt, stream)
 
 
 def la_state_increment(k, v, delta_out, B, H, N, d, dt, stream):
@@ -283,6 +289,22 @@ def prefill_varlen(q, k, v, cu_seqlens, blk: int = 128, want_state: bool = True,
                                           _stream_ptr(stream), chunk_tokens, flags)
     _raise(status, "la_prefill_varlen")
     return o, st
+
+
+def prefill_backward(q, k, v, do, blk: int = 128, stream=None):
+    """Gradients (dq, dk, dv) of sum(do * prefill(q, k, v)[0]) for [B,H,N,d] tensors."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (do, "do")):
+        _check(t, n)
+    if not (k.shape == q.shape == v.shape == do.shape) or q.dim() != 4:
+        raise ValueError("q, k, v, do must share one [B,H,N,d] shape")
+    B, H, N, d = q.shape
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    status = la_prefill_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(),
+                                 dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, blk,
+                                 _dtype_code(q), _stream_ptr(stream))
+    _raise(status, "la_prefill_backward")
+    return dq, dk, dv
 
 
 def state_increment(k, v, out=None, stream=None):

@@ -17,6 +17,7 @@
 #include "ptx.cuh"
 #include "prefill_tc.cuh"
 #include "prefill_simt.cuh"
+#include "tokens.cuh"
 #include "decode.cuh"
 
 namespace la {
@@ -758,6 +759,59 @@ int la_prefill_varlen_from_state(const void* q, const void* k, const void* v, vo
                                  void* stream, int chunk_tokens, int flags) {
     return varlen_impl(q, k, v, o, state_in, state_out, cu_seqlens, num_seqs, total_tokens, H, d, blk,
                        dt, stream, chunk_tokens, flags);
+}
+
+int la_prefill_backward(const void* q, const void* k, const void* v, const void* do_, void* dq,
+                        void* dk, void* dv, int B, int H, int N, int d, int blk, la_dtype dt,
+                        void* stream) {
+    if (B < 1 || H < 1 || N < 1 || !do_ || !dq || !dk || !dv) return LA_ERR_INVALID_ARG;
+    if (!aligned16(do_) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return LA_ERR_INVALID_ARG;
+    int st = validate_common(q, k, v, dq, d, blk, dt);
+    if (st != LA_OK) return st;
+    if ((long long)B * H > (1ll << 30) || (long long)N > (1ll << 30)) return LA_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    st = device_setup(&dev, &sms);
+    if (st != LA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // dq_t = sum_{s <= t} (dO_t . v_s) k_s : the causal form with (q, k, v) = (dO, v, k)
+    st = prefill_impl(do_, v, k, dq, nullptr, nullptr, B, H, N, d, blk, dt, stream, 0, 0);
+    if (st != LA_OK) return st;
+    // dk_s = sum_{t >= s} (v_s . dO_t) q_t and dv_s = sum_{t >= s} (k_s . q_t) dO_t are
+    // causal sums of the token-reversed sequence, reversed back
+    const long Z = (long)B * H;
+    const size_t elems = (size_t)Z * N * d;
+    const size_t esz = dt == LA_BF16 ? 2 : 4;
+    const int row16 = (int)(d * esz / 16);
+    uint8_t* buf = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&buf), 5 * elems * esz, s) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_ALLOC;
+    }
+    uint8_t* rq = buf;
+    uint8_t* rk = rq + elems * esz;
+    uint8_t* rv = rk + elems * esz;
+    uint8_t* rg = rv + elems * esz;
+    uint8_t* tmp = rg + elems * esz;
+    const long words = (long)elems * (long)esz / 16;
+    const int grid = (int)std::min<long>((words + 255) / 256, 8L * sms);
+    auto reverse = [&](const void* src, void* dst) {
+        TimedLaunch tl(LA_KERNEL_AUX, s);
+        reverse_tokens_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(src),
+                                                   reinterpret_cast<uint4*>(dst), Z, N, row16);
+    };
+    reverse(q, rq);
+    reverse(k, rk);
+    reverse(v, rv);
+    reverse(do_, rg);
+    st = prefill_impl(rv, rg, rq, tmp, nullptr, nullptr, B, H, N, d, blk, dt, stream, 0, 0);
+    if (st == LA_OK) {
+        reverse(tmp, dk);
+        st = prefill_impl(rk, rq, rg, tmp, nullptr, nullptr, B, H, N, d, blk, dt, stream, 0, 0);
+    }
+    if (st == LA_OK) reverse(tmp, dv);
+    if (st == LA_OK) st = note_cuda(cudaGetLastError());
+    cudaFreeAsync(buf, s);
+    return st;
 }
 
 int la_state_increment(const void* k, const void* v, float* delta_out, int B, int H, int N, int d,

@@ -1,0 +1,61 @@
+"""GPU parity of la_prefill_backward (and the autograd wrapper) with the fp64
+oracle's gradients of sum(dO * o)."""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_13_b200 as la
+from linear_attention_13_b200 import inputs
+import oracle
+from _util import TOL_O_BF16, TOL_O_F32, host64, per_head_rel_err, round_like
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _grads_ref(q, k, v, do):
+    return oracle.prefill_backward(host64(q), host64(k), host64(v), host64(do))
+
+
+@pytest.mark.parametrize("blk", [128, 64])
+@pytest.mark.parametrize("N", [1, 129, 1000, 2049])
+def test_bf16_backward(N, blk):
+    q, k, v = inputs.qkv((2, 3, N, 128), dtype=torch.bfloat16, device=DEV, seed=N)
+    do = inputs.qkv((2, 3, N, 128), dtype=torch.bfloat16, device=DEV, seed=N + 99)[2]
+    dq, dk, dv = la.prefill_backward(q, k, v, do, blk=blk)
+    assert la.la_get_last_error() == la.LA_OK
+    for got, ref in zip((dq, dk, dv), _grads_ref(q, k, v, do)):
+        assert per_head_rel_err(host64(got), ref) <= TOL_O_BF16
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp32_backward(d):
+    q, k, v = inputs.qkv((1, 3, 300, d), dtype=torch.float32, device=DEV, seed=d)
+    do = inputs.qkv((1, 3, 300, d), dtype=torch.float32, device=DEV, seed=d + 1)[2]
+    dq, dk, dv = la.prefill_backward(q, k, v, do, blk=64)
+    assert la.la_get_last_error() == la.LA_OK
+    for got, ref in zip((dq, dk, dv), _grads_ref(q, k, v, do)):
+        assert per_head_rel_err(host64(got), ref) <= TOL_O_F32
+
+
+@pytest.mark.parametrize("N", [100, 256])
+def test_bf16_backward_ternary_bit_exact(N):
+    q, k, v = inputs.ternary_qkv((1, 4, N, 128), dtype=torch.bfloat16, device=DEV, seed=N)
+    do = inputs.ternary_qkv((1, 4, N, 128), dtype=torch.bfloat16, device=DEV, seed=N + 1)[0]
+    dq, dk, dv = la.prefill_backward(q, k, v, do)
+    for got, ref in zip((dq, dk, dv), _grads_ref(q, k, v, do)):
+        assert np.array_equal(host64(got), round_like(ref, torch.bfloat16))
+
+
+def test_autograd_matches_oracle():
+    from linear_attention_13_b200.autograd import lightning_attention
+    q, k, v = inputs.qkv((1, 2, 700, 128), dtype=torch.bfloat16, device=DEV, seed=8)
+    w = inputs.qkv((1, 2, 700, 128), dtype=torch.bfloat16, device=DEV, seed=9)[2]
+    q, k, v = (x.clone().requires_grad_(True) for x in (q, k, v))
+    o = lightning_attention(q, k, v)
+    (o.float() * w.float()).sum().backward()
+    o_ref, _ = oracle.prefill_recurrent(host64(q.detach()), host64(k.detach()), host64(v.detach()))
+    assert per_head_rel_err(host64(o.detach()), o_ref) <= TOL_O_BF16
+    refs = _grads_ref(q.detach(), k.detach(), v.detach(), w)
+    for x, ref in zip((q, k, v), refs):
+        assert per_head_rel_err(host64(x.grad), ref) <= TOL_O_BF16
