@@ -1119,7 +1119,10 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                         ptx::mma_commit(bar(ctrl->empty[s]));
                     } else {
                         // MMA4: dS = K^T V into buffer b, once block g-2's dS has been read
+                        // and this block's MMA1 has completed: MMA1 -> P -> MMA2 is the
+                        // critical chain, so MMA4 runs while the epilogue builds P
                         if (g >= 2 && !ptx::mbar_wait(bar(ctrl->ds_free[b]), prev, abort_flag)) { ok = false; break; }
+                        if (!ptx::mbar_wait(bar(ctrl->s_full[b]), par, abort_flag)) { ok = false; break; }
                         ptx::tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
