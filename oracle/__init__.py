@@ -18,6 +18,12 @@ function cites the passage it follows in ``oracle.c``:
   product, section 1 of the futurefh page.
 * ``decode_step``        -- one recurrent step (update, then read).
 * ``prefill_varlen``     -- recurrent form per packed sequence, state reset.
+* ``decode_step_slots``  -- decode over a pool of states addressed by slot id,
+  negative ids being padding rows (the multi-level padding of section 3 of
+  the futurefh page).
+* ``state_quantize_q8`` / ``state_dequantize_q8`` / ``decode_step_q8`` -- the
+  8-bit state (int8 codes, one fp32 scale per key row) that the yuliangy.com
+  digest's 8-bit quantisation is read as; decisions taken in fp32.
 
 Pins (what checks this oracle against something other than itself) live in
 ``tests/test_oracle_pins.py``.
@@ -38,7 +44,7 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 def compile_source(src_path: str, out_path: str) -> str:
     """Compile a C source of the oracle into a shared library with gcc."""
     tmp = out_path + ".tmp.%d" % os.getpid()
-    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", src_path, "-o", tmp]
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", src_path, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, out_path)
     return out_path
@@ -60,6 +66,27 @@ def _ptr(a):
     if a is None:
         return None
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def _f32_exact(a) -> np.ndarray:
+    """fp32 copy that must not round (the 8-bit state's inputs are fp32 or bf16)."""
+    x = np.asarray(a, dtype=np.float64)
+    y = _f32(x)
+    if not np.array_equal(y.astype(np.float64), x):
+        raise ValueError("inputs of the 8-bit decode step must be exact in fp32")
+    return y
+
+
+def _fptr(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+
+
+def _cptr(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_byte))
 
 
 def _shape_bhnd(q):
@@ -89,8 +116,14 @@ class Oracle:
         lib.oracle_decode_step.argtypes = [dp, dp, dp, dp, dp, L, L]
         lib.oracle_prefill_varlen.argtypes = [dp, dp, dp, ip, L, L, L, L, dp, dp, ip, L]
         lib.oracle_prefill_backward.argtypes = [dp, dp, dp, dp, dp, dp, dp, L, L, L]
+        fp = ctypes.POINTER(ctypes.c_float)
+        cp = ctypes.POINTER(ctypes.c_byte)
+        lib.oracle_state_quantize_q8.argtypes = [fp, cp, fp, L, L]
+        lib.oracle_state_dequantize_q8.argtypes = [cp, fp, fp, L, L]
+        lib.oracle_decode_step_q8.argtypes = [fp, fp, fp, cp, fp, dp, L, L]
         for f in ("oracle_prefill_quadratic", "oracle_prefill_recurrent",
-                  "oracle_prefill_blockwise", "oracle_decode_step", "oracle_prefill_varlen"):
+                  "oracle_prefill_blockwise", "oracle_decode_step", "oracle_prefill_varlen",
+                  "oracle_state_quantize_q8", "oracle_state_dequantize_q8", "oracle_decode_step_q8"):
             getattr(lib, f).restype = None
         self.lib = lib
 
@@ -147,6 +180,41 @@ class Oracle:
         o = np.zeros(q.shape, dtype=np.float64)
         self.lib.oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(S), _ptr(o), BH, d)
         return o, S
+
+    def state_quantize_q8(self, state):
+        """fp32 states [..., d, d] -> (int8 codes [..., d, d], fp32 scales [..., d])."""
+        S = _f32(state)
+        d = S.shape[-1]
+        rows = S.size // d
+        codes = np.zeros(S.shape, dtype=np.int8)
+        scales = np.zeros(S.shape[:-1], dtype=np.float32)
+        self.lib.oracle_state_quantize_q8(_fptr(S), _cptr(codes), _fptr(scales), rows, d)
+        return codes, scales
+
+    def state_dequantize_q8(self, codes, scales):
+        """(codes, scales) -> fp32 states, S_ij = c_ij * a_i."""
+        c = np.ascontiguousarray(codes, dtype=np.int8)
+        a = _f32(scales)
+        d = c.shape[-1]
+        S = np.zeros(c.shape, dtype=np.float32)
+        self.lib.oracle_state_dequantize_q8(_cptr(c), _fptr(a), _fptr(S), c.size // d, d)
+        return S
+
+    def decode_step_q8(self, q, k, v, codes, scales):
+        """One step on the 8-bit state; returns (o fp64, codes', scales'), inputs untouched.
+
+        q, k, v must hold values exact in fp32 (fp32 or bf16 inputs)."""
+        qf, kf, vf = _f32_exact(q), _f32_exact(k), _f32_exact(v)
+        c = np.array(codes, dtype=np.int8, copy=True, order="C")
+        a = np.array(scales, dtype=np.float32, copy=True, order="C")
+        d = qf.shape[-1]
+        BH = qf.size // d
+        if c.size != BH * d * d or a.size != BH * d:
+            raise ValueError("codes must be [..., d, d] and scales [..., d] for every q row")
+        o = np.zeros(qf.shape, dtype=np.float64)
+        self.lib.oracle_decode_step_q8(_fptr(qf), _fptr(kf), _fptr(vf), _cptr(c), _fptr(a),
+                                       _ptr(o), BH, d)
+        return o, c, a
 
     def prefill_varlen(self, q, k, v, cu_seqlens, heads=None):
         """Packed prefill over [H,T,d] inputs split by cu_seqlens.
@@ -208,3 +276,60 @@ def prefill_backward(q, k, v, do):
 
 def prefill_varlen(q, k, v, cu_seqlens, heads=None):
     return _get().prefill_varlen(q, k, v, cu_seqlens, heads)
+
+
+def state_quantize_q8(state):
+    return _get().state_quantize_q8(state)
+
+
+def state_dequantize_q8(codes, scales):
+    return _get().state_dequantize_q8(codes, scales)
+
+
+def _slot_rows(slots, num_slots):
+    slots = np.asarray(slots, dtype=np.int64).reshape(-1)
+    if np.any(slots >= num_slots):
+        raise ValueError("slot id out of range")
+    live = slots[slots >= 0]
+    if len(np.unique(live)) != len(live):
+        raise ValueError("a slot may appear once per batch")
+    return slots
+
+
+def decode_step_slots(q, k, v, pool, slots):
+    """Decode step for a batch whose row b uses state pool[slots[b]].
+
+    q, k, v: [B, H, d]; pool: [num_slots, H, d, d]; a negative slot marks a
+    padding row, whose output is zero and which touches no state.  Returns
+    (o [B, H, d], pool') in fp64; the input pool is untouched.  Each live row is
+    ``decode_step`` applied to its own slot's state."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    pool = _f64(pool).copy()
+    slots = _slot_rows(slots, pool.shape[0])
+    o = np.zeros(q.shape, dtype=np.float64)
+    for b, slot in enumerate(slots):
+        if slot < 0:
+            continue
+        o[b], pool[slot] = decode_step(q[b], k[b], v[b], pool[slot])
+    return o, pool
+
+
+def decode_step_q8(q, k, v, codes, scales, slots=None):
+    """One step on the 8-bit state, optionally over a slot pool (as above).
+
+    codes: [num_slots, H, d, d] int8, scales: [num_slots, H, d] fp32; without
+    ``slots`` row b uses slot b.  Returns (o fp64, codes', scales')."""
+    orc = _get()
+    q = np.asarray(q)
+    if slots is None:
+        return orc.decode_step_q8(q, np.asarray(k), np.asarray(v), codes, scales)
+    k, v = np.asarray(k), np.asarray(v)
+    codes = np.array(codes, dtype=np.int8, copy=True)
+    scales = np.array(scales, dtype=np.float32, copy=True)
+    slots = _slot_rows(slots, codes.shape[0])
+    o = np.zeros(q.shape, dtype=np.float64)
+    for b, slot in enumerate(slots):
+        if slot < 0:
+            continue
+        o[b], codes[slot], scales[slot] = orc.decode_step_q8(q[b], k[b], v[b], codes[slot], scales[slot])
+    return o, codes, scales

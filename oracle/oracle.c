@@ -41,6 +41,7 @@
  * packed [H][T][d]; cu_seqlens has num_seqs+1 entries; states are
  * [num_seqs][H][d][d].
  */
+#include <math.h>
 #include <stddef.h>
 #include <stdlib.h>
 #include <string.h>
@@ -272,5 +273,88 @@ void oracle_prefill_varlen(const double* q, const double* k, const double* v,
         }
         if (state_out) memcpy(state_out + (j * H + h) * d * d, S, (size_t)(d * d) * sizeof(double));
         free(S);
+    }
+}
+
+/*
+ * Decode on an 8-bit state.  The yuliangy.com digest of the MiniMax-01 report
+ * credits 8-bit quantisation with fitting more than a million tokens on one
+ * eight-GPU machine; none of the pages gives a format.  The reading taken
+ * here: row i of a head's state (key dimension i) is held as int8 codes c_ij
+ * in [-127, 127] and one fp32 scale a_i, standing for S_ij = c_ij * a_i.
+ *
+ * Quantising one fp32 row x_0 .. x_{d-1}:
+ *     m = max_j |x_j|
+ *     if m < 2^-100:  a = 0 and every code is 0        (zero or negligible row)
+ *     else:           a = m / 127,  c_j = nearest-even integer to x_j * (127 / m)
+ * m / 127, 127 / m and x_j * (127 / m) are each one correctly rounded fp32
+ * operation.  Codes are integer decisions, so they are taken in fp32 (the
+ * precision the state is held in) and compared code for code with the kernel.
+ */
+static void quantize_row_q8(const float* x, signed char* c, float* a, long d) {
+    float m = 0.0f;
+    for (long j = 0; j < d; ++j) {
+        const float ax = fabsf(x[j]);
+        if (ax > m) m = ax;
+    }
+    if (m < 0x1p-100f) {
+        *a = 0.0f;
+        for (long j = 0; j < d; ++j) c[j] = 0;
+        return;
+    }
+    const float inv = 127.0f / m;
+    *a = m / 127.0f;
+    for (long j = 0; j < d; ++j) {
+        float r = rintf(x[j] * inv);
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+        c[j] = (signed char)r;
+    }
+}
+
+/* rows x d fp32 states -> int8 codes [rows][d] and scales [rows]. */
+void oracle_state_quantize_q8(const float* S, signed char* codes, float* scales, long rows, long d) {
+    for (long r = 0; r < rows; ++r) quantize_row_q8(S + r * d, codes + r * d, scales + r, d);
+}
+
+/* codes [rows][d], scales [rows] -> S_ij = c_ij * a_i (one fp32 product). */
+void oracle_state_dequantize_q8(const signed char* codes, const float* scales, float* S, long rows,
+                                long d) {
+    for (long r = 0; r < rows; ++r)
+        for (long j = 0; j < d; ++j) S[r * d + j] = (float)codes[r * d + j] * scales[r];
+}
+
+/*
+ * One decode step on the 8-bit state, update first and read second as in
+ * oracle_decode_step:
+ *     s_ij = fma(k_i, v_j, c_ij * a_i)    fp32: dequantise, then add k^T v
+ *     o_j  = sum_i q_i s_ij              fp64 sum over the fp32 s
+ *     codes, scales <- row-wise quantisation of s (above)
+ * q, k, v are [BH][d] fp32 (bf16 inputs convert exactly); codes [BH][d][d]
+ * and scales [BH][d] are updated in place; o is [BH][d].
+ */
+void oracle_decode_step_q8(const float* q, const float* k, const float* v, signed char* codes,
+                           float* scales, double* o, long BH, long d) {
+    long bh;
+#pragma omp parallel for schedule(static)
+    for (bh = 0; bh < BH; ++bh) {
+        const float* qb = q + bh * d;
+        const float* kb = k + bh * d;
+        const float* vb = v + bh * d;
+        signed char* cb = codes + bh * d * d;
+        float* ab = scales + bh * d;
+        float* s = (float*)malloc((size_t)(d * d) * sizeof(float));
+        for (long i = 0; i < d; ++i)
+            for (long j = 0; j < d; ++j) {
+                const float deq = (float)cb[i * d + j] * ab[i];
+                s[i * d + j] = fmaf(kb[i], vb[j], deq);
+            }
+        for (long j = 0; j < d; ++j) {
+            double acc = 0.0;
+            for (long i = 0; i < d; ++i) acc += (double)qb[i] * (double)s[i * d + j];
+            o[bh * d + j] = acc;
+        }
+        for (long i = 0; i < d; ++i) quantize_row_q8(s + i * d, cb + i * d, ab + i, d);
+        free(s);
     }
 }

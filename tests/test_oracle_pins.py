@@ -11,7 +11,12 @@ Each pin states what fixes the expected value:
   * exact brute force in Python integers on small ternary inputs,
   * the running-state semantics of the closing analogy of the same page:
     prefill(N) followed by one decode step equals prefill(N+1),
-  * packing (section 4 of the futurefh page): varlen == dense per sequence.
+  * packing (section 4 of the futurefh page): varlen == dense per sequence,
+  * the 8-bit state: a hand-worked example of its rounding rules and of one
+    step (tests/golden/), integer-exact trajectories, and the fp64 recurrence
+    within the error bound the rounding rules give,
+  * decode over a slot pool: padding rows touch nothing, live rows equal the
+    dense step on their own slot.
 
 ``test_pins_catch_planted_mistakes`` compiles altered copies of oracle.c (a
 dropped diagonal, a transposed operand, a wrong sign, ...) and checks that every
@@ -222,9 +227,107 @@ def pin_backward_d1_sums(orc):
     assert np.allclose(dv[0, :, 0], kf * suffix_gq, atol=1e-12)
 
 
+def pin_q8_golden(orc):
+    g = json.load(open(os.path.join(GOLDEN, "q8_state_worked_example.json")))
+    for row in g["quantize"]:
+        c, a = orc.state_quantize_q8(np.array([row["x"]], np.float32))
+        assert c[0].tolist() == row["codes"], row["why"]
+        assert a[0] == np.float32(row["scale"]), row["why"]
+        back = orc.state_dequantize_q8(c, a)
+        assert np.array_equal(back[0], np.array(row["codes"], np.float32) * np.float32(row["scale"]))
+    st = g["step"]
+    o, c, a = orc.decode_step_q8(np.array([st["q"]], np.float32), np.array([st["k"]], np.float32),
+                                 np.array([st["v"]], np.float32), np.array([st["codes"]], np.int8),
+                                 np.array([st["scales"]], np.float32))
+    assert o[0].tolist() == st["o"]
+    assert c[0].tolist() == st["codes_out"]
+    assert a[0].tolist() == [float(np.float32(x)) for x in st["scales_out"]]
+
+
+def pin_q8_integer_trajectory(orc):
+    """Rows whose largest magnitude stays exactly 127 have scale 1, so codes are
+    the state itself: one-hot keys and small integer values keep every step
+    exact, and the result is brute force in Python integers."""
+    rng = _rng(21)
+    BH, d, T = 2, 8, 30
+    S = rng.integers(-60, 61, (BH, d, d))
+    S[:, :, 0] = 127                       # column 0 holds each row's maximum ...
+    codes = S.astype(np.int8)
+    scales = np.ones((BH, d), np.float32)
+    for t in range(T):
+        q = rng.integers(-3, 4, (BH, d))
+        k = np.zeros((BH, d), int)
+        r = rng.integers(0, d, BH)
+        k[np.arange(BH), r] = rng.choice([-1, 1], BH)
+        v = rng.integers(-2, 3, (BH, d))
+        v[:, 0] = 0                        # ... and no step changes it
+        for b in range(BH):                # keep the updated row inside [-127, 127]
+            row = S[b, r[b]] + k[b, r[b]] * v[b]
+            v[b] = np.where(np.abs(row) > 120, 0, v[b])
+        S = S + np.einsum("bi,bj->bij", k, v)
+        o_ref = np.einsum("bi,bij->bj", q, S)
+        o, codes, scales = orc.decode_step_q8(q.astype(np.float32), k.astype(np.float32),
+                                              v.astype(np.float32), codes, scales)
+        assert np.array_equal(codes.astype(int), S), t
+        assert np.all(scales == 1.0)
+        assert np.array_equal(o, o_ref.astype(float)), t
+
+
+def pin_q8_within_rounding_bound(orc):
+    """Against the fp64 recurrence started from the same dequantised state:
+    each step adds at most half a quantisation step (a/2) plus fp32 rounding
+    (2^-20 of the row's largest magnitude) to every element of a row."""
+    rng = _rng(22)
+    BH, d, T = 3, 16, 48
+    c, a = orc.state_quantize_q8(rng.standard_normal((BH, d, d)).astype(np.float32))
+    exact = orc.state_dequantize_q8(c, a).astype(np.float64)
+    bound = np.zeros((BH, d))
+    for t in range(T):
+        q, k, v = (rng.standard_normal((BH, d)).astype(np.float32) for _ in range(3))
+        o, c, a_new = orc.decode_step_q8(q, k, v, c, a)
+        exact = exact + np.einsum("bi,bj->bij", k.astype(float), v.astype(float))
+        m = 127.0 * a_new.astype(float)
+        step_bound = bound + 2.0 ** -20 * m   # s before quantisation
+        o_ref = np.einsum("bi,bij->bj", q.astype(float), exact)
+        o_bound = np.einsum("bi,bi->b", np.abs(q.astype(float)), step_bound)[:, None]
+        assert np.all(np.abs(o - o_ref) <= o_bound + 1e-9), t
+        bound = bound + 0.5 * a_new.astype(float) + 2.0 ** -20 * m
+        got = orc.state_dequantize_q8(c, a_new).astype(np.float64)
+        assert np.all(np.abs(got - exact) <= bound[:, :, None] + 1e-12), t
+        a = a_new
+    assert np.max(bound) < 0.2 * np.max(np.abs(exact))   # and the bound is not vacuous
+
+
+def pin_decode_slots(orc):
+    """Padding rows (negative slot) give zero output and touch no state; every
+    live row equals the dense step on its own slot's state."""
+    rng = _rng(23)
+    H, d, n_slots = 2, 6, 5
+    pool = rng.standard_normal((n_slots, H, d, d))
+    slots = [3, -1, 0, 4]
+    q, k, v = (rng.standard_normal((len(slots), H, d)) for _ in range(3))
+    o, pool2 = oracle.decode_step_slots(q, k, v, pool, slots)
+    assert not np.any(o[1])
+    assert np.array_equal(pool2[1], pool[1]) and np.array_equal(pool2[2], pool[2])
+    for b, s in enumerate(slots):
+        if s < 0:
+            continue
+        want = np.einsum("hd,hde->he", q[b], pool[s] + np.einsum("hd,he->hde", k[b], v[b]))
+        assert _rel(o[b], want) < 1e-12
+        assert _rel(pool2[s], pool[s] + np.einsum("hd,he->hde", k[b], v[b])) < 1e-12
+    # the 8-bit form over the same slots: padding rows untouched as well
+    c, a = orc.state_quantize_q8(pool.astype(np.float32))
+    qf, kf, vf = (x.astype(np.float32) for x in (q, k, v))
+    o8, c2, a2 = oracle.decode_step_q8(qf, kf, vf, c, a, slots)
+    assert not np.any(o8[1]) and np.array_equal(c2[1], c[1]) and np.array_equal(a2[2], a[2])
+    o_dense, c_dense, a_dense = orc.decode_step_q8(qf[0], kf[0], vf[0], c[3], a[3])
+    assert np.array_equal(o8[0], o_dense) and np.array_equal(c2[3], c_dense)
+
+
 PINS = [pin_golden, pin_forms_agree, pin_state_is_KtV, pin_last_row, pin_d1_prefix_sum, pin_N1,
         pin_ternary_bruteforce, pin_state_in, pin_decode, pin_varlen, pin_backward_finite_differences,
-        pin_backward_d1_sums]
+        pin_backward_d1_sums, pin_q8_golden, pin_q8_integer_trajectory, pin_q8_within_rounding_bound,
+        pin_decode_slots]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -257,6 +360,13 @@ MUTANTS = {
     "backward_dq_uses_q": ("DQ[t * d + c] += gv * K[s * d + c];", "DQ[t * d + c] += gv * Q[s * d + c];"),
     "backward_dk_wrong_token": ("DK[s * d + c] += gv * Q[t * d + c];", "DK[s * d + c] += gv * Q[s * d + c];"),
     "backward_drops_diagonal": ("for (long s = 0; s <= t; s++) {", "for (long s = 0; s < t; s++) {"),
+    "q8_truncates": ("rintf(x[j] * inv)", "truncf(x[j] * inv)"),
+    "q8_signed_max": ("const float ax = fabsf(x[j]);", "const float ax = x[j];"),
+    "q8_no_small_row_cut": ("if (m < 0x1p-100f) {", "if (m <= 0.0f) {"),
+    "q8_transposed_update": ("fmaf(kb[i], vb[j], deq)", "fmaf(kb[j], vb[i], deq)"),
+    "q8_column_scale": ("(float)cb[i * d + j] * ab[i]", "(float)cb[i * d + j] * ab[j]"),
+    "q8_reads_before_update": ("acc += (double)qb[i] * (double)s[i * d + j];",
+                               "acc += (double)qb[i] * (double)cb[i * d + j] * ab[i];"),
 }
 
 
@@ -277,7 +387,8 @@ def test_pins_catch_planted_mistakes(name):
     assert src.count(old) == 1, "mutation anchor must occur exactly once"
     if name == "decode_reads_before_update":
         # move the state update after the read: o = q S_old, then S += k^T v
-        read_end = "            o[bh * d + j] = acc;\n        }\n"
+        read_end = ("            for (long i = 0; i < d; ++i) acc += qb[i] * Sb[i * d + j];\n"
+                    "            o[bh * d + j] = acc;\n        }\n")
         assert src.count(read_end) == 1
         mutated = src.replace(old, "").replace(read_end, read_end + old)
     else:
