@@ -53,7 +53,8 @@ typedef enum {
     LA_ERR_CUDA = -3,          /* a CUDA runtime/driver call failed           */
     LA_ERR_ALLOC = -4,         /* workspace allocation failed                 */
     LA_ERR_TIMEOUT = -5,       /* a bounded device-side wait gave up          */
-    LA_ERR_BAD_SEQLENS = -6    /* cu_seqlens not 0..total_tokens non-decreasing */
+    LA_ERR_BAD_SEQLENS = -6,   /* cu_seqlens not 0..total_tokens non-decreasing */
+    LA_ERR_BAD_SLOT = -7       /* a decode slot id >= num_slots (row skipped)  */
 } la_status;
 
 typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
@@ -198,6 +199,57 @@ int la_state_prefix(const float* states, int R, int rank, float* prefix_out, int
  */
 int la_decode_step(const void* q, const void* k, const void* v, float* state, void* o,
                    int B, int H, int d, la_dtype dt, void* stream);
+
+/*
+ * la_decode_step_slots -- batched decode over a pool of states.  Section 3 of
+ * the futurefh page pads batches in several levels to keep padding overhead
+ * small; here row b of a batch padded to B rows addresses the state
+ * state_pool[slots[b]], and a row with a negative slot is padding: its o row
+ * is written as zeros and no state is read or written.  So a batch padded up
+ * to a fixed level (for one captured CUDA graph per level) costs state
+ * traffic only for its live rows.
+ *   q, k, v  : [B, H, d] of dt (read only);  o : [B, H, d] of dt (written)
+ *   state_pool: [num_slots, H, d, d] fp32, live slots updated in place
+ *   slots    : [B] int32 on the device; NULL means row b uses slot b (then
+ *              num_slots >= B).  Each live slot may appear once per call
+ *              (a repeated slot gives an unspecified result for that slot, but
+ *              no access outside the pool).
+ * A slot >= num_slots is recorded as LA_ERR_BAD_SLOT in the device status and
+ * its row is treated as padding.
+ */
+int la_decode_step_slots(const void* q, const void* k, const void* v, float* state_pool,
+                         const int32_t* slots, int num_slots, void* o, int B, int H, int d,
+                         la_dtype dt, void* stream);
+
+/*
+ * 8-bit decode state.  The yuliangy.com digest of the MiniMax-01 report
+ * credits 8-bit quantisation with fitting more than a million tokens on one
+ * eight-GPU machine; the format is this library's reading: row i of a head's
+ * state (key dimension i) is int8 codes c_ij in [-127, 127] plus one fp32
+ * scale a_i, S_ij = c_ij * a_i.  Quantising a row: m = max_j |x_j|; if
+ * m < 2^-100 the row is stored as zero (a = 0); else a = m / 127 and
+ * c_j = nearest-even integer to x_j * (127 / m), each one correctly rounded
+ * fp32 operation, so results are reproducible bit for bit.
+ *   codes : [n_heads, d, d] int8;  scales : [n_heads, d] fp32 (16-byte aligned)
+ *
+ * la_state_quantize_q8   fp32 states [n_heads, d, d] -> (codes, scales)
+ * la_state_dequantize_q8 (codes, scales) -> fp32 states (one fp32 product each)
+ *
+ * la_decode_step_q8 -- la_decode_step_slots on the 8-bit state:
+ *     s_ij = fma(k_i, v_j, c_ij * a_i)   (fp32, rounded once)
+ *     o_j  = sum_i q_i s_ij               (fp32 accumulation)
+ *     codes, scales <- the rows of s quantised as above
+ *   codes : [num_slots, H, d, d] int8, scales : [num_slots, H, d] fp32, in place
+ *   slots, padding rows and LA_ERR_BAD_SLOT as for la_decode_step_slots.
+ * State traffic per head-step is 2 (d*d + 4 d) bytes against 8 d*d for fp32.
+ */
+int la_state_quantize_q8(const float* state, int8_t* codes, float* scales, long long n_heads, int d,
+                         void* stream);
+int la_state_dequantize_q8(const int8_t* codes, const float* scales, float* state, long long n_heads,
+                           int d, void* stream);
+int la_decode_step_q8(const void* q, const void* k, const void* v, int8_t* codes, float* scales,
+                      const int32_t* slots, int num_slots, void* o, int B, int H, int d, la_dtype dt,
+                      void* stream);
 
 /* Human-readable name of an la_status value (static storage). */
 const char* la_status_string(int status);

@@ -28,6 +28,7 @@ LA_ERR_CUDA = -3
 LA_ERR_ALLOC = -4
 LA_ERR_TIMEOUT = -5
 LA_ERR_BAD_SEQLENS = -6
+LA_ERR_BAD_SLOT = -7
 
 LA_F32 = 0
 LA_BF16 = 1
@@ -50,7 +51,8 @@ EXPORTED = ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step"
             "la_timing_enable", "la_timing_read", "la_kernel_name", "la_prefill_noalloc",
             "la_prefill_main_kernel", "la_prefill_from_state", "la_prefill_varlen_from_state",
             "la_state_increment", "la_state_prefix", "la_prefill_backward",
-            "la_prefill_varlen_ex")
+            "la_prefill_varlen_ex", "la_decode_step_slots", "la_decode_step_q8",
+            "la_state_quantize_q8", "la_state_dequantize_q8")
 
 LA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -84,6 +86,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la_state_prefix.argtypes = [vp, i, i, vp, i, i, i, vp]
     lib.la_prefill_varlen_from_state.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i]
     lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, vp]
+    lib.la_decode_step_slots.argtypes = [vp, vp, vp, vp, vp, i, vp, i, i, i, i, vp]
+    lib.la_decode_step_q8.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, i, i, i, i, vp]
+    ll = ctypes.c_longlong
+    lib.la_state_quantize_q8.argtypes = [vp, vp, vp, ll, i, vp]
+    lib.la_state_dequantize_q8.argtypes = [vp, vp, vp, ll, i, vp]
     lib.la_status_string.argtypes = [i]
     lib.la_status_string.restype = ctypes.c_char_p
     lib.la_get_last_error.argtypes = []
@@ -100,7 +107,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                  "la_get_last_error", "la_device_sm_count", "la_timing_enable",
                  "la_timing_read", "la_prefill_noalloc", "la_prefill_from_state",
                  "la_prefill_varlen_from_state", "la_state_increment", "la_state_prefix",
-                 "la_prefill_backward"):
+                 "la_prefill_backward", "la_decode_step_slots", "la_decode_step_q8",
+                 "la_state_quantize_q8", "la_state_dequantize_q8"):
         getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -166,6 +174,24 @@ def la_prefill_varlen_ex(q, k, v, o, state_out, cu_seqlens, num_seqs, total_toke
 
 def la_decode_step(q, k, v, state, o, B, H, d, dt, stream):
     return load_library().la_decode_step(q, k, v, state, o, B, H, d, dt, stream)
+
+
+def la_decode_step_slots(q, k, v, state_pool, slots, num_slots, o, B, H, d, dt, stream):
+    return load_library().la_decode_step_slots(q, k, v, state_pool, slots, num_slots, o, B, H, d,
+                                               dt, stream)
+
+
+def la_decode_step_q8(q, k, v, codes, scales, slots, num_slots, o, B, H, d, dt, stream):
+    return load_library().la_decode_step_q8(q, k, v, codes, scales, slots, num_slots, o, B, H, d,
+                                            dt, stream)
+
+
+def la_state_quantize_q8(state, codes, scales, n_heads, d, stream):
+    return load_library().la_state_quantize_q8(state, codes, scales, n_heads, d, stream)
+
+
+def la_state_dequantize_q8(codes, scales, state, n_heads, d, stream):
+    return load_library().la_state_dequantize_q8(codes, scales, state, n_heads, d, stream)
 
 
 def la_status_string(status):
@@ -345,4 +371,82 @@ def decode_step(q, k, v, state, out=None, stream=None):
     status = la_decode_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), state.data_ptr(),
                             o.data_ptr(), B, H, d, _dtype_code(q), _stream_ptr(stream))
     _raise(status, "la_decode_step")
+    return o
+
+
+def _slots_arg(slots, B, torch):
+    if slots is None:
+        return None
+    _check(slots, "slots")
+    if slots.dtype != torch.int32 or slots.shape != (B,):
+        raise ValueError("slots must be an int32 tensor of shape [B]")
+    return slots.data_ptr()
+
+
+def decode_step_slots(q, k, v, state_pool, slots, out=None, stream=None):
+    """Decode step where row b of the [B,H,d] batch updates state_pool[slots[b]]
+    ([num_slots,H,d,d] fp32, in place); rows with a negative slot are padding
+    (zero output, no state access).  ``slots`` is an int32 CUDA tensor [B]."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (state_pool, "state_pool")):
+        _check(t, n)
+    if state_pool.dtype != torch.float32:
+        raise TypeError("state_pool must be float32")
+    B, H, d = q.shape
+    if state_pool.dim() != 4 or state_pool.shape[1:] != (H, d, d):
+        raise ValueError("state_pool must be [num_slots, H, d, d]")
+    o = out if out is not None else torch.empty_like(q)
+    status = la_decode_step_slots(q.data_ptr(), k.data_ptr(), v.data_ptr(), state_pool.data_ptr(),
+                                  _slots_arg(slots, B, torch), state_pool.shape[0], o.data_ptr(),
+                                  B, H, d, _dtype_code(q), _stream_ptr(stream))
+    _raise(status, "la_decode_step_slots")
+    return o
+
+
+def decode_step_q8(q, k, v, codes, scales, slots=None, out=None, stream=None):
+    """Decode step on the 8-bit state: ``codes`` [num_slots,H,d,d] int8 and
+    ``scales`` [num_slots,H,d] fp32, updated in place; ``slots`` as for
+    ``decode_step_slots`` (None: row b uses slot b)."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (codes, "codes"), (scales, "scales")):
+        _check(t, n)
+    if codes.dtype != torch.int8 or scales.dtype != torch.float32:
+        raise TypeError("codes must be int8 and scales float32")
+    B, H, d = q.shape
+    if codes.dim() != 4 or codes.shape[1:] != (H, d, d) or scales.shape != codes.shape[:3]:
+        raise ValueError("codes must be [num_slots, H, d, d] and scales [num_slots, H, d]")
+    o = out if out is not None else torch.empty_like(q)
+    status = la_decode_step_q8(q.data_ptr(), k.data_ptr(), v.data_ptr(), codes.data_ptr(),
+                               scales.data_ptr(), _slots_arg(slots, B, torch), codes.shape[0],
+                               o.data_ptr(), B, H, d, _dtype_code(q), _stream_ptr(stream))
+    _raise(status, "la_decode_step_q8")
+    return o
+
+
+def state_quantize_q8(state, codes=None, scales=None, stream=None):
+    """fp32 states [..., d, d] -> (int8 codes [..., d, d], fp32 scales [..., d])."""
+    torch = _torch()
+    _check(state, "state")
+    if state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    d = state.shape[-1]
+    c = codes if codes is not None else torch.empty(state.shape, dtype=torch.int8, device=state.device)
+    a = scales if scales is not None else torch.empty(state.shape[:-1], dtype=torch.float32,
+                                                      device=state.device)
+    status = la_state_quantize_q8(state.data_ptr(), c.data_ptr(), a.data_ptr(),
+                                  state.numel() // (d * d), d, _stream_ptr(stream))
+    _raise(status, "la_state_quantize_q8")
+    return c, a
+
+
+def state_dequantize_q8(codes, scales, out=None, stream=None):
+    """(codes, scales) -> fp32 states, S_ij = c_ij * a_i."""
+    torch = _torch()
+    _check(codes, "codes")
+    _check(scales, "scales")
+    d = codes.shape[-1]
+    o = out if out is not None else torch.empty(codes.shape, dtype=torch.float32, device=codes.device)
+    status = la_state_dequantize_q8(codes.data_ptr(), scales.data_ptr(), o.data_ptr(),
+                                    codes.numel() // (d * d), d, _stream_ptr(stream))
+    _raise(status, "la_state_dequantize_q8")
     return o

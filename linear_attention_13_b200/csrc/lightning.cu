@@ -628,6 +628,56 @@ int launch_prefill_bf16_noalloc(const void* q, const void* k, const void* v, voi
 
 using namespace la;
 
+namespace {
+
+int decode_args_ok(const void* q, const void* k, const void* v, const void* o, int B, int H, int d,
+                   la_dtype dt) {
+    if (B < 1 || H < 1) return LA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LA_ERR_INVALID_ARG;
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1ll << 31) - 1) return LA_ERR_INVALID_ARG;
+    return LA_OK;
+}
+
+int slots_ok(const int32_t* slots, int num_slots, int B, int H) {
+    if (slots == nullptr) return num_slots >= B ? LA_OK : LA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(slots) & 3u) != 0 || num_slots < 1) return LA_ERR_INVALID_ARG;
+    if ((long long)num_slots * H > (1ll << 31) - 1) return LA_ERR_INVALID_ARG;
+    return LA_OK;
+}
+
+template <typename T>
+void launch_decode(const void* q, const void* k, const void* v, float* state, void* o,
+                   const int32_t* slots, int num_slots, int B, int H, int d, cudaStream_t s) {
+    const T* qt = reinterpret_cast<const T*>(q);
+    const T* kt = reinterpret_cast<const T*>(k);
+    const T* vt = reinterpret_cast<const T*>(v);
+    T* ot = reinterpret_cast<T*>(o);
+    const unsigned grid = (unsigned)(B * H);
+    if (d == 128)
+        decode::decode_step_kernel<T, 128><<<grid, decode::kThreads, 0, s>>>(qt, kt, vt, state, ot, slots, H, num_slots);
+    else
+        decode::decode_step_kernel<T, 64><<<grid, decode::kThreads, 0, s>>>(qt, kt, vt, state, ot, slots, H, num_slots);
+}
+
+template <typename T>
+void launch_decode_q8(const void* q, const void* k, const void* v, int8_t* codes, float* scales,
+                      void* o, const int32_t* slots, int num_slots, int B, int H, int d, cudaStream_t s) {
+    const T* qt = reinterpret_cast<const T*>(q);
+    const T* kt = reinterpret_cast<const T*>(k);
+    const T* vt = reinterpret_cast<const T*>(v);
+    T* ot = reinterpret_cast<T*>(o);
+    const unsigned grid = (unsigned)(B * H);
+    if (d == 128)
+        decode::decode_step_q8_kernel<T, 128><<<grid, decode::kThreads, 0, s>>>(qt, kt, vt, codes, scales, ot, slots, H, num_slots);
+    else
+        decode::decode_step_q8_kernel<T, 64><<<grid, decode::kThreads, 0, s>>>(qt, kt, vt, codes, scales, ot, slots, H, num_slots);
+}
+
+}  // namespace
+
 extern "C" {
 
 namespace {
@@ -859,38 +909,81 @@ int la_state_prefix(const float* states, int R, int rank, float* prefix_out, int
 
 int la_decode_step(const void* q, const void* k, const void* v, float* state, void* o, int B, int H,
                    int d, la_dtype dt, void* stream) {
-    if (B < 1 || H < 1) return LA_ERR_INVALID_ARG;
-    if (!q || !k || !v || !o || !state) return LA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state))
-        return LA_ERR_INVALID_ARG;
-    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    return la_decode_step_slots(q, k, v, state, nullptr, B, o, B, H, d, dt, stream);
+}
+
+int la_decode_step_slots(const void* q, const void* k, const void* v, float* state_pool,
+                         const int32_t* slots, int num_slots, void* o, int B, int H, int d,
+                         la_dtype dt, void* stream) {
+    int st = decode_args_ok(q, k, v, o, B, H, d, dt);
+    if (st != LA_OK) return st;
+    if (!state_pool || !aligned16(state_pool)) return LA_ERR_INVALID_ARG;
+    if ((st = slots_ok(slots, num_slots, B, H)) != LA_OK) return st;
+    int dev = 0, sms = 0;
+    if ((st = device_setup(&dev, &sms)) != LA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    TimedLaunch tl(LA_KERNEL_DECODE, s);
+    if (dt == LA_BF16)
+        launch_decode<__nv_bfloat16>(q, k, v, state_pool, o, slots, num_slots, B, H, d, s);
+    else
+        launch_decode<float>(q, k, v, state_pool, o, slots, num_slots, B, H, d, s);
+    return note_cuda(cudaGetLastError());
+}
+
+int la_decode_step_q8(const void* q, const void* k, const void* v, int8_t* codes, float* scales,
+                      const int32_t* slots, int num_slots, void* o, int B, int H, int d, la_dtype dt,
+                      void* stream) {
+    int st = decode_args_ok(q, k, v, o, B, H, d, dt);
+    if (st != LA_OK) return st;
+    if (!codes || !scales || !aligned16(codes) || !aligned16(scales)) return LA_ERR_INVALID_ARG;
+    if ((st = slots_ok(slots, num_slots, B, H)) != LA_OK) return st;
+    int dev = 0, sms = 0;
+    if ((st = device_setup(&dev, &sms)) != LA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    TimedLaunch tl(LA_KERNEL_DECODE, s);
+    if (dt == LA_BF16)
+        launch_decode_q8<__nv_bfloat16>(q, k, v, codes, scales, o, slots, num_slots, B, H, d, s);
+    else
+        launch_decode_q8<float>(q, k, v, codes, scales, o, slots, num_slots, B, H, d, s);
+    return note_cuda(cudaGetLastError());
+}
+
+int la_state_quantize_q8(const float* state, int8_t* codes, float* scales, long long n_heads, int d,
+                         void* stream) {
+    if (n_heads < 1 || !state || !codes || !scales) return LA_ERR_INVALID_ARG;
+    if (!aligned16(state) || !aligned16(codes) || !aligned16(scales)) return LA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
-    if ((long long)B * H > (1ll << 31) - 1) return LA_ERR_INVALID_ARG;
     int dev = 0, sms = 0;
     int st = device_setup(&dev, &sms);
     if (st != LA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const unsigned grid = (unsigned)(B * H);
-    TimedLaunch tl(LA_KERNEL_DECODE, s);
-    if (dt == LA_BF16) {
-        const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(q);
-        const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(k);
-        const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(v);
-        __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(o);
-        if (d == 128)
-            decode::decode_step_kernel<__nv_bfloat16, 128><<<grid, decode::kThreads, 0, s>>>(qb, kb, vb, state, ob);
-        else
-            decode::decode_step_kernel<__nv_bfloat16, 64><<<grid, decode::kThreads, 0, s>>>(qb, kb, vb, state, ob);
-    } else {
-        const float* qf = reinterpret_cast<const float*>(q);
-        const float* kf = reinterpret_cast<const float*>(k);
-        const float* vf = reinterpret_cast<const float*>(v);
-        float* of = reinterpret_cast<float*>(o);
-        if (d == 128)
-            decode::decode_step_kernel<float, 128><<<grid, decode::kThreads, 0, s>>>(qf, kf, vf, state, of);
-        else
-            decode::decode_step_kernel<float, 64><<<grid, decode::kThreads, 0, s>>>(qf, kf, vf, state, of);
-    }
+    const long long rows = n_heads * d;
+    const long long warps_needed = (rows * (d / 4) + 31) / 32;
+    const int grid = (int)std::min<long long>((warps_needed + 7) / 8, 8LL * sms);
+    TimedLaunch tl(LA_KERNEL_AUX, s);
+    if (d == 128)
+        decode::state_quantize_q8_kernel<128><<<grid, 256, 0, s>>>(state, codes, scales, rows);
+    else
+        decode::state_quantize_q8_kernel<64><<<grid, 256, 0, s>>>(state, codes, scales, rows);
+    return note_cuda(cudaGetLastError());
+}
+
+int la_state_dequantize_q8(const int8_t* codes, const float* scales, float* state, long long n_heads,
+                           int d, void* stream) {
+    if (n_heads < 1 || !state || !codes || !scales) return LA_ERR_INVALID_ARG;
+    if (!aligned16(state) || !aligned16(codes) || !aligned16(scales)) return LA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
+    int dev = 0, sms = 0;
+    int st = device_setup(&dev, &sms);
+    if (st != LA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const long long n4 = n_heads * d * d / 4;
+    const int grid = (int)std::min<long long>((n4 + 255) / 256, 8LL * sms);
+    TimedLaunch tl(LA_KERNEL_AUX, s);
+    if (d == 128)
+        decode::state_dequantize_q8_kernel<128><<<grid, 256, 0, s>>>(codes, scales, state, n4);
+    else
+        decode::state_dequantize_q8_kernel<64><<<grid, 256, 0, s>>>(codes, scales, state, n4);
     return note_cuda(cudaGetLastError());
 }
 
@@ -903,6 +996,7 @@ const char* la_status_string(int status) {
         case LA_ERR_ALLOC: return "LA_ERR_ALLOC";
         case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT";
         case LA_ERR_BAD_SEQLENS: return "LA_ERR_BAD_SEQLENS";
+        case LA_ERR_BAD_SLOT: return "LA_ERR_BAD_SLOT";
         default: return "LA_UNKNOWN_STATUS";
     }
 }
