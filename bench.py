@@ -13,17 +13,19 @@ schedule the library picks for it.  Inputs (384 MiB) and outputs exceed the
   roofline  the dominant kernel (the prefill output pass; the variant the
             library dispatched is named) against measured HBM
             bandwidth: algorithmic bytes per launch / CUDA-event launch time
-  secondary decode GB/s (128 seq x 64 heads, 256 steps), long-context prefill
-            (B=1, H=64, N=262144), the bf16 blk=64 prefill and the packed
-            varlen prefill where supported (single-GPU runs only)
+  secondary decode GB/s (128 seq x 64 heads, 256 steps) with the fp32 and the
+            8-bit state (and a batch padded from 96 live rows to 128),
+            long-context prefill (B=1, H=64, N=262144), the bf16 blk=64
+            prefill and the packed varlen prefill where supported (single-GPU
+            runs only)
 
 ``--impl reference`` times the fp64 CPU oracle (the reference arm of this
 build) on a bounded sample of the same workload.
 
 ``--profile-case NAME`` runs one workload for --warmup + --steps calls with no
 timing and prints a one-line summary: the command the ncu summaries under
-profiles/ were captured with (prefill, prefill_blk64, decode, long_prefill_32k,
-varlen_32k).
+profiles/ were captured with (prefill, prefill_blk64, decode, decode_q8,
+long_prefill_32k, varlen_32k).
 """
 from __future__ import annotations
 
@@ -489,7 +491,43 @@ def bench_secondary(args, device, stream, peaks):
         "kernel_GB/s": round(bytes_step / (k_ms / 1e3) / 1e9, 1),
         "hbm_frac": round(bytes_step / (k_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
         "bytes_per_step": bytes_step}
-    del step_inputs, S, od
+
+    # -- the same decode on the 8-bit state (int8 codes + one fp32 scale per
+    #    key row), all 128 rows live, then a batch padded from 96 live rows to
+    #    a 128-row level through the slot pool
+    codes, scales = la.state_quantize_q8(S)
+    del S
+    torch.cuda.empty_cache()
+
+    def qstep(slots=None):
+        i = next(it) % steps
+        qq, kk, vv = step_inputs[i]
+        la.decode_step_q8(qq, kk, vv, codes, scales, slots, out=od)
+
+    la.la_timing_enable(steps + 64)
+    ms = timed(stream, qstep, steps, 5, solo, device)
+    kt = kernel_times(la)
+    la.la_timing_enable(0)
+    dec = kt.get("decode_step_kernel", {"total_ms": float("nan"), "launches": 1})
+    k_ms = dec["total_ms"] / max(dec["launches"], 1)
+    bytes_q8 = n_seq * Hd * (2 * (D * D + 4 * D) + 8 * D)
+    padded = torch.tensor(list(range(96)) + [-1] * 32, dtype=torch.int32, device=device)
+    la.la_timing_enable(steps + 64)
+    ms_pad = timed(stream, lambda: qstep(padded), steps, 5, solo, device)
+    kt_pad = kernel_times(la)
+    la.la_timing_enable(0)
+    dec_pad = kt_pad.get("decode_step_kernel", {"total_ms": float("nan"), "launches": 1})
+    out["decode_q8"] = {
+        "workload": "decode step, 128 seq x 64 heads, d=128, 8-bit state (int8 + fp32 row scales), "
+                    "256 steps",
+        "ms_per_step": round(ms / steps, 5), "kernel_ms": round(k_ms, 5),
+        "kernel_GB/s": round(bytes_q8 / (k_ms / 1e3) / 1e9, 1),
+        "hbm_frac": round(bytes_q8 / (k_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+        "bytes_per_step": bytes_q8,
+        "speedup_vs_fp32_state_kernel": round(out["decode"]["bytes_per_step"] /
+                                              out["decode"]["kernel_GB/s"] / 1e9 / (k_ms / 1e3), 3),
+        "padded_96_of_128_kernel_ms": round(dec_pad["total_ms"] / max(dec_pad["launches"], 1), 5)}
+    del step_inputs, codes, scales, od
     torch.cuda.empty_cache()
 
     # -- long-context prefill B=1 H=64 N=262144
@@ -541,6 +579,7 @@ PROFILE_CASES = {
     "prefill": "prefill bf16 B=4 H=16 N=8192 d=128 blk=128 (the headline launch)",
     "prefill_blk64": "prefill bf16 B=4 H=16 N=8192 d=128 blk=64",
     "decode": "decode step, 128 seq x 64 heads, d=128, fp32 state (random state)",
+    "decode_q8": "decode step, 128 seq x 64 heads, d=128, 8-bit state (random state, quantised)",
     "long_prefill_32k": "prefill bf16 B=1 H=64 N=32768 d=128 blk=128 (long-context shape, "
                         "1/8 of the length)",
     "varlen_32k": "packed prefill bf16 T=2^15, lengths U[1024,8192] seed 0, H=64, d=128",
@@ -573,6 +612,15 @@ def profile_case(args):
 
         def call():
             la.decode_step(qq, kk, vv, S, out=od)
+    elif name == "decode_q8":
+        n_seq, Hd = 128, 64
+        codes, scales = la.state_quantize_q8(
+            torch.randn((n_seq, Hd, D, D), dtype=torch.float32, device=device))
+        qq, kk, vv = inputs.decode_step_inputs(n_seq, Hd, D, 1, device=device)
+        od = torch.empty((n_seq, Hd, D), dtype=torch.bfloat16, device=device)
+
+        def call():
+            la.decode_step_q8(qq, kk, vv, codes, scales, out=od)
     elif name == "varlen_32k":
         Tv, Hv = 1 << 15, 64
         lens = inputs.varlen_lengths(Tv, 1024, 8192, seed=0)

@@ -27,6 +27,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace la {
 namespace decode {
@@ -213,6 +214,39 @@ __device__ __forceinline__ float4 codes_to_f32(int packed) {
     return r;
 }
 
+// Packed (two fp32 lanes per instruction, sm_100) forms of the same steps.
+// Each half is the identical correctly rounded fp32 operation as the scalar
+// form.  The packed multiply may be fused by the compiler with a packed add
+// that consumes it (one rounding instead of two: near-tie codes moved by one
+// when that happened), so no packed product here feeds a packed add: the
+// quantising product stays a scalar __fmul_rn, which is never contracted, and
+// the dequantising product feeds only the addend of a fused multiply-add.
+struct Row4 {
+    float2 lo, hi;   // columns 4c, 4c+1 and 4c+2, 4c+3
+};
+
+__device__ __forceinline__ Row4 codes_to_f32x2(int packed) {
+    constexpr float kBias = 8388736.0f;     // 2^23 + 128, as in codes_to_f32
+    const unsigned u = (unsigned)packed ^ 0x80808080u;
+    const float2 nb = make_float2(-kBias, -kBias);
+    Row4 r;
+    r.lo = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440u)),
+                                  __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7441u))), nb);
+    r.hi = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7442u)),
+                                  __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7443u))), nb);
+    return r;
+}
+
+__device__ __forceinline__ int pack4_q8x2(const Row4& s, float inv) {
+    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23, as in pack4_q8
+    const float2 rr = make_float2(kRound, kRound);
+    const float2 tl = __fadd2_rn(make_float2(__fmul_rn(s.lo.x, inv), __fmul_rn(s.lo.y, inv)), rr);
+    const float2 th = __fadd2_rn(make_float2(__fmul_rn(s.hi.x, inv), __fmul_rn(s.hi.y, inv)), rr);
+    const unsigned lo = __byte_perm(__float_as_uint(tl.x), __float_as_uint(tl.y), 0x0040u);
+    const unsigned hi = __byte_perm(__float_as_uint(th.x), __float_as_uint(th.y), 0x0040u);
+    return (int)__byte_perm(lo, hi, 0x5410u);
+}
+
 // N consecutive values of a row-vector (q or k rows of one lane) as fp32,
 // with 16- or 8-byte loads (the offsets used are multiples of the load size).
 template <typename T, int N>
@@ -286,104 +320,154 @@ __device__ __forceinline__ float row_max_scatter(const float (&lm)[R], int lane_
     return cur[0];
 }
 
-// One decode step on the 8-bit state.  Same thread layout as
-// decode_step_kernel: a lane owns 4 value columns (one 32-bit word of codes)
-// of kRowsPer rows, and the kCols4 lanes of a row are consecutive lanes of one
-// warp.  The rows' maxima come from row_max_scatter; the lanes holding a row's
-// max compute its 127 / m and m / 127 and pass 127 / m back by shuffle.
+// One decode step on the 8-bit state.  Persistent CTAs walk the batch rows
+// (b, h) with a stride of the grid; thread 0 streams each row's codes and
+// scales into a ring of kQ8Stages shared-memory stages with bulk copies
+// (cp.async.bulk, completion on an mbarrier), so the loads of the next rows
+// overlap the arithmetic of this one.  Compute layout as decode_step_kernel:
+// a lane owns 4 value columns (one 32-bit word of codes) of kRowsPer rows, and
+// the kCols4 lanes of a row are consecutive lanes of one warp.  The rows'
+// maxima come from row_max_scatter; the lanes holding a row's max compute its
+// 127 / m and m / 127 and pass 127 / m back by shuffle.  New codes and scales
+// go straight from registers to global memory.
+constexpr int kQ8Stages = 4;
+
+template <int D>
+struct Q8Smem {
+    static constexpr int kCodeBytes = D * D;
+    static constexpr int kScaleBytes = D * 4;
+    static constexpr int kStageBytes = kCodeBytes + kScaleBytes;
+    static constexpr int kRowGroups = kThreads / (D / 4);
+    static constexpr int kRedOff = kQ8Stages * kStageBytes;                 // float4 red[2][groups][D/4]
+    static constexpr int kCtrlOff = kRedOff + 2 * kRowGroups * (D / 4) * 16;
+    static constexpr int kBytes = kCtrlOff + 128;                           // mbarriers, slot ids, flag
+};
+
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 decode_step_q8_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                       int8_t* __restrict__ codes, float* __restrict__ scales, T* __restrict__ o,
-                      const int32_t* __restrict__ slots, int H, int num_slots) {
+                      const int32_t* __restrict__ slots, int H, int num_slots, long long n_rows) {
+    using L = Q8Smem<D>;
     constexpr int kCols4 = D / 4;                       // lanes per row
-    constexpr int kRowGroups = kThreads / kCols4;
+    constexpr int kRowGroups = L::kRowGroups;
     constexpr int kRowsPer = D / kRowGroups;            // rows per lane
     constexpr int kHolders = kCols4 / kRowsPer;         // lanes holding one row's max
     static_assert(kCols4 * kRowGroups == kThreads && kRowsPer % 4 == 0 && kRowsPer <= kCols4, "layout");
 
-    __shared__ float4 red[kRowGroups][kCols4];
-    const size_t head = blockIdx.x;
-    const long long sh = state_head(head, slots, H, num_slots);
-    if (sh < 0) {
-        write_zero_row<T, D>(o, head);
-        return;
+    extern __shared__ __align__(128) uint8_t smem[];
+    float4* red = reinterpret_cast<float4*>(smem + L::kRedOff);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kCtrlOff);
+    long long* stage_head = reinterpret_cast<long long*>(smem + L::kCtrlOff + 8 * kQ8Stages);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kCtrlOff + 16 * kQ8Stages);
+    auto bar = [&](int s) { return ptx::smem_u32(bars + s); };
+    const uint32_t stage0 = ptx::smem_u32(smem);
+
+    const long long G = gridDim.x;
+    // thread 0: resolve the slot of the j-th row of this CTA and start its copies
+    auto issue = [&](long long j) {
+        const long long r = blockIdx.x + j * G;
+        if (r >= n_rows) return;
+        const int s = (int)(j % kQ8Stages);
+        const long long sh = state_head((size_t)r, slots, H, num_slots);
+        stage_head[s] = sh;
+        if (sh < 0) {
+            ptx::mbar_arrive(bar(s));
+            return;
+        }
+        ptx::mbar_arrive_expect_tx(bar(s), L::kStageBytes);
+        const uint32_t dst = stage0 + s * L::kStageBytes;
+        ptx::bulk_load(dst, codes + (size_t)sh * L::kCodeBytes, L::kCodeBytes, bar(s));
+        ptx::bulk_load(dst + L::kCodeBytes, scales + (size_t)sh * D, L::kScaleBytes, bar(s));
+    };
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < kQ8Stages; ++s) ptx::mbar_init(bar(s), 1);
+        ptx::fence_mbar_init();
     }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        for (int j = 0; j < kQ8Stages; ++j) issue(j);
+
     const int cg = threadIdx.x % kCols4;
     const int rg = threadIdx.x / kCols4;
     const int row0 = rg * kRowsPer;
-
-    int* C = reinterpret_cast<int*>(codes + (size_t)sh * D * D);
-    float* A = scales + (size_t)sh * D;
-    int c[kRowsPer];
+    long long j = 0;
+    for (; blockIdx.x + j * G < n_rows; ++j) {
+        const size_t head = (size_t)(blockIdx.x + j * G);
+        const int s = (int)(j % kQ8Stages);
+        float kr[kRowsPer], qr[kRowsPer], vc[4];
+        load_f32<T, kRowsPer>(k + head * D + row0, kr);
+        load_f32<T, kRowsPer>(q + head * D + row0, qr);
+        load_f32<T, 4>(v + head * D + 4 * cg, vc);
+        const bool ok = ptx::mbar_wait(bar(s), (uint32_t)((j / kQ8Stages) & 1), abort_flag);
+        const long long sh = stage_head[s];
+        float4* red_j = red + (j & 1) * (kRowGroups * kCols4);
+        if (ok && sh >= 0) {
+            const uint8_t* st = smem + s * L::kStageBytes;
+            const int* Cs = reinterpret_cast<const int*>(st);
+            const float* As = reinterpret_cast<const float*>(st + L::kCodeBytes);
+            Row4 x[kRowsPer];
+            float lm[kRowsPer];
+            float2 acc_lo = make_float2(0.f, 0.f), acc_hi = make_float2(0.f, 0.f);
+            const float2 v_lo = make_float2(vc[0], vc[1]), v_hi = make_float2(vc[2], vc[3]);
 #pragma unroll
-    for (int i = 0; i < kRowsPer; ++i) c[i] = __ldcs(C + (size_t)(row0 + i) * kCols4 + cg);
-    float a[kRowsPer];
+            for (int i = 0; i < kRowsPer; ++i) {
+                const float2 ai = make_float2(As[row0 + i], As[row0 + i]);
+                const float2 ki = make_float2(kr[i], kr[i]);
+                const float2 qi = make_float2(qr[i], qr[i]);
+                x[i] = codes_to_f32x2(Cs[(row0 + i) * kCols4 + cg]);
+                // s = fma(k_i, v_j, c_ij * a_i), then o += q_i s
+                x[i].lo = __ffma2_rn(ki, v_lo, __fmul2_rn(x[i].lo, ai));
+                x[i].hi = __ffma2_rn(ki, v_hi, __fmul2_rn(x[i].hi, ai));
+                acc_lo = __ffma2_rn(qi, x[i].lo, acc_lo);
+                acc_hi = __ffma2_rn(qi, x[i].hi, acc_hi);
+                lm[i] = fmaxf(fmaxf(fabsf(x[i].lo.x), fabsf(x[i].lo.y)), fmaxf(fabsf(x[i].hi.x), fabsf(x[i].hi.y)));
+            }
+            const float m = row_max_scatter<kRowsPer, kCols4>(lm, cg);
+            const bool zero_row = m < kQ8MinRowMax;
+            const float inv_mine = zero_row ? 0.f : __fdiv_rn(127.f, m);
+            const float a_mine = zero_row ? 0.f : __fdiv_rn(m, 127.f);
+            int* C = reinterpret_cast<int*>(codes + (size_t)sh * L::kCodeBytes);
+            if (cg % kHolders == 0) scales[(size_t)sh * D + row0 + cg / kHolders] = a_mine;
 #pragma unroll
-    for (int i = 0; i < kRowsPer; i += 4) {
-        const float4 t = __ldcs(reinterpret_cast<const float4*>(A + row0 + i));
-        a[i] = t.x;
-        a[i + 1] = t.y;
-        a[i + 2] = t.z;
-        a[i + 3] = t.w;
-    }
-    float kr[kRowsPer], qr[kRowsPer], vc[4];
-    load_f32<T, kRowsPer>(k + head * D + row0, kr);
-    load_f32<T, kRowsPer>(q + head * D + row0, qr);
-    load_f32<T, 4>(v + head * D + 4 * cg, vc);
-    const float v0 = vc[0], v1 = vc[1], v2 = vc[2], v3 = vc[3];
-
-    float4 x[kRowsPer];
-    float lm[kRowsPer];
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < kRowsPer; ++i) {
-        const float ki = kr[i];
-        const float qi = qr[i];
-        x[i] = codes_to_f32(c[i]);
-        x[i].x = __fmul_rn(x[i].x, a[i]);
-        x[i].y = __fmul_rn(x[i].y, a[i]);
-        x[i].z = __fmul_rn(x[i].z, a[i]);
-        x[i].w = __fmul_rn(x[i].w, a[i]);
-        x[i].x = __fmaf_rn(ki, v0, x[i].x);
-        x[i].y = __fmaf_rn(ki, v1, x[i].y);
-        x[i].z = __fmaf_rn(ki, v2, x[i].z);
-        x[i].w = __fmaf_rn(ki, v3, x[i].w);
-        acc.x = fmaf(qi, x[i].x, acc.x);
-        acc.y = fmaf(qi, x[i].y, acc.y);
-        acc.z = fmaf(qi, x[i].z, acc.z);
-        acc.w = fmaf(qi, x[i].w, acc.w);
-        lm[i] = fmaxf(fmaxf(fabsf(x[i].x), fabsf(x[i].y)), fmaxf(fabsf(x[i].z), fabsf(x[i].w)));
-    }
-    // scales: the rows' own lanes read them above and every write below
-    // depends on those reads, so the in-place update is ordered
-    const float m = row_max_scatter<kRowsPer, kCols4>(lm, cg);
-    const bool zero_row = m < kQ8MinRowMax;
-    const float inv_mine = zero_row ? 0.f : __fdiv_rn(127.f, m);
-    const float a_mine = zero_row ? 0.f : __fdiv_rn(m, 127.f);
-    if (cg % kHolders == 0) A[row0 + cg / kHolders] = a_mine;
-#pragma unroll
-    for (int i = 0; i < kRowsPer; ++i) {
-        const float inv = __shfl_sync(0xffffffffu, inv_mine, i * kHolders, kCols4);
-        __stcs(C + (size_t)(row0 + i) * kCols4 + cg, pack4_q8(x[i], inv));
-    }
-    red[rg][cg] = acc;
-    __syncthreads();
-    if (rg == 0) {
-        float4 t = red[0][cg];
-#pragma unroll
-        for (int g = 1; g < kRowGroups; ++g) {
-            const float4 u = red[g][cg];
-            t.x += u.x;
-            t.y += u.y;
-            t.z += u.z;
-            t.w += u.w;
+            for (int i = 0; i < kRowsPer; ++i) {
+                const float inv = __shfl_sync(0xffffffffu, inv_mine, i * kHolders, kCols4);
+                __stcs(C + (size_t)(row0 + i) * kCols4 + cg, pack4_q8x2(x[i], inv));
+            }
+            const float4 acc = make_float4(acc_lo.x, acc_lo.y, acc_hi.x, acc_hi.y);
+            red_j[rg * kCols4 + cg] = acc;
         }
-        T* oh = o + head * D;
-        oh[4 * cg + 0] = from_f32<T>(t.x);
-        oh[4 * cg + 1] = from_f32<T>(t.y);
-        oh[4 * cg + 2] = from_f32<T>(t.z);
-        oh[4 * cg + 3] = from_f32<T>(t.w);
+        // every thread is done with stage s and has written its partial sums
+        if (__syncthreads_or(!ok)) break;
+        if (threadIdx.x == 0) issue(j + kQ8Stages);
+        if (sh < 0) {
+            write_zero_row<T, D>(o, head);
+        } else if (rg == 0) {
+            float4 t = red_j[cg];
+#pragma unroll
+            for (int g = 1; g < kRowGroups; ++g) {
+                const float4 u = red_j[g * kCols4 + cg];
+                t.x += u.x;
+                t.y += u.y;
+                t.z += u.z;
+                t.w += u.w;
+            }
+            T* oh = o + head * D;
+            oh[4 * cg + 0] = from_f32<T>(t.x);
+            oh[4 * cg + 1] = from_f32<T>(t.y);
+            oh[4 * cg + 2] = from_f32<T>(t.z);
+            oh[4 * cg + 3] = from_f32<T>(t.w);
+        }
+    }
+    // after a timeout: let the copies already issued land (bounded) before exit
+    if (threadIdx.x == 0 && *abort_flag) {
+        for (long long jj = j; jj < j + kQ8Stages && blockIdx.x + jj * G < n_rows; ++jj) {
+            const unsigned long long t0 = globaltimer_ns();
+            while (!ptx::mbar_try_wait(bar((int)(jj % kQ8Stages)), (uint32_t)((jj / kQ8Stages) & 1)) &&
+                   globaltimer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
     }
 }
 

@@ -80,7 +80,19 @@ int device_setup(int* dev_out, int* sms_out) {
                                  simt::smem_bytes<64>()) != cudaSuccess ||
             cudaFuncSetAttribute(simt::prefill_simt_varlen_kernel<128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 simt::smem_bytes<128>()) != cudaSuccess) {
+                                 simt::smem_bytes<128>()) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::decode_step_q8_kernel<__nv_bfloat16, 128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::Q8Smem<128>::kBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::decode_step_q8_kernel<__nv_bfloat16, 64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::Q8Smem<64>::kBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::decode_step_q8_kernel<float, 128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::Q8Smem<128>::kBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::decode_step_q8_kernel<float, 64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::Q8Smem<64>::kBytes) != cudaSuccess) {
             cudaGetLastError();
             return LA_ERR_CUDA;
         }
@@ -662,18 +674,32 @@ void launch_decode(const void* q, const void* k, const void* v, float* state, vo
         decode::decode_step_kernel<T, 64><<<grid, decode::kThreads, 0, s>>>(qt, kt, vt, state, ot, slots, H, num_slots);
 }
 
+template <typename T, int D>
+int launch_decode_q8_d(const T* q, const T* k, const T* v, int8_t* codes, float* scales, T* o,
+                       const int32_t* slots, int num_slots, int B, int H, int sms, cudaStream_t s) {
+    // the dynamic shared-memory size was opted into by device_setup
+    auto kern = decode::decode_step_q8_kernel<T, D>;
+    const int smem = decode::Q8Smem<D>::kBytes;
+    const long long rows = (long long)B * H;
+    int per_sm = 0;   // resident CTAs per SM (registers bound it: 2 at d = 128, 3 at d = 64)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, decode::kThreads, smem) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int grid = (int)std::min<long long>(rows, (long long)per_sm * sms);
+    kern<<<grid, decode::kThreads, smem, s>>>(q, k, v, codes, scales, o, slots, H, num_slots, rows);
+    return LA_OK;
+}
+
 template <typename T>
-void launch_decode_q8(const void* q, const void* k, const void* v, int8_t* codes, float* scales,
-                      void* o, const int32_t* slots, int num_slots, int B, int H, int d, cudaStream_t s) {
+int launch_decode_q8(const void* q, const void* k, const void* v, int8_t* codes, float* scales,
+                     void* o, const int32_t* slots, int num_slots, int B, int H, int d, int sms,
+                     cudaStream_t s) {
     const T* qt = reinterpret_cast<const T*>(q);
     const T* kt = reinterpret_cast<const T*>(k);
     const T* vt = reinterpret_cast<const T*>(v);
     T* ot = reinterpret_cast<T*>(o);
-    const unsigned grid = (unsigned)(B * H);
-    if (d == 128)
-        decode::decode_step_q8_kernel<T, 128><<<grid, decode::kThreads, 0, s>>>(qt, kt, vt, codes, scales, ot, slots, H, num_slots);
-    else
-        decode::decode_step_q8_kernel<T, 64><<<grid, decode::kThreads, 0, s>>>(qt, kt, vt, codes, scales, ot, slots, H, num_slots);
+    if (d == 128) return launch_decode_q8_d<T, 128>(qt, kt, vt, codes, scales, ot, slots, num_slots, B, H, sms, s);
+    return launch_decode_q8_d<T, 64>(qt, kt, vt, codes, scales, ot, slots, num_slots, B, H, sms, s);
 }
 
 }  // namespace
@@ -941,10 +967,10 @@ int la_decode_step_q8(const void* q, const void* k, const void* v, int8_t* codes
     if ((st = device_setup(&dev, &sms)) != LA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     TimedLaunch tl(LA_KERNEL_DECODE, s);
-    if (dt == LA_BF16)
-        launch_decode_q8<__nv_bfloat16>(q, k, v, codes, scales, o, slots, num_slots, B, H, d, s);
-    else
-        launch_decode_q8<float>(q, k, v, codes, scales, o, slots, num_slots, B, H, d, s);
+    st = dt == LA_BF16
+             ? launch_decode_q8<__nv_bfloat16>(q, k, v, codes, scales, o, slots, num_slots, B, H, d, sms, s)
+             : launch_decode_q8<float>(q, k, v, codes, scales, o, slots, num_slots, B, H, d, sms, s);
+    if (st != LA_OK) return st;
     return note_cuda(cudaGetLastError());
 }
 
