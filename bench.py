@@ -13,7 +13,8 @@ schedule the library picks for it.  Inputs (384 MiB) and outputs exceed the
   roofline  the dominant kernel (the prefill output pass; the variant the
             library dispatched is named) against measured HBM
             bandwidth: algorithmic bytes per launch / CUDA-event launch time
-  secondary decode GB/s (128 seq x 64 heads, 256 steps) with the fp32 and the
+  secondary the backward of the headline prefill (dq, dk, dv), decode GB/s
+            (128 seq x 64 heads, 256 steps) with the fp32 and the
             8-bit state (and a batch padded from 96 live rows to 128),
             long-context prefill (B=1, H=64, N=262144), the bf16 blk=64
             prefill and the packed varlen prefill where supported (single-GPU
@@ -447,6 +448,27 @@ def bench_secondary(args, device, stream, peaks):
                              peaks["bf16_tflops"], 4),
         "kernels": {k_: round(v_["total_ms"] / max(v_["launches"], 1), 5) for k_, v_ in kt.items()}}
     del q, k, v, o, st
+    torch.cuda.empty_cache()
+
+    # -- backward of the same prefill (dq, dk, dv of sum(dO * o)), blk=128
+    q, k, v = inputs.qkv((B, H, N, D), dtype=torch.bfloat16, device=device, seed=0)
+    do = inputs.qkv((B, H, N, D), dtype=torch.bfloat16, device=device, seed=1)[2]
+    grads = tuple(torch.empty_like(q) for _ in range(3))
+    la.la_timing_enable(64 * 8)
+    nb = 20
+    ms = timed(stream, lambda: la.prefill_backward(q, k, v, do, blk=BLK, out=grads), nb, 3, solo, device)
+    kt = kernel_times(la)
+    la.la_timing_enable(0)
+    bytes_bwd = B * H * N * 7 * D * 2      # q, k, v, dO read; dq, dk, dv written (bf16)
+    out["backward"] = {
+        "workload": f"prefill backward bf16 B={B} H={H} N={N} d={D} blk=128 (dq, dk, dv)",
+        "ms_per_step": round(ms / nb, 5),
+        "tokens_per_s": round(B * N / (ms / nb / 1e3), 1),
+        "hbm_frac": round(bytes_bwd / (ms / nb / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+        "algorithmic_bytes": bytes_bwd,
+        "kernels": {k_: [v_["launches"] // nb, round(v_["total_ms"] / max(v_["launches"], 1), 5)]
+                    for k_, v_ in kt.items()}}
+    del q, k, v, do, grads
     torch.cuda.empty_cache()
 
     # -- decode: 128 sequences x 64 heads, d=128; state from a 4096-token prefill

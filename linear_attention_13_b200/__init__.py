@@ -317,15 +317,23 @@ def prefill_varlen(q, k, v, cu_seqlens, blk: int = 128, want_state: bool = True,
     return o, st
 
 
-def prefill_backward(q, k, v, do, blk: int = 128, stream=None):
-    """Gradients (dq, dk, dv) of sum(do * prefill(q, k, v)[0]) for [B,H,N,d] tensors."""
+def prefill_backward(q, k, v, do, blk: int = 128, stream=None, out=None):
+    """Gradients (dq, dk, dv) of sum(do * prefill(q, k, v)[0]) for [B,H,N,d] tensors
+    (written into ``out`` = (dq, dk, dv) when given)."""
     torch = _torch()
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (do, "do")):
         _check(t, n)
     if not (k.shape == q.shape == v.shape == do.shape) or q.dim() != 4:
         raise ValueError("q, k, v, do must share one [B,H,N,d] shape")
     B, H, N, d = q.shape
-    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    if out is not None:
+        dq, dk, dv = out
+        for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+            _check(t, n)
+            if t.shape != q.shape or t.dtype != q.dtype:
+                raise ValueError(f"{n} must match q in shape and dtype")
+    else:
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
     status = la_prefill_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(),
                                  dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, blk,
                                  _dtype_code(q), _stream_ptr(stream))

@@ -356,6 +356,32 @@ int launch_fused(const tc::TileMaps& m, tc::Params p,
     return note_cuda(cudaGetLastError());
 }
 
+// The anti-causal form o_t = sum_{s >= t} (q_t . k_s) v_s, bf16, d = 128, 128-token
+// blocks: prefill_seq_kernel with one chunk per sequence, walking its blocks from
+// the last to the first (the state then holds suffix sums).  Sequences longer
+// than kReverseMaxN are not covered (LA_ERR_UNSUPPORTED): one CTA pair per
+// sequence would serialise too many blocks.
+constexpr int kReverseMaxN = 16384;
+
+int launch_prefill_reverse_bf16(const void* q, const void* k, const void* v, void* o, int BH, int N,
+                                cudaStream_t stream, int sms) {
+    if (N > kReverseMaxN) return LA_ERR_UNSUPPORTED;
+    tc::TileMaps m;
+    if (make_tile_maps(&m, q, k, v, o, N, BH)) return LA_ERR_CUDA;
+    tc::Params p = dense_params(BH, N, ((N + kTileRows - 1) / kTileRows) * kTileRows, o);
+    p.vparts = 2;
+    p.blk = 128;
+    p.n_items *= 2;
+    p.reverse = 1;
+    const int grid = std::min(p.n_items, sms);
+    {
+        TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
+        g_main_kernel = "prefill_seq_kernel";
+        tc::prefill_seq_kernel<<<grid, tc::sq::kThreads, tc::sq::kSmemBytes, stream>>>(m, p);
+    }
+    return note_cuda(cudaGetLastError());
+}
+
 int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, float* state_out,
                         int BH, int N, int blk, cudaStream_t stream, int sms, int chunk_tokens,
                         int flags, const float* state_in) {
@@ -853,7 +879,15 @@ int la_prefill_backward(const void* q, const void* k, const void* v, const void*
     st = prefill_impl(do_, v, k, dq, nullptr, nullptr, B, H, N, d, blk, dt, stream, 0, 0);
     if (st != LA_OK) return st;
     // dk_s = sum_{t >= s} (v_s . dO_t) q_t and dv_s = sum_{t >= s} (k_s . q_t) dO_t are
-    // causal sums of the token-reversed sequence, reversed back
+    // anti-causal forms: (q, k, v) = (v, dO, q) and (k, q, dO).  The split kernel
+    // runs them directly for 128-token blocks of bf16 sequences up to
+    // kReverseMaxN tokens; otherwise they are causal sums of the token-reversed
+    // sequence, reversed back.
+    if (dt == LA_BF16 && blk == 128 && N <= kReverseMaxN) {
+        st = launch_prefill_reverse_bf16(v, do_, q, dk, B * H, N, s, sms);
+        if (st == LA_OK) st = launch_prefill_reverse_bf16(k, q, do_, dv, B * H, N, s, sms);
+        return st;
+    }
     const long Z = (long)B * H;
     const size_t elems = (size_t)Z * N * d;
     const size_t esz = dt == LA_BF16 ? 2 : 4;

@@ -128,6 +128,9 @@ struct Params {
                                 // (non-empty sequences, longest first), or null
     const float* state_in;      // starting state of every sequence (layout of state_out),
                                 // or null (zero)
+    int reverse;                // prefill_seq_kernel, dense, one chunk per sequence:
+                                // the anti-causal form o_t = sum_{s >= t} (q_t.k_s) v_s,
+                                // blocks taken from the last to the first
 };
 
 // One work item: rows [t0, t1) of slice z, chunk c of its sequence, value
@@ -998,6 +1001,12 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
     const int n_items = num_items(p);
     const bool packed = p.mode == kModeVarlen;
     const int stride = gridDim.x;
+    // Row of the tile processed at step t (t = it.t0, it.t0 + 128, ...): the
+    // same in the causal form; from the last tile back in the anti-causal one
+    const bool rev = p.reverse != 0;
+    auto tile_row = [&](const Item& it, int t) {
+        return rev ? it.t0 + ((it.t1 - it.t0 - 1) / kTileRows) * kTileRows - (t - it.t0) : t;
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -1012,9 +1021,10 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         auto prefetch = [&](const Item& it, int t, int ahead) {
             const int tp = t + ahead * kTileRows;
             if (lane == 0 && tp < it.t1) {
-                ptx::tma_prefetch_4d(&maps.q, 0, tp, 0, it.z);
-                ptx::tma_prefetch_4d(&maps.k, 0, tp, 0, it.z);
-                ptx::tma_prefetch_3d(&maps.v_half, it.vp * sq::kNV, tp, it.z);
+                const int row = tile_row(it, tp);
+                ptx::tma_prefetch_4d(&maps.q, 0, row, 0, it.z);
+                ptx::tma_prefetch_4d(&maps.k, 0, row, 0, it.z);
+                ptx::tma_prefetch_3d(&maps.v_half, it.vp * sq::kNV, row, it.z);
             }
         };
         for (int item = blockIdx.x; ok && item < n_items; item += stride) {
@@ -1032,11 +1042,12 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 if (lane == 0) {
                     if (g >= 2) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
                     if (w) {
+                        const int row = tile_row(it, t);
                         ptx::mbar_arrive_expect_tx(fb, 2 * kTileBytes + kHalfBytes);
-                        ptx::tma_load_4d(stage, &maps.q, fb, 0, t, 0, it.z, pol_qk);
-                        ptx::tma_load_4d(stage + kTileBytes, &maps.k, fb, 0, t, 0, it.z, pol_qk);
+                        ptx::tma_load_4d(stage, &maps.q, fb, 0, row, 0, it.z, pol_qk);
+                        ptx::tma_load_4d(stage + kTileBytes, &maps.k, fb, 0, row, 0, it.z, pol_qk);
                         if (g >= 2) w = ptx::mbar_wait(bar(ctrl->v_empty[s]), ((g >> 1) + 1) & 1, abort_flag);
-                        if (w) ptx::tma_load_3d(stage + 2 * kTileBytes, &maps.v_half, fb, it.vp * sq::kNV, t, it.z, pol_v);
+                        if (w) ptx::tma_load_3d(stage + 2 * kTileBytes, &maps.v_half, fb, it.vp * sq::kNV, row, it.z, pol_v);
                     }
                 }
                 if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
@@ -1157,7 +1168,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
                     if (!ptx::mbar_wait(bar(ctrl->o_staged), g & 1, abort_flag)) { ok = false; break; }
                     if (!(packed && t + kTileRows > it.t1)) {
-                        ptx::tma_store_3d(&maps.o, sbase + sq::kOstOff, it.vp * sq::kNV, t, it.z);
+                        ptx::tma_store_3d(&maps.o, sbase + sq::kOstOff, it.vp * sq::kNV, tile_row(it, t), it.z);
                         ptx::bulk_commit_group();
                         ptx::bulk_wait_group_read0();
                     }
@@ -1213,7 +1224,9 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 {
                     const uint32_t scol = tl + sq::kColSP + b * 128 + k0;
                     uint32_t pk[32];
-                    if (k0 > sp * 32 + 31) {
+                    // keys [k0, k0 + 64) all masked for this warp's rows: above the
+                    // diagonal (causal) or below it (anti-causal)
+                    if (rev ? (k0 + 63 < sp * 32) : (k0 > sp * 32 + 31)) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) pk[j] = 0u;
                     } else {
@@ -1224,8 +1237,10 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const int key = k0 + 2 * j;
-                            const float a = (key <= r) ? __uint_as_float(v[2 * j]) : 0.0f;
-                            const float bb = (key + 1 <= r) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
+                            const bool keep_a = rev ? key >= r : key <= r;
+                            const bool keep_b = rev ? key + 1 >= r : key + 1 <= r;
+                            const float a = keep_a ? __uint_as_float(v[2 * j]) : 0.0f;
+                            const float bb = keep_b ? __uint_as_float(v[2 * j + 1]) : 0.0f;
                             pk[j] = ptx::pack_bf16x2(a, bb);
                         }
                     }

@@ -28,6 +28,17 @@ def test_bf16_backward(N, blk):
         assert per_head_rel_err(host64(got), ref) <= TOL_O_BF16
 
 
+def test_bf16_backward_many_tiles_ragged():
+    # 24 tiles per sequence with a ragged last one: dk and dv come from the
+    # anti-causal pass, which walks the tiles from the last (partial) one back
+    q, k, v = inputs.qkv((1, 4, 3000, 128), dtype=torch.bfloat16, device=DEV, seed=31)
+    do = inputs.qkv((1, 4, 3000, 128), dtype=torch.bfloat16, device=DEV, seed=32)[2]
+    dq, dk, dv = la.prefill_backward(q, k, v, do)
+    assert la.la_get_last_error() == la.LA_OK
+    for got, ref in zip((dq, dk, dv), _grads_ref(q, k, v, do)):
+        assert per_head_rel_err(host64(got), ref) <= TOL_O_BF16
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_fp32_backward(d):
     q, k, v = inputs.qkv((1, 3, 300, d), dtype=torch.float32, device=DEV, seed=d)
