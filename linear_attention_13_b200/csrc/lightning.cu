@@ -65,7 +65,9 @@ int device_setup(int* dev_out, int* sms_out) {
                                  tc::smem_bytes(64)) != cudaSuccess ||
             cudaFuncSetAttribute(tc::prefill_tc_kernel<128, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tc::smem_bytes(128)) != cudaSuccess ||
-            cudaFuncSetAttribute(tc::prefill_seq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(tc::prefill_seq_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::sq::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(tc::prefill_seq_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tc::sq::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(tc::chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tc::cs::kSmemBytes) != cudaSuccess ||
@@ -241,7 +243,7 @@ void launch_main(const tc::TileMaps& m, const tc::Params& p, int grid, cudaStrea
         tc::prefill_tc_kernel<128, 64><<<grid, tc::kThreads, tc::smem_bytes(128), stream>>>(m, p);
     } else if (p.vparts == 2 && !p.fused) {
         g_main_kernel = "prefill_seq_kernel";
-        tc::prefill_seq_kernel<<<grid, tc::sq::kThreads, tc::sq::kSmemBytes, stream>>>(m, p);
+        tc::prefill_seq_kernel<false><<<grid, tc::sq::kThreads, tc::sq::kSmemBytes, stream>>>(m, p);
     } else if (p.vparts == 2) {
         g_main_kernel = "prefill_tc_kernel<64>";
         tc::prefill_tc_kernel<64><<<grid, tc::kThreads, tc::smem_bytes(64), stream>>>(m, p);
@@ -372,12 +374,11 @@ int launch_prefill_reverse_bf16(const void* q, const void* k, const void* v, voi
     p.vparts = 2;
     p.blk = 128;
     p.n_items *= 2;
-    p.reverse = 1;
     const int grid = std::min(p.n_items, sms);
     {
         TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
-        g_main_kernel = "prefill_seq_kernel";
-        tc::prefill_seq_kernel<<<grid, tc::sq::kThreads, tc::sq::kSmemBytes, stream>>>(m, p);
+        g_main_kernel = "prefill_seq_kernel<anti-causal>";
+        tc::prefill_seq_kernel<true><<<grid, tc::sq::kThreads, tc::sq::kSmemBytes, stream>>>(m, p);
     }
     return note_cuda(cudaGetLastError());
 }

@@ -128,9 +128,6 @@ struct Params {
                                 // (non-empty sequences, longest first), or null
     const float* state_in;      // starting state of every sequence (layout of state_out),
                                 // or null (zero)
-    int reverse;                // prefill_seq_kernel, dense, one chunk per sequence:
-                                // the anti-causal form o_t = sum_{s >= t} (q_t.k_s) v_s,
-                                // blocks taken from the last to the first
 };
 
 // One work item: rows [t0, t1) of slice z, chunk c of its sequence, value
@@ -948,6 +945,11 @@ struct Ctrl {
 };
 }  // namespace sq
 
+// kRev: the anti-causal form o_t = sum_{s >= t} (q_t . k_s) v_s (dense, one
+// chunk per sequence): tiles are taken from the last to the first and the
+// intra-block mask keeps keys at or after the row.  A template parameter, so
+// that the causal instantiation carries none of it.
+template <bool kRev>
 __global__ void __launch_bounds__(sq::kThreads, 1)
 prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                    const Params p) {
@@ -1003,9 +1005,9 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
     const int stride = gridDim.x;
     // Row of the tile processed at step t (t = it.t0, it.t0 + 128, ...): the
     // same in the causal form; from the last tile back in the anti-causal one
-    const bool rev = p.reverse != 0;
     auto tile_row = [&](const Item& it, int t) {
-        return rev ? it.t0 + ((it.t1 - it.t0 - 1) / kTileRows) * kTileRows - (t - it.t0) : t;
+        if constexpr (kRev) return it.t0 + ((it.t1 - it.t0 - 1) / kTileRows) * kTileRows - (t - it.t0);
+        else return t;
     };
 
     if (warp == 0) {
@@ -1226,7 +1228,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     uint32_t pk[32];
                     // keys [k0, k0 + 64) all masked for this warp's rows: above the
                     // diagonal (causal) or below it (anti-causal)
-                    if (rev ? (k0 + 63 < sp * 32) : (k0 > sp * 32 + 31)) {
+                    if (kRev ? (k0 + 63 < sp * 32) : (k0 > sp * 32 + 31)) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) pk[j] = 0u;
                     } else {
@@ -1237,8 +1239,8 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const int key = k0 + 2 * j;
-                            const bool keep_a = rev ? key >= r : key <= r;
-                            const bool keep_b = rev ? key + 1 >= r : key + 1 <= r;
+                            const bool keep_a = kRev ? key >= r : key <= r;
+                            const bool keep_b = kRev ? key + 1 >= r : key + 1 <= r;
                             const float a = keep_a ? __uint_as_float(v[2 * j]) : 0.0f;
                             const float bb = keep_b ? __uint_as_float(v[2 * j + 1]) : 0.0f;
                             pk[j] = ptx::pack_bf16x2(a, bb);
