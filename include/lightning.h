@@ -154,11 +154,15 @@ int la_prefill_varlen_from_state(const void* q, const void* k, const void* v, vo
  * la_prefill_backward -- gradients of L = sum_t dO_t . o_t for o = la_prefill
  * (q, k, v) (zero starting state), the training direction:
  *     dq_t = sum_{s <= t} (dO_t . v_s) k_s     (the causal form of (dO, v, k))
- *     dk_s = sum_{t >= s} (dO_t . v_s) q_t     (anti-causal: the causal form
- *     dv_s = sum_{t >= s} (q_t . k_s) dO_t      of the token-reversed sequence)
+ *     dk_s = sum_{t >= s} (dO_t . v_s) q_t     (the anti-causal form of (v, dO, q))
+ *     dv_s = sum_{t >= s} (q_t . k_s) dO_t     (the anti-causal form of (k, q, dO))
  *   q, k, v, do_ : [B, H, N, d] of dt (read only); dq, dk, dv : [B, H, N, d]
- *   of dt (written).  Same dtype, d, blk rules as la_prefill.  Scratch: five
- *   tensors of the input size from the stream-ordered allocator.  The pages
+ *   of dt (written).  Same dtype, d, blk rules as la_prefill.  For bf16 with
+ *   blk = 128 and N <= 16384 the anti-causal forms run directly (the tiles of
+ *   each sequence taken from the last) and no scratch is used; otherwise they
+ *   are causal forms of the token-reversed sequence, reversed back, with five
+ *   tensors of the input size of scratch from the stream-ordered allocator
+ *   (LA_ERR_ALLOC if that fails).  The pages
  *   give no backward pass (training is the context of section 2 of the
  *   futurefh page); this is the derivative of the forward definition.
  */
