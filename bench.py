@@ -56,13 +56,15 @@ PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "prefill_seq_kernel_b4h16n8192.
 
 
 def kernel_source_sha256() -> str:
-    """Hash of the CUDA sources (csrc/*.cu, *.cuh): identifies the kernel
-    version an ncu capture was taken of."""
+    """Hash of the kernel sources (csrc/*.cuh, which hold every __global__ and
+    __device__ function): identifies the kernel version an ncu capture was
+    taken of.  lightning.cu (host-side validation, dispatch and launches) is
+    not part of it."""
     import hashlib
     csrc = os.path.join(ROOT, "linear_attention_13_b200", "csrc")
     h = hashlib.sha256()
     for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
+        if name.endswith(".cuh"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()

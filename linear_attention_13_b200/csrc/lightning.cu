@@ -4,6 +4,7 @@
 // kernel so that the device status word needs no separate device link.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -168,6 +169,16 @@ struct TimedLaunch {
     cudaStream_t s;
     TimedLaunch(int id, cudaStream_t st) : slot(timing_begin(id, st)), s(st) {}
     ~TimedLaunch() { timing_end(slot, s); }
+};
+
+// NVTX range named after a C entry point, around the whole host call (checks,
+// descriptor set-up, launches), so that profiler timelines group the kernels
+// by call.  A pointer test when no profiler is attached.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -772,12 +783,14 @@ int prefill_impl(const void* q, const void* k, const void* v, void* o, const flo
 
 int la_prefill(const void* q, const void* k, const void* v, void* o, float* state_out, int B, int H,
                int N, int d, int blk, la_dtype dt, void* stream) {
+    NvtxRange nvtx_range("la_prefill");
     return la_prefill_ex(q, k, v, o, state_out, B, H, N, d, blk, dt, stream, 0, 0);
 }
 
 int la_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* state_out,
                       const int32_t* cu_seqlens, int num_seqs, int total_tokens, int H, int d,
                       int blk, la_dtype dt, void* stream) {
+    NvtxRange nvtx_range("la_prefill_varlen");
     return la_prefill_varlen_ex(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens, H, d,
                                 blk, dt, stream, 0, 0);
 }
@@ -840,18 +853,21 @@ int varlen_impl(const void* q, const void* k, const void* v, void* o, const floa
 int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* state_out, int B,
                   int H, int N, int d, int blk, la_dtype dt, void* stream, int chunk_tokens,
                   int flags) {
+    NvtxRange nvtx_range("la_prefill_ex");
     return prefill_impl(q, k, v, o, nullptr, state_out, B, H, N, d, blk, dt, stream, chunk_tokens, flags);
 }
 
 int la_prefill_from_state(const void* q, const void* k, const void* v, void* o, const float* state_in,
                           float* state_out, int B, int H, int N, int d, int blk, la_dtype dt,
                           void* stream, int chunk_tokens, int flags) {
+    NvtxRange nvtx_range("la_prefill_from_state");
     return prefill_impl(q, k, v, o, state_in, state_out, B, H, N, d, blk, dt, stream, chunk_tokens, flags);
 }
 
 int la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o, float* state_out,
                          const int32_t* cu_seqlens, int num_seqs, int total_tokens, int H, int d,
                          int blk, la_dtype dt, void* stream, int chunk_tokens, int flags) {
+    NvtxRange nvtx_range("la_prefill_varlen_ex");
     return varlen_impl(q, k, v, o, nullptr, state_out, cu_seqlens, num_seqs, total_tokens, H, d, blk,
                        dt, stream, chunk_tokens, flags);
 }
@@ -860,6 +876,7 @@ int la_prefill_varlen_from_state(const void* q, const void* k, const void* v, vo
                                  const float* state_in, float* state_out, const int32_t* cu_seqlens,
                                  int num_seqs, int total_tokens, int H, int d, int blk, la_dtype dt,
                                  void* stream, int chunk_tokens, int flags) {
+    NvtxRange nvtx_range("la_prefill_varlen_from_state");
     return varlen_impl(q, k, v, o, state_in, state_out, cu_seqlens, num_seqs, total_tokens, H, d, blk,
                        dt, stream, chunk_tokens, flags);
 }
@@ -867,6 +884,7 @@ int la_prefill_varlen_from_state(const void* q, const void* k, const void* v, vo
 int la_prefill_backward(const void* q, const void* k, const void* v, const void* do_, void* dq,
                         void* dk, void* dv, int B, int H, int N, int d, int blk, la_dtype dt,
                         void* stream) {
+    NvtxRange nvtx_range("la_prefill_backward");
     if (B < 1 || H < 1 || N < 1 || !do_ || !dq || !dk || !dv) return LA_ERR_INVALID_ARG;
     if (!aligned16(do_) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return LA_ERR_INVALID_ARG;
     int st = validate_common(q, k, v, dq, d, blk, dt);
@@ -927,6 +945,7 @@ int la_prefill_backward(const void* q, const void* k, const void* v, const void*
 
 int la_state_increment(const void* k, const void* v, float* delta_out, int B, int H, int N, int d,
                        la_dtype dt, void* stream) {
+    NvtxRange nvtx_range("la_state_increment");
     if (B < 1 || H < 1 || N < 1 || !k || !v || !delta_out) return LA_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(v) || !aligned16(delta_out)) return LA_ERR_INVALID_ARG;
     if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
@@ -951,6 +970,7 @@ int la_state_increment(const void* k, const void* v, float* delta_out, int B, in
 
 int la_state_prefix(const float* states, int R, int rank, float* prefix_out, int B, int H, int d,
                     void* stream) {
+    NvtxRange nvtx_range("la_state_prefix");
     if (!states || !prefix_out || R < 1 || rank < 0 || rank > R || B < 1 || H < 1) return LA_ERR_INVALID_ARG;
     if (!aligned16(states) || !aligned16(prefix_out)) return LA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
@@ -970,12 +990,14 @@ int la_state_prefix(const float* states, int R, int rank, float* prefix_out, int
 
 int la_decode_step(const void* q, const void* k, const void* v, float* state, void* o, int B, int H,
                    int d, la_dtype dt, void* stream) {
+    NvtxRange nvtx_range("la_decode_step");
     return la_decode_step_slots(q, k, v, state, nullptr, B, o, B, H, d, dt, stream);
 }
 
 int la_decode_step_slots(const void* q, const void* k, const void* v, float* state_pool,
                          const int32_t* slots, int num_slots, void* o, int B, int H, int d,
                          la_dtype dt, void* stream) {
+    NvtxRange nvtx_range("la_decode_step_slots");
     int st = decode_args_ok(q, k, v, o, B, H, d, dt);
     if (st != LA_OK) return st;
     if (!state_pool || !aligned16(state_pool)) return LA_ERR_INVALID_ARG;
@@ -994,6 +1016,7 @@ int la_decode_step_slots(const void* q, const void* k, const void* v, float* sta
 int la_decode_step_q8(const void* q, const void* k, const void* v, int8_t* codes, float* scales,
                       const int32_t* slots, int num_slots, void* o, int B, int H, int d, la_dtype dt,
                       void* stream) {
+    NvtxRange nvtx_range("la_decode_step_q8");
     int st = decode_args_ok(q, k, v, o, B, H, d, dt);
     if (st != LA_OK) return st;
     if (!codes || !scales || !aligned16(codes) || !aligned16(scales)) return LA_ERR_INVALID_ARG;
@@ -1011,6 +1034,7 @@ int la_decode_step_q8(const void* q, const void* k, const void* v, int8_t* codes
 
 int la_state_quantize_q8(const float* state, int8_t* codes, float* scales, long long n_heads, int d,
                          void* stream) {
+    NvtxRange nvtx_range("la_state_quantize_q8");
     if (n_heads < 1 || !state || !codes || !scales) return LA_ERR_INVALID_ARG;
     if (!aligned16(state) || !aligned16(codes) || !aligned16(scales)) return LA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
@@ -1031,6 +1055,7 @@ int la_state_quantize_q8(const float* state, int8_t* codes, float* scales, long 
 
 int la_state_dequantize_q8(const int8_t* codes, const float* scales, float* state, long long n_heads,
                            int d, void* stream) {
+    NvtxRange nvtx_range("la_state_dequantize_q8");
     if (n_heads < 1 || !state || !codes || !scales) return LA_ERR_INVALID_ARG;
     if (!aligned16(state) || !aligned16(codes) || !aligned16(scales)) return LA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
@@ -1092,6 +1117,7 @@ int la_device_sm_count(void) {
 
 int la_prefill_noalloc(const void* q, const void* k, const void* v, void* o, float* state_out,
                        int B, int H, int N, int d, int blk, la_dtype dt, void* stream) {
+    NvtxRange nvtx_range("la_prefill_noalloc");
     if (B < 1 || H < 1 || N < 1) return LA_ERR_INVALID_ARG;
     int st = validate_common(q, k, v, o, d, blk, dt);
     if (st != LA_OK) return st;
