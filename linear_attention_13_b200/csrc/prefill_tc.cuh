@@ -922,7 +922,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kStoreWarp = 2 + kEpiWarps;   // TMA stores of the staged O tiles
 constexpr int kMmaBWarp = 3 + kEpiWarps;    // second MMA issuer
 constexpr int kThreads = 32 * (4 + kEpiWarps);
-constexpr int kL2Ahead = 3;                 // tiles prefetched into L2 ahead of the load
+constexpr int kL2Ahead = 2;                 // tiles prefetched into L2 ahead of the load
 
 struct Ctrl {
     uint64_t full[kStages];
