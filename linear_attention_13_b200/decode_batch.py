@@ -118,6 +118,10 @@ class PaddedDecoder:
                  for name in ("q", "k", "v", "o")}
             b["slots"] = torch.full((level,), -1, dtype=torch.int32, device=self.device)
             b["slots_host"] = torch.full((level,), -1, dtype=torch.int32).pin_memory()
+            # the asynchronous upload of slots_host must have run before the host
+            # overwrites it for the next step of this level
+            b["uploaded"] = torch.cuda.Event()
+            b["pending"] = False
             self._bufs[level] = b
         return b
 
@@ -159,8 +163,12 @@ class PaddedDecoder:
         b["q"][:n].copy_(q)
         b["k"][:n].copy_(k)
         b["v"][:n].copy_(v)
+        if b["pending"]:
+            b["uploaded"].synchronize()
         b["slots_host"].copy_(self.torch.tensor(padded, dtype=self.torch.int32))
         b["slots"].copy_(b["slots_host"], non_blocking=True)
+        b["uploaded"].record()
+        b["pending"] = True
         if self.use_graphs:
             self._graph(level, b).replay()
         else:
