@@ -1,7 +1,10 @@
 /*
  * lightning.h -- C ABI of liblightning.so: causal linear attention
- * ("Lightning Attention") prefill, packed variable-length prefill and decode
- * on NVIDIA B200 (sm_100a).
+ * ("Lightning Attention") on NVIDIA B200 (sm_100a).  Entry points: prefill
+ * (dense and packed variable-length, optionally continued from a given
+ * state), its backward, the state increment and prefix used for sequence
+ * parallelism, and decode (fp32 state, a slot pool with padding rows, and an
+ * 8-bit state with its conversions); status and timing queries.
  *
  * The operation (no softmax, no scale, no normaliser, diagonal included):
  *
