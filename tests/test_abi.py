@@ -47,7 +47,26 @@ def test_library_is_built_for_sm100a():
 def test_status_strings(lib):
     assert la.status_string(la.LA_OK) == "LA_OK"
     assert la.status_string(la.LA_ERR_BAD_SEQLENS) == "LA_ERR_BAD_SEQLENS"
+    assert la.status_string(la.LA_ERR_BAD_SLOT) == "LA_ERR_BAD_SLOT"
     assert la.status_string(12345) == "LA_UNKNOWN_STATUS"
+
+
+@pytest.mark.parametrize("compiler,std", [("gcc", "-std=c99"), ("g++", "-std=c++11")])
+def test_header_compiles_as_plain_c_and_cpp(tmp_path, compiler, std):
+    # the boundary is a C ABI: the header alone must compile in C and C++
+    src = tmp_path / ("use.c" if compiler == "gcc" else "use.cpp")
+    src.write_text('#include "lightning.h"\n'
+                   "int main(void) {\n"
+                   "    la_dtype dt = LA_BF16;\n"
+                   "    int (*f)(const void*, const void*, const void*, void*, float*, int, int, int,\n"
+                   "             int, int, la_dtype, void*) = la_prefill;\n"
+                   "    return (f != 0 && dt == LA_BF16 && LA_ERR_BAD_SLOT < 0) ? 0 : 1;\n"
+                   "}\n")
+    import subprocess
+    r = subprocess.run([compiler, std, "-Wall", "-Werror", "-pedantic", "-fsyntax-only",
+                        "-I", os.path.join(ROOT, "include"), str(src)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
 
 
 FAKE = 0x100000  # 16-byte aligned, never dereferenced: validation fails first
@@ -82,6 +101,45 @@ def test_varlen_and_decode_argument_validation(lib):
                              None) == la.LA_ERR_UNSUPPORTED
     assert la.la_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 128, la.LA_BF16,
                              None) == la.LA_ERR_INVALID_ARG
+
+
+def test_slot_decode_and_8bit_state_argument_validation(lib):
+    I, U = la.LA_ERR_INVALID_ARG, la.LA_ERR_UNSUPPORTED
+    # slot pool: misaligned slot array, empty pool, no slots with a pool smaller than B
+    assert la.la_decode_step_slots(FAKE, FAKE, FAKE, FAKE, FAKE + 2, 4, FAKE, 2, 1, 128,
+                                   la.LA_BF16, None) == I
+    assert la.la_decode_step_slots(FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, 2, 1, 128,
+                                   la.LA_BF16, None) == I
+    assert la.la_decode_step_slots(FAKE, FAKE, FAKE, FAKE, None, 1, FAKE, 2, 1, 128,
+                                   la.LA_BF16, None) == I
+    assert la.la_decode_step_slots(FAKE, FAKE, FAKE, None, FAKE, 4, FAKE, 2, 1, 128,
+                                   la.LA_BF16, None) == I
+    assert la.la_decode_step_slots(FAKE, FAKE, FAKE, FAKE, FAKE, 4, FAKE, 2, 1, 96,
+                                   la.LA_BF16, None) == U
+    # 8-bit state: missing or misaligned codes / scales
+    assert la.la_decode_step_q8(FAKE, FAKE, FAKE, None, FAKE, None, 2, FAKE, 2, 1, 128,
+                                la.LA_BF16, None) == I
+    assert la.la_decode_step_q8(FAKE, FAKE, FAKE, FAKE, FAKE + 4, None, 2, FAKE, 2, 1, 128,
+                                la.LA_BF16, None) == I
+    assert la.la_decode_step_q8(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, FAKE, 2, 1, 128,
+                                la.LA_BF16, None) == I
+    assert la.la_state_quantize_q8(FAKE, FAKE, FAKE, 0, 128, None) == I
+    assert la.la_state_quantize_q8(FAKE, FAKE, FAKE, 1, 96, None) == U
+    assert la.la_state_dequantize_q8(FAKE, None, FAKE, 1, 128, None) == I
+    assert la.la_state_dequantize_q8(FAKE, FAKE, FAKE, 1, 32, None) == U
+
+
+def test_backward_and_sequence_parallel_argument_validation(lib):
+    I = la.LA_ERR_INVALID_ARG
+    assert la.la_prefill_backward(FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, 1, 1, 16, 128, 128,
+                                  la.LA_BF16, None) == I
+    assert la.la_prefill_backward(FAKE, FAKE, FAKE, FAKE, FAKE + 2, FAKE, FAKE, 1, 1, 16, 128,
+                                  128, la.LA_BF16, None) == I
+    assert la.la_prefill_backward(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 128, 128,
+                                  la.LA_BF16, None) == I
+    assert la.la_state_increment(None, FAKE, FAKE, 1, 1, 16, 128, la.LA_BF16, None) == I
+    assert la.la_state_increment(FAKE, FAKE, FAKE, 1, 1, 16, 64, la.LA_BF16,
+                                 None) == la.LA_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("flags", [
