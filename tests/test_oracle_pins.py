@@ -227,6 +227,29 @@ def pin_backward_d1_sums(orc):
     assert np.allclose(dv[0, :, 0], kf * suffix_gq, atol=1e-12)
 
 
+def pin_zero_keys_and_unmasked_identity(orc):
+    """k = 0 gives o = 0 and a zero state in every form; and the associativity
+    the block form rests on, (Q K^T) V = Q (K^T V), holds for plain numpy
+    products, while the causal oracle differs from the unmasked product (the
+    mask matters)."""
+    r = _rng(24)
+    q, v = r.standard_normal((2, 9, 5)), r.standard_normal((2, 9, 5))
+    k = np.zeros((2, 9, 5))
+    assert not np.any(orc.prefill_quadratic(q, k, v))
+    o, s = orc.prefill_recurrent(q, k, v)
+    assert not np.any(o) and not np.any(s)
+    for blk in (1, 4):
+        o, s = orc.prefill_blockwise(q, k, v, blk)
+        assert not np.any(o) and not np.any(s)
+    k = r.standard_normal((2, 9, 5))
+    left = np.einsum("bnd,bmd,bme->bne", q, k, v)
+    right = np.einsum("bnd,bde->bne", q, np.einsum("bmd,bme->bde", k, v))
+    assert _rel(left, right) < 1e-12
+    causal = orc.prefill_quadratic(q, k, v)
+    assert _rel(causal[:, -1], left[:, -1]) < 1e-12      # the last row sees every key
+    assert _rel(causal[:, 0], left[:, 0]) > 1e-3          # the first row sees only itself
+
+
 def pin_q8_golden(orc):
     g = json.load(open(os.path.join(GOLDEN, "q8_state_worked_example.json")))
     for row in g["quantize"]:
@@ -326,7 +349,7 @@ def pin_decode_slots(orc):
 
 PINS = [pin_golden, pin_forms_agree, pin_state_is_KtV, pin_last_row, pin_d1_prefix_sum, pin_N1,
         pin_ternary_bruteforce, pin_state_in, pin_decode, pin_varlen, pin_backward_finite_differences,
-        pin_backward_d1_sums, pin_q8_golden, pin_q8_integer_trajectory, pin_q8_within_rounding_bound,
+        pin_backward_d1_sums, pin_zero_keys_and_unmasked_identity, pin_q8_golden, pin_q8_integer_trajectory, pin_q8_within_rounding_bound,
         pin_decode_slots]
 
 
