@@ -7,6 +7,7 @@ import socket
 import sys
 
 import numpy as np
+import pytest
 import torch
 import torch.multiprocessing as mp
 
@@ -49,7 +50,7 @@ def _oracle_compute():
     return ShardCompute(increment, prefix, prefill)
 
 
-def _rank_main(rank, port, out_q):
+def _rank_main(rank, port, out_q, cuts):
     os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(R), "MASTER_ADDR": "127.0.0.1",
                        "MASTER_PORT": str(port)})
     import torch.distributed as dist
@@ -57,7 +58,7 @@ def _rank_main(rank, port, out_q):
 
     dist.init_process_group("gloo", rank=rank, world_size=R)
     q, k, v = _global_inputs()
-    lo, hi = rank * N // R, (rank + 1) * N // R
+    lo, hi = cuts[rank], cuts[rank + 1]
     shard = [torch.from_numpy(np.ascontiguousarray(x[:, :, lo:hi])) for x in (q, k, v)]
     o, s = prefill_sequence_parallel(*shard, compute=_oracle_compute())
     dist.barrier()
@@ -65,13 +66,15 @@ def _rank_main(rank, port, out_q):
     out_q.put((rank, o.numpy(), s.numpy()))
 
 
-def test_three_rank_sequence_split_reassembles_the_sequence():
+@pytest.mark.parametrize("cuts", [[0, 32, 64, 96], [0, 7, 61, 96]], ids=["even", "uneven"])
+def test_three_rank_sequence_split_reassembles_the_sequence(cuts):
+    # shards of any lengths: only the d x d states cross ranks
     import oracle
     oracle.build()
     port = _free_port()
     ctx = mp.get_context("spawn")
     q_ = ctx.Queue()
-    procs = [ctx.Process(target=_rank_main, args=(r, port, q_)) for r in range(R)]
+    procs = [ctx.Process(target=_rank_main, args=(r, port, q_, cuts)) for r in range(R)]
     for p in procs:
         p.start()
     res = sorted([q_.get(timeout=120) for _ in range(R)], key=lambda x: x[0])
@@ -85,6 +88,6 @@ def test_three_rank_sequence_split_reassembles_the_sequence():
     np.testing.assert_allclose(res[-1][2], s_ref, rtol=0, atol=1e-10)
     # rank r's state is the state after its last token
     for rank, _, s in res:
-        hi = (rank + 1) * N // R
+        hi = cuts[rank + 1]
         _, s_hi = oracle.prefill_recurrent(q[:, :, :hi], k[:, :, :hi], v[:, :, :hi])
         np.testing.assert_allclose(s, s_hi, rtol=0, atol=1e-10)
