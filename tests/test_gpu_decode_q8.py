@@ -101,6 +101,35 @@ def test_q8_integer_state_exact():
     assert np.array_equal(_np(c).astype(np.float64), want)
 
 
+@pytest.mark.parametrize("dt", DTS)
+def test_q8_rows_becoming_zero(dt):
+    # a row the step cancels exactly and a row below 2^-100 become zero rows
+    # (codes 0, scale 0), every other row as the oracle says
+    d = 128
+    g = torch.Generator().manual_seed(17)
+    S = torch.randn((1, 2, d, d), generator=g) * 2.0
+    c, a = oracle.state_quantize_q8(S.numpy())
+    c[0, 0, 0] = 0
+    c[0, 0, 0, :4] = [1, 2, 0, -3]
+    a[0, 0, 0] = 1.0
+    c[0, 1, 5] = 0
+    c[0, 1, 5, 0] = 127
+    a[0, 1, 5] = np.float32(2.0 ** -108) / np.float32(127)
+    q, k, v = inputs.decode_step_inputs(1, 2, d, 3, dtype=dt, device="cpu")
+    k[0, 0] = 0
+    k[0, 0, 0] = -1.0
+    v[0, 0] = 0
+    v[0, 0, :4] = torch.tensor([1.0, 2.0, 0.0, -3.0])
+    k[0, 1, 5] = 0
+    cd, ad = torch.from_numpy(c).to(DEV), torch.from_numpy(a).to(DEV)
+    o = la.decode_step_q8(q.to(DEV), k.to(DEV), v.to(DEV), cd, ad)
+    assert la.la_get_last_error() == la.LA_OK
+    o_ref, c_ref, a_ref = oracle.decode_step_q8(host64(q), host64(k), host64(v), c, a)
+    assert a_ref[0, 0, 0] == 0 and a_ref[0, 1, 5] == 0 and not np.any(c_ref[0, 0, 0])
+    assert np.array_equal(_np(cd), c_ref) and np.array_equal(_np(ad), a_ref)
+    assert per_head_rel_err(host64(o), o_ref, head_dims=1) <= _tol(dt)
+
+
 def _slot_batch(num_slots, B, n_pad, seed):
     rng = np.random.default_rng(seed)
     live = rng.choice(num_slots, size=B - n_pad, replace=False).tolist()

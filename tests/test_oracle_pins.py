@@ -267,6 +267,22 @@ def pin_q8_golden(orc):
     assert a[0].tolist() == [float(np.float32(x)) for x in st["scales_out"]]
 
 
+def pin_q8_rows_becoming_zero(orc):
+    """Worked by hand: a row that a step cancels exactly, and a row whose values
+    fall below 2^-100, are both stored as zero rows: codes 0 and scale 0 (not
+    the scale they had before)."""
+    a1 = np.float32(2.0 ** -108) / np.float32(127)           # row 1 dequantises to ~2^-108
+    codes = np.array([[[1, 2, 0, -3], [127, 0, 0, 0], [0, 0, 0, 0], [0, 0, 0, 0]]], np.int8)
+    scales = np.array([[1.0, a1, 0.0, 0.0]], np.float32)
+    q = np.array([[1.0, 1.0, 1.0, 1.0]], np.float32)
+    k = np.array([[-1.0, 0.0, 0.0, 0.0]], np.float32)        # row 0: s = c - v = 0
+    v = np.array([[1.0, 2.0, 0.0, -3.0]], np.float32)
+    o, c2, a2 = orc.decode_step_q8(q, k, v, codes, scales)
+    assert not np.any(c2) and not np.any(a2)
+    tiny = float(np.float32(127) * a1)                       # row 1's first value, kept in o
+    assert o[0].tolist() == [tiny, 0.0, 0.0, 0.0]
+
+
 def pin_q8_integer_trajectory(orc):
     """Rows whose largest magnitude stays exactly 127 have scale 1, so codes are
     the state itself: one-hot keys and small integer values keep every step
@@ -349,7 +365,7 @@ def pin_decode_slots(orc):
 
 PINS = [pin_golden, pin_forms_agree, pin_state_is_KtV, pin_last_row, pin_d1_prefix_sum, pin_N1,
         pin_ternary_bruteforce, pin_state_in, pin_decode, pin_varlen, pin_backward_finite_differences,
-        pin_backward_d1_sums, pin_zero_keys_and_unmasked_identity, pin_q8_golden, pin_q8_integer_trajectory, pin_q8_within_rounding_bound,
+        pin_backward_d1_sums, pin_zero_keys_and_unmasked_identity, pin_q8_golden, pin_q8_rows_becoming_zero, pin_q8_integer_trajectory, pin_q8_within_rounding_bound,
         pin_decode_slots]
 
 
@@ -388,6 +404,10 @@ MUTANTS = {
     "q8_no_small_row_cut": ("if (m < 0x1p-100f) {", "if (m <= 0.0f) {"),
     "q8_transposed_update": ("fmaf(kb[i], vb[j], deq)", "fmaf(kb[j], vb[i], deq)"),
     "q8_column_scale": ("(float)cb[i * d + j] * ab[i]", "(float)cb[i * d + j] * ab[j]"),
+    "q8_dequantize_column_scale": ("S[r * d + j] = (float)codes[r * d + j] * scales[r];",
+                                   "S[r * d + j] = (float)codes[r * d + j] * scales[j % rows];"),
+    "q8_zero_row_keeps_old_scale": ("        *a = 0.0f;\n        for (long j = 0; j < d; ++j) c[j] = 0;",
+                                    "        for (long j = 0; j < d; ++j) c[j] = 0;"),
     "q8_reads_before_update": ("acc += (double)qb[i] * (double)s[i * d + j];",
                                "acc += (double)qb[i] * (double)cb[i * d + j] * ab[i];"),
 }
