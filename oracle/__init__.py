@@ -100,6 +100,16 @@ def _shape_bhnd(q):
     raise ValueError("q must be [B,H,N,d] or [BH,N,d]")
 
 
+def _slot_rows(slots, num_slots):
+    slots = np.asarray(slots, dtype=np.int64).reshape(-1)
+    if np.any(slots >= num_slots):
+        raise ValueError("slot id out of range")
+    live = slots[slots >= 0]
+    if len(np.unique(live)) != len(live):
+        raise ValueError("a slot may appear once per batch")
+    return slots
+
+
 class Oracle:
     """ctypes view of one compiled copy of oracle.c (the default one, or a
     deliberately altered copy built by the pin-strength tests)."""
@@ -200,10 +210,41 @@ class Oracle:
         self.lib.oracle_state_dequantize_q8(_cptr(c), _fptr(a), _fptr(S), c.size // d, d)
         return S
 
-    def decode_step_q8(self, q, k, v, codes, scales):
+    def decode_step_slots(self, q, k, v, pool, slots):
+        """Decode step for a batch whose row b uses state pool[slots[b]].
+
+        q, k, v: [B, H, d]; pool: [num_slots, H, d, d]; a negative slot marks a
+        padding row, whose output is zero and which touches no state.  Returns
+        (o [B, H, d], pool') in fp64; the input pool is untouched.  Each live row
+        is ``decode_step`` applied to its own slot's state."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        pool = _f64(pool).copy()
+        slots = _slot_rows(slots, pool.shape[0])
+        o = np.zeros(q.shape, dtype=np.float64)
+        for b, slot in enumerate(slots):
+            if slot < 0:
+                continue
+            o[b], pool[slot] = self.decode_step(q[b], k[b], v[b], pool[slot])
+        return o, pool
+
+    def decode_step_q8(self, q, k, v, codes, scales, slots=None):
         """One step on the 8-bit state; returns (o fp64, codes', scales'), inputs untouched.
 
-        q, k, v must hold values exact in fp32 (fp32 or bf16 inputs)."""
+        q, k, v must hold values exact in fp32 (fp32 or bf16 inputs).  With
+        ``slots`` (one per row of q, negative = padding) row b updates state
+        codes[slots[b]], scales[slots[b]] of a [num_slots, H, d, d] pool."""
+        if slots is not None:
+            q, k, v = np.asarray(q), np.asarray(k), np.asarray(v)
+            codes = np.array(codes, dtype=np.int8, copy=True)
+            scales = np.array(scales, dtype=np.float32, copy=True)
+            slots = _slot_rows(slots, codes.shape[0])
+            o = np.zeros(q.shape, dtype=np.float64)
+            for b, slot in enumerate(slots):
+                if slot < 0:
+                    continue
+                o[b], codes[slot], scales[slot] = self.decode_step_q8(q[b], k[b], v[b], codes[slot],
+                                                                      scales[slot])
+            return o, codes, scales
         qf, kf, vf = _f32_exact(q), _f32_exact(k), _f32_exact(v)
         c = np.array(codes, dtype=np.int8, copy=True, order="C")
         a = np.array(scales, dtype=np.float32, copy=True, order="C")
@@ -286,50 +327,9 @@ def state_dequantize_q8(codes, scales):
     return _get().state_dequantize_q8(codes, scales)
 
 
-def _slot_rows(slots, num_slots):
-    slots = np.asarray(slots, dtype=np.int64).reshape(-1)
-    if np.any(slots >= num_slots):
-        raise ValueError("slot id out of range")
-    live = slots[slots >= 0]
-    if len(np.unique(live)) != len(live):
-        raise ValueError("a slot may appear once per batch")
-    return slots
-
-
 def decode_step_slots(q, k, v, pool, slots):
-    """Decode step for a batch whose row b uses state pool[slots[b]].
-
-    q, k, v: [B, H, d]; pool: [num_slots, H, d, d]; a negative slot marks a
-    padding row, whose output is zero and which touches no state.  Returns
-    (o [B, H, d], pool') in fp64; the input pool is untouched.  Each live row is
-    ``decode_step`` applied to its own slot's state."""
-    q, k, v = _f64(q), _f64(k), _f64(v)
-    pool = _f64(pool).copy()
-    slots = _slot_rows(slots, pool.shape[0])
-    o = np.zeros(q.shape, dtype=np.float64)
-    for b, slot in enumerate(slots):
-        if slot < 0:
-            continue
-        o[b], pool[slot] = decode_step(q[b], k[b], v[b], pool[slot])
-    return o, pool
+    return _get().decode_step_slots(q, k, v, pool, slots)
 
 
 def decode_step_q8(q, k, v, codes, scales, slots=None):
-    """One step on the 8-bit state, optionally over a slot pool (as above).
-
-    codes: [num_slots, H, d, d] int8, scales: [num_slots, H, d] fp32; without
-    ``slots`` row b uses slot b.  Returns (o fp64, codes', scales')."""
-    orc = _get()
-    q = np.asarray(q)
-    if slots is None:
-        return orc.decode_step_q8(q, np.asarray(k), np.asarray(v), codes, scales)
-    k, v = np.asarray(k), np.asarray(v)
-    codes = np.array(codes, dtype=np.int8, copy=True)
-    scales = np.array(scales, dtype=np.float32, copy=True)
-    slots = _slot_rows(slots, codes.shape[0])
-    o = np.zeros(q.shape, dtype=np.float64)
-    for b, slot in enumerate(slots):
-        if slot < 0:
-            continue
-        o[b], codes[slot], scales[slot] = orc.decode_step_q8(q[b], k[b], v[b], codes[slot], scales[slot])
-    return o, codes, scales
+    return _get().decode_step_q8(q, k, v, codes, scales, slots)

@@ -283,6 +283,38 @@ def pin_q8_rows_becoming_zero(orc):
     assert o[0].tolist() == [tiny, 0.0, 0.0, 0.0]
 
 
+def pin_q8_threshold_and_single_rounding(orc):
+    """Worked by hand.  The zero-row cut is strict and sits at 2^-100: rows with
+    largest magnitude 2^-100 and 2^-95 quantise normally (code 127, scale
+    m / 127), one at 2^-101 is stored as zero.  The step's update is one fused
+    multiply-add: with k = v = 1 + 2^-12 and a dequantised -1, k v - 1 =
+    2^-11 + 2^-24 exactly, which a separately rounded product would lose
+    (fl(k v) = 1 + 2^-11, a tie rounded to even); the row's only non-zero value
+    then sets the scale (2^-11 + 2^-24) / 127."""
+    for e, zero in ((-100, False), (-95, False), (-101, True)):
+        x = np.zeros((1, 8), np.float32)
+        x[0, 3] = np.float32(2.0 ** e)
+        c, a = orc.state_quantize_q8(x)
+        if zero:
+            assert not np.any(c) and a[0] == 0
+        else:
+            assert c[0].tolist() == [0, 0, 0, 127, 0, 0, 0, 0]
+            assert a[0] == np.float32(2.0 ** e) / np.float32(127)
+    d = 2
+    codes = np.array([[[-1, 0], [0, 0]]], np.int8)
+    scales = np.array([[1.0, 0.0]], np.float32)
+    w = np.float32(1.0 + 2.0 ** -12)
+    q = np.array([[1.0, 0.0]], np.float32)
+    k = np.array([[w, 0.0]], np.float32)
+    v = np.array([[w, 0.0]], np.float32)
+    o, c2, a2 = orc.decode_step_q8(q, k, v, codes, scales)
+    s00 = 2.0 ** -11 + 2.0 ** -24
+    assert o[0].tolist() == [s00, 0.0]
+    assert c2[0].tolist() == [[127, 0], [0, 0]]
+    assert a2[0, 0] == np.float32(s00) / np.float32(127) and a2[0, 1] == 0
+    assert d == codes.shape[-1]
+
+
 def pin_q8_integer_trajectory(orc):
     """Rows whose largest magnitude stays exactly 127 have scale 1, so codes are
     the state itself: one-hot keys and small integer values keep every step
@@ -345,7 +377,7 @@ def pin_decode_slots(orc):
     pool = rng.standard_normal((n_slots, H, d, d))
     slots = [3, -1, 0, 4]
     q, k, v = (rng.standard_normal((len(slots), H, d)) for _ in range(3))
-    o, pool2 = oracle.decode_step_slots(q, k, v, pool, slots)
+    o, pool2 = orc.decode_step_slots(q, k, v, pool, slots)
     assert not np.any(o[1])
     assert np.array_equal(pool2[1], pool[1]) and np.array_equal(pool2[2], pool[2])
     for b, s in enumerate(slots):
@@ -357,7 +389,7 @@ def pin_decode_slots(orc):
     # the 8-bit form over the same slots: padding rows untouched as well
     c, a = orc.state_quantize_q8(pool.astype(np.float32))
     qf, kf, vf = (x.astype(np.float32) for x in (q, k, v))
-    o8, c2, a2 = oracle.decode_step_q8(qf, kf, vf, c, a, slots)
+    o8, c2, a2 = orc.decode_step_q8(qf, kf, vf, c, a, slots)
     assert not np.any(o8[1]) and np.array_equal(c2[1], c[1]) and np.array_equal(a2[2], a[2])
     o_dense, c_dense, a_dense = orc.decode_step_q8(qf[0], kf[0], vf[0], c[3], a[3])
     assert np.array_equal(o8[0], o_dense) and np.array_equal(c2[3], c_dense)
@@ -365,7 +397,7 @@ def pin_decode_slots(orc):
 
 PINS = [pin_golden, pin_forms_agree, pin_state_is_KtV, pin_last_row, pin_d1_prefix_sum, pin_N1,
         pin_ternary_bruteforce, pin_state_in, pin_decode, pin_varlen, pin_backward_finite_differences,
-        pin_backward_d1_sums, pin_zero_keys_and_unmasked_identity, pin_q8_golden, pin_q8_rows_becoming_zero, pin_q8_integer_trajectory, pin_q8_within_rounding_bound,
+        pin_backward_d1_sums, pin_zero_keys_and_unmasked_identity, pin_q8_golden, pin_q8_rows_becoming_zero, pin_q8_threshold_and_single_rounding, pin_q8_integer_trajectory, pin_q8_within_rounding_bound,
         pin_decode_slots]
 
 
@@ -408,6 +440,8 @@ MUTANTS = {
                                    "S[r * d + j] = (float)codes[r * d + j] * scales[j % rows];"),
     "q8_zero_row_keeps_old_scale": ("        *a = 0.0f;\n        for (long j = 0; j < d; ++j) c[j] = 0;",
                                     "        for (long j = 0; j < d; ++j) c[j] = 0;"),
+    "q8_threshold_too_high": ("if (m < 0x1p-100f) {", "if (m < 0x1p-90f) {"),
+    "q8_update_rounded_twice": ("s[i * d + j] = fmaf(kb[i], vb[j], deq);", "s[i * d + j] = kb[i] * vb[j] + deq;"),
     "q8_reads_before_update": ("acc += (double)qb[i] * (double)s[i * d + j];",
                                "acc += (double)qb[i] * (double)cb[i * d + j] * ab[i];"),
 }
