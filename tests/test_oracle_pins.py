@@ -440,6 +440,19 @@ MUTANTS = {
                                    "S[r * d + j] = (float)codes[r * d + j] * scales[j % rows];"),
     "q8_zero_row_keeps_old_scale": ("        *a = 0.0f;\n        for (long j = 0; j < d; ++j) c[j] = 0;",
                                     "        for (long j = 0; j < d; ++j) c[j] = 0;"),
+    "varlen_state_layout_transposed": ("memcpy(state_out + (j * H + h) * d * d, S,",
+                                       "memcpy(state_out + (h * num_seqs + j) * d * d, S,"),
+    "varlen_head_list_ignored": ("long h = head_list ? head_list[item / num_seqs] : item / num_seqs;",
+                                 "long h = item / num_seqs;"),
+    "varlen_reads_other_head_k": ("const double* K = k + h * T * d;",
+                                  "const double* K = k + ((h + 1) % H) * T * d;"),
+    "blockwise_intra_uses_previous_block_v": (
+        "intra += P[r * blk + c] * V[(b0 + c) * d + j];",
+        "intra += P[r * blk + c] * V[((b0 >= blk ? b0 - blk : b0) + c) * d + j];"),
+    "quadratic_score_uses_q_twice": ("score += Q[t * d + c] * K[s * d + c];",
+                                     "score += Q[t * d + c] * Q[s * d + c];"),
+    "backward_dv_uses_wrong_score": ("DV[s * d + c] += qk * G[t * d + c];",
+                                     "DV[s * d + c] += gv * G[t * d + c];"),
     "q8_threshold_too_high": ("if (m < 0x1p-100f) {", "if (m < 0x1p-90f) {"),
     "q8_update_rounded_twice": ("s[i * d + j] = fmaf(kb[i], vb[j], deq);", "s[i * d + j] = kb[i] * vb[j] + deq;"),
     "q8_reads_before_update": ("acc += (double)qb[i] * (double)s[i * d + j];",
