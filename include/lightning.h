@@ -38,7 +38,10 @@
  *  - Scratch: long sequences are split into chunks processed in parallel; the
  *    per-chunk states live in a workspace the library takes from the stream-
  *    ordered allocator (cudaMallocAsync / cudaFreeAsync on `stream`).
- *  - Thread safety: calls on different streams may run concurrently.
+ *  - Thread safety: calls from several threads, on different streams, may run
+ *    concurrently.  The device status word (la_get_last_error) and the
+ *    bounded-wait limit (la_set_wait_limit_ns) are per device, shared by all
+ *    streams and threads of the process.
  */
 #ifndef LIGHTNING_H_
 #define LIGHTNING_H_
@@ -265,6 +268,11 @@ const char* la_status_string(int status);
  * la_get_last_error -- sticky error: the first device-side error recorded
  * since the last call (see la_status), else the last asynchronous CUDA error,
  * else LA_OK.  It synchronises the current device and clears the status.
+ * The status word is one per device for the whole process, not one per
+ * stream: an error recorded by work on any stream or thread is reported to,
+ * and cleared by, whichever caller asks first.  Entry points may be called
+ * from several threads and streams at once; callers that need to attribute
+ * a device error to one stream must serialise their checks.
  */
 int la_get_last_error(void);
 
@@ -310,6 +318,37 @@ const char* la_kernel_name(int kernel_id);
 const char* la_prefill_main_kernel(void);
 
 /*
+ * Bounded waits.  Every wait of the device code (an mbarrier phase, a chunk
+ * prefix published by another CTA, a bulk copy landing) gives up after a time
+ * limit of %globaltimer: the kernel then records LA_ERR_TIMEOUT in the device
+ * status, every role of the CTA leaves its loop, the copies and MMAs already
+ * issued are let land, TMEM is freed and the kernel returns; the outputs of
+ * that call are unspecified, the context stays usable.
+ * la_set_wait_limit_ns -- set that limit on the current device for kernels
+ *   launched after the call returns (0 restores the default of 2 s); the old
+ *   value is stored in *previous_ns when previous_ns is not NULL.  One value
+ *   per device for the whole process.  Synchronous; not for use during
+ *   stream capture.
+ */
+int la_set_wait_limit_ns(unsigned long long limit_ns, unsigned long long* previous_ns);
+
+/*
+ * la_debug_fail_allocations -- host-side failure injection for tests: the next
+ * `count` workspace allocations of the library (from any thread) fail as if
+ * the stream-ordered allocator were out of memory, so the calls that need
+ * them return LA_ERR_ALLOC before launching anything; 0 cancels.  Nothing
+ * runs on the device.  Returns LA_OK (LA_ERR_INVALID_ARG if count < 0).
+ */
+int la_debug_fail_allocations(int count);
+
+/*
+ * la_binary_version -- the compute capability the library's kernels were
+ * compiled for, as major * 10 + minor (100 for sm_100a), read from the
+ * loaded code object on the current device; LA_ERR_CUDA if it cannot be read.
+ */
+int la_binary_version(void);
+
+/*
  * la_prefill_noalloc -- la_prefill (bf16, d = 128) that allocates no device
  * memory.  The paper has no counterpart to this entry point: it is a
  * packaging variant of the bf16 prefill for callers that cannot call
@@ -321,10 +360,15 @@ const char* la_prefill_main_kernel(void);
  * Arguments, layouts, results and errors are those of la_prefill.  The
  * per-chunk states that la_prefill keeps in an allocated workspace live here
  * in one fixed array inside the library, LA_NOALLOC_SCRATCH_BYTES large,
- * which every GPU that loads the library holds until the process exits.  The
- * chunking is the one la_prefill chooses; if B*H*n_chunks*d*d*4 bytes of chunk
- * states exceed the array, the call returns LA_ERR_UNSUPPORTED and launches
- * nothing.  (A sequence that fits one chunk needs no scratch at all.)
+ * which every GPU that loads the library holds until the process exits.  It
+ * always runs the three-pass schedule over whole value rows, with the chunk
+ * length la_prefill_ex chooses for flags LA_FLAG_THREE_PASS |
+ * LA_FLAG_NO_SPLIT_V and chunk_tokens = 0 (which depends on B*H, N and the
+ * SM count, and is never shorter than 512 tokens).  With n_chunks =
+ * ceil(N / chunk length), the chunk states take B*H*n_chunks*d*d*4 bytes; if
+ * that exceeds the array the call returns LA_ERR_UNSUPPORTED and launches
+ * nothing.  B*H*ceil(N/512) <= 256 always fits.  (A sequence that fits one
+ * chunk needs no scratch at all.)
  *
  * The first call on each device looks up the device address of the array
  * (cudaGetSymbolAddress) with that device current; make that first call

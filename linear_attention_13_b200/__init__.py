@@ -52,7 +52,8 @@ EXPORTED = ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step"
             "la_prefill_main_kernel", "la_prefill_from_state", "la_prefill_varlen_from_state",
             "la_state_increment", "la_state_prefix", "la_prefill_backward",
             "la_prefill_varlen_ex", "la_decode_step_slots", "la_decode_step_q8",
-            "la_state_quantize_q8", "la_state_dequantize_q8")
+            "la_state_quantize_q8", "la_state_dequantize_q8", "la_set_wait_limit_ns",
+            "la_debug_fail_allocations", "la_binary_version")
 
 LA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -101,6 +102,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la_kernel_name.argtypes = [i]
     lib.la_kernel_name.restype = ctypes.c_char_p
     lib.la_prefill_main_kernel.argtypes = []
+    lib.la_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.la_debug_fail_allocations.argtypes = [i]
+    lib.la_binary_version.argtypes = []
     lib.la_prefill_main_kernel.restype = ctypes.c_char_p
     for name in ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_prefill_varlen_ex",
                  "la_decode_step",
@@ -108,7 +112,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                  "la_timing_read", "la_prefill_noalloc", "la_prefill_from_state",
                  "la_prefill_varlen_from_state", "la_state_increment", "la_state_prefix",
                  "la_prefill_backward", "la_decode_step_slots", "la_decode_step_q8",
-                 "la_state_quantize_q8", "la_state_dequantize_q8"):
+                 "la_state_quantize_q8", "la_state_dequantize_q8", "la_set_wait_limit_ns",
+                 "la_debug_fail_allocations", "la_binary_version"):
         getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -222,6 +227,24 @@ def la_kernel_name(kernel_id):
     return load_library().la_kernel_name(kernel_id).decode()
 
 
+def la_set_wait_limit_ns(limit_ns):
+    """Bounded-wait limit of the device code on the current device (0 = the
+    default of 2 s).  Returns (status, previous limit in ns)."""
+    prev = ctypes.c_ulonglong(0)
+    st = load_library().la_set_wait_limit_ns(int(limit_ns), ctypes.byref(prev))
+    return st, prev.value
+
+
+def la_debug_fail_allocations(count):
+    """Make the library's next ``count`` workspace allocations fail (tests)."""
+    return load_library().la_debug_fail_allocations(count)
+
+
+def la_binary_version():
+    """Compute capability the loaded kernels were built for (100 = sm_100a)."""
+    return load_library().la_binary_version()
+
+
 def la_prefill_main_kernel():
     """Kernel the most recent bf16 prefill launched for its output pass."""
     return load_library().la_prefill_main_kernel().decode()
@@ -249,6 +272,26 @@ def _check(t, name):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _like(t, ref, name, ref_name):
+    """``t`` must be a contiguous CUDA tensor with ``ref``'s shape, dtype and
+    device: the C entry points take raw pointers and cannot check sizes, so a
+    mismatch would become an out-of-bounds access on the device."""
+    _check(t, name)
+    if t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device:
+        raise ValueError(f"{name} must match {ref_name} in shape, dtype and device "
+                         f"(got {tuple(t.shape)} {t.dtype} {t.device}, expected "
+                         f"{tuple(ref.shape)} {ref.dtype} {ref.device})")
+
+
+def _state(t, shape, device, name):
+    """``t`` must be a contiguous float32 CUDA tensor of ``shape`` on ``device``."""
+    _check(t, name)
+    torch = _torch()
+    if t.dtype != torch.float32 or tuple(t.shape) != tuple(shape) or t.device != device:
+        raise ValueError(f"{name} must be float32 {list(shape)} on {device} "
+                         f"(got {t.dtype} {list(t.shape)} on {t.device})")
+
+
 def _stream_ptr(stream):
     torch = _torch()
     s = stream if stream is not None else torch.cuda.current_stream()
@@ -265,19 +308,21 @@ def prefill(q, k, v, blk: int = 128, want_state: bool = True, chunk_tokens: int 
     """Causal linear attention prefill of [B,H,N,d] tensors, from ``state_in``
     ([B,H,d,d] fp32; None = zero).  Returns (o, state)."""
     torch = _torch()
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _check(t, n)
-    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+    _check(q, "q")
+    if q.dim() != 4:
         raise ValueError("q, k, v must share one [B,H,N,d] shape")
+    _like(k, q, "k", "q")
+    _like(v, q, "v", "q")
     B, H, N, d = q.shape
     o = out if out is not None else torch.empty_like(q)
+    _like(o, q, "out", "q")
     st = state_out
     if st is None and want_state:
         st = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    if st is not None:
+        _state(st, (B, H, d, d), q.device, "state_out")
     if state_in is not None:
-        _check(state_in, "state_in")
-        if state_in.dtype != torch.float32 or tuple(state_in.shape) != (B, H, d, d):
-            raise ValueError("state_in must be float32 [B,H,d,d]")
+        _state(state_in, (B, H, d, d), q.device, "state_in")
     status = la_prefill_from_state(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                    state_in.data_ptr() if state_in is not None else None,
                                    st.data_ptr() if st is not None else None, B, H, N, d, blk,
@@ -294,20 +339,27 @@ def prefill_varlen(q, k, v, cu_seqlens, blk: int = 128, want_state: bool = True,
 
     Returns (o, state [num_seqs,H,d,d])."""
     torch = _torch()
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (cu_seqlens, "cu_seqlens")):
-        _check(t, n)
-    if cu_seqlens.dtype != torch.int32:
-        raise TypeError("cu_seqlens must be int32")
+    _check(q, "q")
+    _check(cu_seqlens, "cu_seqlens")
+    if q.dim() != 3:
+        raise ValueError("q, k, v must share one packed [H,T,d] shape")
+    _like(k, q, "k", "q")
+    _like(v, q, "v", "q")
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise TypeError("cu_seqlens must be a 1-D int32 tensor of num_seqs + 1 offsets")
+    if cu_seqlens.device != q.device:
+        raise ValueError("cu_seqlens must be on q's device")
     H, T, d = q.shape
     S = cu_seqlens.numel() - 1
     o = out if out is not None else torch.empty_like(q)
+    _like(o, q, "out", "q")
     st = state_out
     if st is None and want_state:
         st = torch.empty((S, H, d, d), dtype=torch.float32, device=q.device)
+    if st is not None:
+        _state(st, (S, H, d, d), q.device, "state_out")
     if state_in is not None:
-        _check(state_in, "state_in")
-        if state_in.dtype != torch.float32 or tuple(state_in.shape) != (S, H, d, d):
-            raise ValueError("state_in must be float32 [num_seqs,H,d,d]")
+        _state(state_in, (S, H, d, d), q.device, "state_in")
     status = la_prefill_varlen_from_state(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                           state_in.data_ptr() if state_in is not None else None,
                                           st.data_ptr() if st is not None else None,
@@ -321,17 +373,16 @@ def prefill_backward(q, k, v, do, blk: int = 128, stream=None, out=None):
     """Gradients (dq, dk, dv) of sum(do * prefill(q, k, v)[0]) for [B,H,N,d] tensors
     (written into ``out`` = (dq, dk, dv) when given)."""
     torch = _torch()
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (do, "do")):
-        _check(t, n)
-    if not (k.shape == q.shape == v.shape == do.shape) or q.dim() != 4:
+    _check(q, "q")
+    if q.dim() != 4:
         raise ValueError("q, k, v, do must share one [B,H,N,d] shape")
+    for t, n in ((k, "k"), (v, "v"), (do, "do")):
+        _like(t, q, n, "q")
     B, H, N, d = q.shape
     if out is not None:
         dq, dk, dv = out
         for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
-            _check(t, n)
-            if t.shape != q.shape or t.dtype != q.dtype:
-                raise ValueError(f"{n} must match q in shape and dtype")
+            _like(t, q, n, "q")
     else:
         dq, dk, dv = (torch.empty_like(q) for _ in range(3))
     status = la_prefill_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(),
@@ -344,10 +395,13 @@ def prefill_backward(q, k, v, do, blk: int = 128, stream=None, out=None):
 def state_increment(k, v, out=None, stream=None):
     """K^T V over the tokens of [B,H,N,d] bf16 k, v: [B,H,d,d] fp32."""
     torch = _torch()
-    for t, n in ((k, "k"), (v, "v")):
-        _check(t, n)
+    _check(k, "k")
+    if k.dim() != 4:
+        raise ValueError("k, v must share one [B,H,N,d] shape")
+    _like(v, k, "v", "k")
     B, H, N, d = k.shape
     o = out if out is not None else torch.empty((B, H, d, d), dtype=torch.float32, device=k.device)
+    _state(o, (B, H, d, d), k.device, "out")
     status = la_state_increment(k.data_ptr(), v.data_ptr(), o.data_ptr(), B, H, N, d,
                                 _dtype_code(k), _stream_ptr(stream))
     _raise(status, "la_state_increment")
@@ -360,8 +414,11 @@ def state_prefix(states, rank, out=None, stream=None):
     _check(states, "states")
     if states.dtype != torch.float32 or states.dim() != 5:
         raise ValueError("states must be float32 [R,B,H,d,d]")
-    R, B, H, d, _ = states.shape
+    R, B, H, d, d2 = states.shape
+    if d2 != d:
+        raise ValueError("states must be float32 [R,B,H,d,d]")
     o = out if out is not None else torch.empty((B, H, d, d), dtype=torch.float32, device=states.device)
+    _state(o, (B, H, d, d), states.device, "out")
     status = la_state_prefix(states.data_ptr(), R, rank, o.data_ptr(), B, H, d, _stream_ptr(stream))
     _raise(status, "la_state_prefix")
     return o
@@ -370,12 +427,16 @@ def state_prefix(states, rank, out=None, stream=None):
 def decode_step(q, k, v, state, out=None, stream=None):
     """One decode step on [B,H,d] inputs; updates ``state`` [B,H,d,d] fp32 in place."""
     torch = _torch()
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (state, "state")):
-        _check(t, n)
-    if state.dtype != torch.float32:
-        raise TypeError("state must be float32")
+    _check(q, "q")
+    if q.dim() != 3:
+        raise ValueError("q, k, v must share one [B,H,d] shape")
+    _like(k, q, "k", "q")
+    _like(v, q, "v", "q")
     B, H, d = q.shape
+    # the C call updates B*H states of d x d: anything smaller would be overrun
+    _state(state, (B, H, d, d), q.device, "state")
     o = out if out is not None else torch.empty_like(q)
+    _like(o, q, "out", "q")
     status = la_decode_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), state.data_ptr(),
                             o.data_ptr(), B, H, d, _dtype_code(q), _stream_ptr(stream))
     _raise(status, "la_decode_step")
@@ -396,14 +457,19 @@ def decode_step_slots(q, k, v, state_pool, slots, out=None, stream=None):
     ([num_slots,H,d,d] fp32, in place); rows with a negative slot are padding
     (zero output, no state access).  ``slots`` is an int32 CUDA tensor [B]."""
     torch = _torch()
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (state_pool, "state_pool")):
-        _check(t, n)
+    _check(q, "q")
+    if q.dim() != 3:
+        raise ValueError("q, k, v must share one [B,H,d] shape")
+    _like(k, q, "k", "q")
+    _like(v, q, "v", "q")
+    _check(state_pool, "state_pool")
     if state_pool.dtype != torch.float32:
         raise TypeError("state_pool must be float32")
     B, H, d = q.shape
-    if state_pool.dim() != 4 or state_pool.shape[1:] != (H, d, d):
-        raise ValueError("state_pool must be [num_slots, H, d, d]")
+    if state_pool.dim() != 4 or state_pool.shape[1:] != (H, d, d) or state_pool.device != q.device:
+        raise ValueError("state_pool must be [num_slots, H, d, d] on q's device")
     o = out if out is not None else torch.empty_like(q)
+    _like(o, q, "out", "q")
     status = la_decode_step_slots(q.data_ptr(), k.data_ptr(), v.data_ptr(), state_pool.data_ptr(),
                                   _slots_arg(slots, B, torch), state_pool.shape[0], o.data_ptr(),
                                   B, H, d, _dtype_code(q), _stream_ptr(stream))
@@ -416,14 +482,23 @@ def decode_step_q8(q, k, v, codes, scales, slots=None, out=None, stream=None):
     ``scales`` [num_slots,H,d] fp32, updated in place; ``slots`` as for
     ``decode_step_slots`` (None: row b uses slot b)."""
     torch = _torch()
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (codes, "codes"), (scales, "scales")):
+    _check(q, "q")
+    if q.dim() != 3:
+        raise ValueError("q, k, v must share one [B,H,d] shape")
+    _like(k, q, "k", "q")
+    _like(v, q, "v", "q")
+    for t, n in ((codes, "codes"), (scales, "scales")):
         _check(t, n)
     if codes.dtype != torch.int8 or scales.dtype != torch.float32:
         raise TypeError("codes must be int8 and scales float32")
     B, H, d = q.shape
-    if codes.dim() != 4 or codes.shape[1:] != (H, d, d) or scales.shape != codes.shape[:3]:
-        raise ValueError("codes must be [num_slots, H, d, d] and scales [num_slots, H, d]")
+    if (codes.dim() != 4 or codes.shape[1:] != (H, d, d) or scales.shape != codes.shape[:3]
+            or codes.device != q.device or scales.device != q.device):
+        raise ValueError("codes must be [num_slots, H, d, d] and scales [num_slots, H, d] on q's device")
+    if slots is None and codes.shape[0] < B:
+        raise ValueError("without slots, row b uses slot b: codes needs at least B slots")
     o = out if out is not None else torch.empty_like(q)
+    _like(o, q, "out", "q")
     status = la_decode_step_q8(q.data_ptr(), k.data_ptr(), v.data_ptr(), codes.data_ptr(),
                                scales.data_ptr(), _slots_arg(slots, B, torch), codes.shape[0],
                                o.data_ptr(), B, H, d, _dtype_code(q), _stream_ptr(stream))
@@ -438,9 +513,17 @@ def state_quantize_q8(state, codes=None, scales=None, stream=None):
     if state.dtype != torch.float32:
         raise TypeError("state must be float32")
     d = state.shape[-1]
+    if state.dim() < 2 or state.shape[-2] != d:
+        raise ValueError("state must be [..., d, d]")
     c = codes if codes is not None else torch.empty(state.shape, dtype=torch.int8, device=state.device)
     a = scales if scales is not None else torch.empty(state.shape[:-1], dtype=torch.float32,
                                                       device=state.device)
+    _check(c, "codes")
+    _check(a, "scales")
+    if c.dtype != torch.int8 or c.shape != state.shape or c.device != state.device:
+        raise ValueError("codes must be int8 with the state's shape and device")
+    if a.dtype != torch.float32 or a.shape != state.shape[:-1] or a.device != state.device:
+        raise ValueError("scales must be float32 [..., d] on the state's device")
     status = la_state_quantize_q8(state.data_ptr(), c.data_ptr(), a.data_ptr(),
                                   state.numel() // (d * d), d, _stream_ptr(stream))
     _raise(status, "la_state_quantize_q8")
@@ -453,7 +536,12 @@ def state_dequantize_q8(codes, scales, out=None, stream=None):
     _check(codes, "codes")
     _check(scales, "scales")
     d = codes.shape[-1]
+    if codes.dtype != torch.int8 or codes.dim() < 2 or codes.shape[-2] != d:
+        raise ValueError("codes must be int8 [..., d, d]")
+    if scales.dtype != torch.float32 or scales.shape != codes.shape[:-1] or scales.device != codes.device:
+        raise ValueError("scales must be float32 [..., d] on the codes' device")
     o = out if out is not None else torch.empty(codes.shape, dtype=torch.float32, device=codes.device)
+    _state(o, codes.shape, codes.device, "out")
     status = la_state_dequantize_q8(codes.data_ptr(), scales.data_ptr(), o.data_ptr(),
                                     codes.numel() // (d * d), d, _stream_ptr(stream))
     _raise(status, "la_state_dequantize_q8")

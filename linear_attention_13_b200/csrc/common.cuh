@@ -18,8 +18,13 @@ __device__ __forceinline__ void record_device_error(int code) {
     atomicCAS(&g_device_status, (int)LA_OK, code);
 }
 
-// Bounded waits give up after this many nanoseconds of %globaltimer.
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+// Bounded waits give up after g_wait_limit_ns nanoseconds of %globaltimer
+// (la_set_wait_limit_ns changes it; kDefaultWaitLimitNs by default).  Read
+// only once a wait has not completed at its first test.
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;  // 2 s
+__device__ unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
+
+__device__ __forceinline__ unsigned long long wait_limit_ns() { return g_wait_limit_ns; }
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
     unsigned long long t;

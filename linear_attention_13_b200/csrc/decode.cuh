@@ -465,7 +465,7 @@ decode_step_q8_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
         for (long long jj = j; jj < j + kQ8Stages && blockIdx.x + jj * G < n_rows; ++jj) {
             const unsigned long long t0 = globaltimer_ns();
             while (!ptx::mbar_try_wait(bar((int)(jj % kQ8Stages)), (uint32_t)((jj / kQ8Stages) & 1)) &&
-                   globaltimer_ns() - t0 < kWaitLimitNs) {
+                   globaltimer_ns() - t0 < wait_limit_ns()) {
             }
         }
     }

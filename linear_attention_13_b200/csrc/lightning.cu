@@ -42,6 +42,26 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
+// Allocations that the next calls must fail, as if the stream-ordered pool
+// were out of memory (la_debug_fail_allocations: host-side failure injection
+// for the tests; zero in normal use).
+std::atomic<int> g_fail_allocs{0};
+
+// Every workspace of the library comes from here: stream-ordered memory on
+// `s`.  Returns false (after clearing the CUDA error) when it cannot be had;
+// the callers then return LA_ERR_ALLOC before launching anything.
+bool ws_alloc(void** ptr, size_t bytes, cudaStream_t s) {
+    int n = g_fail_allocs.load();
+    while (n > 0) {
+        if (g_fail_allocs.compare_exchange_weak(n, n - 1)) return false;
+    }
+    if (cudaMallocAsync(ptr, bytes, s) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return true;
+}
+
 int note_cuda(cudaError_t e) {
     if (e == cudaSuccess) return LA_OK;
     std::lock_guard<std::mutex> lk(g_mutex);
@@ -344,9 +364,7 @@ int launch_fused(const tc::TileMaps& m, tc::Params p,
         const size_t flag_words = (size_t)n_chunk_slots * p.vparts * tc::kChainWarps;
         const size_t flag_bytes = (flag_words * sizeof(int) + 255) / 256 * 256;
         uint8_t* buf = nullptr;
-        if (cudaMallocAsync(reinterpret_cast<void**>(&buf), chain_bytes + flag_bytes, stream) !=
-            cudaSuccess) {
-            cudaGetLastError();
+        if (!ws_alloc(reinterpret_cast<void**>(&buf), chain_bytes + flag_bytes, stream)) {
             return LA_ERR_ALLOC;
         }
         p.flags = reinterpret_cast<int*>(buf);
@@ -434,8 +452,7 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
     }
     float* ws = nullptr;
     const size_t ws_bytes = (size_t)BH * p.n_chunks * kHeadDim * kHeadDim * sizeof(float);
-    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), ws_bytes, stream) != cudaSuccess) {
-        cudaGetLastError();
+    if (!ws_alloc(reinterpret_cast<void**>(&ws), ws_bytes, stream)) {
         return LA_ERR_ALLOC;
     }
     launch_three_pass(m, p, ws, state_out, grid, stream);
@@ -476,8 +493,7 @@ int launch_prefill_varlen_split(const void* q, const void* k, const void* v, voi
     const int chunk_tokens = ((rows + kTileRows - 1) / kTileRows) * kTileRows;  // >= every length
     const size_t aux_bytes = ((size_t)(2 * num_seqs + 2) * sizeof(int32_t) + 255) / 256 * 256;
     uint8_t* buf = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void**>(&buf), aux_bytes, stream) != cudaSuccess) {
-        cudaGetLastError();
+    if (!ws_alloc(reinterpret_cast<void**>(&buf), aux_bytes, stream)) {
         return LA_ERR_ALLOC;
     }
     int* ok = reinterpret_cast<int*>(buf);
@@ -538,9 +554,7 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
     const size_t ws_bytes = (size_t)H * max_chunks * kHeadDim * kHeadDim * sizeof(float);
     const size_t flag_bytes = three_pass ? 0 : (size_t)H * max_chunks * tc::kChainWarps * sizeof(int);
     uint8_t* buf = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void**>(&buf), aux_bytes + ws_bytes + flag_bytes, stream) !=
-        cudaSuccess) {
-        cudaGetLastError();
+    if (!ws_alloc(reinterpret_cast<void**>(&buf), aux_bytes + ws_bytes + flag_bytes, stream)) {
         return LA_ERR_ALLOC;
     }
     int* ok = reinterpret_cast<int*>(buf);
@@ -822,8 +836,7 @@ int varlen_impl(const void* q, const void* k, const void* v, void* o, const floa
                                           H, blk, s, sms, (flags & LA_FLAG_THREE_PASS) != 0,
                                           chunk_tokens, state_in);
     int* ok = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void**>(&ok), sizeof(int), s) != cudaSuccess) {
-        cudaGetLastError();
+    if (!ws_alloc(reinterpret_cast<void**>(&ok), sizeof(int), s)) {
         return LA_ERR_ALLOC;
     }
     {
@@ -912,8 +925,7 @@ int la_prefill_backward(const void* q, const void* k, const void* v, const void*
     const size_t esz = dt == LA_BF16 ? 2 : 4;
     const int row16 = (int)(d * esz / 16);
     uint8_t* buf = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void**>(&buf), 5 * elems * esz, s) != cudaSuccess) {
-        cudaGetLastError();
+    if (!ws_alloc(reinterpret_cast<void**>(&buf), 5 * elems * esz, s)) {
         return LA_ERR_ALLOC;
     }
     uint8_t* rq = buf;
@@ -1175,6 +1187,40 @@ int la_timing_read(int kernel_id, double* total_ms, int* launches) {
 }
 
 const char* la_prefill_main_kernel(void) { return g_main_kernel.load(); }
+
+int la_set_wait_limit_ns(unsigned long long limit_ns, unsigned long long* previous_ns) {
+    int dev = 0, sms = 0;
+    int st = device_setup(&dev, &sms);
+    if (st != LA_OK) return st;
+    const unsigned long long v = limit_ns == 0 ? kDefaultWaitLimitNs : limit_ns;
+    if (previous_ns != nullptr &&
+        cudaMemcpyFromSymbol(previous_ns, la::g_wait_limit_ns, sizeof(v)) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    if (cudaMemcpyToSymbol(la::g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    return LA_OK;
+}
+
+int la_debug_fail_allocations(int count) {
+    if (count < 0) return LA_ERR_INVALID_ARG;
+    g_fail_allocs.store(count);
+    return LA_OK;
+}
+
+int la_binary_version(void) {
+    int dev = 0, sms = 0;
+    if (device_setup(&dev, &sms) != LA_OK) return LA_ERR_CUDA;
+    cudaFuncAttributes a;
+    if (cudaFuncGetAttributes(&a, tc::prefill_seq_kernel<false>) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    return a.binaryVersion;
+}
 
 const char* la_kernel_name(int kernel_id) {
     switch (kernel_id) {

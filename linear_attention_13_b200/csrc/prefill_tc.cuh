@@ -797,7 +797,7 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
                     const int v = ptx::ld_acquire_gpu(f);
                     if (__all_sync(0xffffffffu, v != 0)) { seen = true; break; }
                     if (*abort_flag) break;
-                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    if (globaltimer_ns() - t0 > wait_limit_ns()) {
                         *abort_flag = 1;
                         record_device_error(LA_ERR_TIMEOUT);
                         break;

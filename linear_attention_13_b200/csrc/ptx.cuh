@@ -52,7 +52,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete, for at most
-// kWaitLimitNs.  `abort_flag` (shared memory) lets one role that gave up stop
+// wait_limit_ns().  `abort_flag` (shared memory) lets one role that gave up stop
 // the others: it is set on timeout and polled while waiting.  Returns false if
 // the wait was abandoned.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
@@ -61,7 +61,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > wait_limit_ns()) {
             *abort_flag = 1;
             record_device_error(LA_ERR_TIMEOUT);
             return false;

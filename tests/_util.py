@@ -34,6 +34,33 @@ def per_head_rel_err(got, ref, head_dims=2) -> float:
     return worst
 
 
+def per_seq_head_rel_err(got, ref, cu_seqlens) -> float:
+    """The parity metric for packed sequences: each (sequence, head) is its own
+    attention problem, so its error is normalised by its own largest |ref|.
+    got, ref are [H, T, d]; cu_seqlens is [S + 1] (host or device).  Returns
+    max over (sequence, head) of max|got - ref| / max|ref| over that
+    sequence's rows of that head; a sequence whose reference is all zero must
+    match exactly.  Empty sequences contribute nothing."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape and ref.ndim == 3, (got.shape, ref.shape)
+    cu = np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens).astype(np.int64)
+    assert cu[0] == 0 and cu[-1] == ref.shape[1], (cu[0], cu[-1], ref.shape)
+    worst = 0.0
+    for a, b in zip(cu[:-1], cu[1:]):
+        if b == a:
+            continue
+        r = ref[:, a:b].reshape(ref.shape[0], -1)
+        d = np.abs(got[:, a:b].reshape(ref.shape[0], -1) - r).max(axis=1)
+        scale = np.abs(r).max(axis=1)
+        if np.any(d[scale == 0.0] != 0.0):
+            return float("inf")
+        nz = scale > 0.0
+        if np.any(nz):
+            worst = max(worst, float(np.max(d[nz] / scale[nz])))
+    return worst
+
+
 def round_like(ref: np.ndarray, dtype) -> np.ndarray:
     """Round fp64 values to ``dtype`` with round-to-nearest-even (as the GPU's
     final conversion does) and widen back to fp64."""

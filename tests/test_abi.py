@@ -39,9 +39,17 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_library_is_built_for_sm100a():
-    labuild.build()
-    out = open(la.LIB_PATH, "rb").read()
-    assert b"sm_100a" in out
+    # the build compiles for sm_100a only (the GPU test reads the loaded code
+    # object's version through la_binary_version)
+    flags = labuild.NVCC_FLAGS
+    i = flags.index("-gencode")
+    assert flags[i + 1] == "arch=compute_100a,code=sm_100a"
+    assert flags.count("-gencode") == 1 and not any("-arch" == f for f in flags)
+
+
+def test_debug_allocation_failures_validate_their_count(lib):
+    assert la.la_debug_fail_allocations(-1) == la.LA_ERR_INVALID_ARG
+    assert la.la_debug_fail_allocations(0) == la.LA_OK
 
 
 def test_status_strings(lib):

@@ -8,7 +8,7 @@ import torch
 import linear_attention_13_b200 as la
 from linear_attention_13_b200 import inputs
 import oracle
-from _util import TOL_O_BF16, TOL_STATE, host64, per_head_rel_err
+from _util import TOL_O_BF16, TOL_STATE, host64, per_head_rel_err, per_seq_head_rel_err
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -54,7 +54,7 @@ def test_random_varlen(case):
     o, st = la.prefill_varlen(q, k, v, cu, blk=128, flags=flags)
     assert la.la_get_last_error() == la.LA_OK
     o_ref, s_ref = oracle.prefill_varlen(host64(q), host64(k), host64(v), cu.cpu().numpy())
-    assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16, (lens, flags)
+    assert per_seq_head_rel_err(host64(o), o_ref, cu) <= TOL_O_BF16, (lens, flags)
     assert per_head_rel_err(host64(st), s_ref) <= TOL_STATE, (lens, flags)
 
 
