@@ -87,7 +87,9 @@ def captured_traffic(kernel: str, path: str = PROFILE_SUMMARY):
     if fields.get("source_sha256") != kernel_source_sha256() or fields.get("kernel") != kernel:
         return None
     try:
-        return int(fields["traffic_bytes_per_launch"])
+        traffic = float(fields["traffic_bytes_per_launch"])
+        traffic *= float(fields.get("traffic_scale_to_full", "1"))
+        return int(traffic)
     except (KeyError, ValueError):
         return None
 
@@ -101,6 +103,22 @@ def load_peaks():
         return p
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS)
+
+
+def line_roofline(kernel: str, alg_bytes: float, launch_ms: float, peaks, summary=None):
+    """Roofline object of one kernel: algorithmic bytes of a launch over its
+    average CUDA-event duration, against measured HBM bandwidth; ``traffic``
+    from the committed ncu summary ``summary`` when it is of this kernel and
+    of the current kernel sources (scaled to a full launch when the summary
+    gives ``traffic_scale_to_full``), else null."""
+    achieved = alg_bytes / (launch_ms / 1e3) / 1e9
+    traffic = None
+    if summary is not None:
+        traffic = captured_traffic(kernel, os.path.join(ROOT, "profiles", summary))
+    return {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+            "peak_source": peaks["source"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic, "algorithmic_bytes_per_launch": int(alg_bytes),
+            "launch_ms": round(launch_ms, 5)}
 
 
 class Dist:
@@ -344,6 +362,12 @@ def bench_ours(args, dist):
         result["secondary"] = bench_secondary(args, device, stream, peaks)
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
+        if "secondary" in result:
+            sec = result["secondary"]
+            budget = max(1.0, args.cpu_budget / 3)
+            sec["long_prefill"]["cpu_baseline"] = cpu_baseline_long(budget)
+            sec["decode"]["cpu_baseline"] = cpu_baseline_decode(budget)
+            sec["varlen_prefill"]["cpu_baseline"] = cpu_baseline_varlen(budget)
     return result
 
 
@@ -442,7 +466,10 @@ def bench_secondary(args, device, stream, peaks):
     la.la_timing_enable(0)
     main64 = kt.get("prefill_main", {"total_ms": float("nan"), "launches": 1})
     k_ms = main64["total_ms"] / max(main64["launches"], 1)
+    kern64 = la.la_prefill_main_kernel()
     out["prefill_blk64"] = {
+        "roofline": line_roofline(kern64, B * H * N * BYTES_PER_TOKEN_HEAD, k_ms, peaks,
+                                  "prefill_tc_kernel_128_64_b4h16n8192.md"),
         "workload": f"prefill bf16 B={B} H={H} N={N} d={D} blk=64",
         "tokens_per_s": round(B * N / (ms / n64 / 1e3), 1), "ms_per_step": round(ms / n64, 5),
         "hbm_frac": round(B * H * N * BYTES_PER_TOKEN_HEAD / (k_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
@@ -463,6 +490,9 @@ def bench_secondary(args, device, stream, peaks):
     la.la_timing_enable(0)
     bytes_bwd = B * H * N * 7 * D * 2      # q, k, v, dO read; dq, dk, dv written (bf16)
     out["backward"] = {
+        "roofline": dict(line_roofline("prefill_seq_kernel (three launches: dq causal, dk and dv "
+                                       "anti-causal)", bytes_bwd, ms / nb, peaks),
+                         note="whole backward step (its three launches) against 1792 B per token-head"),
         "workload": f"prefill backward bf16 B={B} H={H} N={N} d={D} blk=128 (dq, dk, dv)",
         "ms_per_step": round(ms / nb, 5),
         "tokens_per_s": round(B * N / (ms / nb / 1e3), 1),
@@ -510,6 +540,8 @@ def bench_secondary(args, device, stream, peaks):
     k_ms = dec["total_ms"] / max(dec["launches"], 1)
     bytes_step = n_seq * Hd * (8 * D * D + 8 * D)
     out["decode"] = {
+        "roofline": line_roofline("decode_step_kernel", bytes_step, k_ms, peaks,
+                                  "decode_step_kernel_128x64.md"),
         "workload": "decode step, 128 seq x 64 heads, d=128, fp32 state, 256 steps",
         "ms_per_step": round(ms / steps, 5), "GB/s": round(bytes_step / (ms / steps / 1e3) / 1e9, 1),
         "kernel_GB/s": round(bytes_step / (k_ms / 1e3) / 1e9, 1),
@@ -542,6 +574,8 @@ def bench_secondary(args, device, stream, peaks):
     la.la_timing_enable(0)
     dec_pad = kt_pad.get("decode_step_kernel", {"total_ms": float("nan"), "launches": 1})
     out["decode_q8"] = {
+        "roofline": line_roofline("decode_step_q8_kernel", bytes_q8, k_ms, peaks,
+                                  "decode_step_q8_kernel_128x64.md"),
         "workload": "decode step, 128 seq x 64 heads, d=128, 8-bit state (int8 + fp32 row scales), "
                     "256 steps",
         "ms_per_step": round(ms / steps, 5), "kernel_ms": round(k_ms, 5),
@@ -564,7 +598,11 @@ def bench_secondary(args, device, stream, peaks):
     kt = kernel_times(la)
     la.la_timing_enable(0)
     bytes_step = Hl * Nl * BYTES_PER_TOKEN_HEAD
+    main_l = kt.get("prefill_main", {"total_ms": float("nan"), "launches": 1})
     out["long_prefill"] = {
+        "roofline": line_roofline(la.la_prefill_main_kernel(), bytes_step,
+                                  main_l["total_ms"] / max(main_l["launches"], 1), peaks,
+                                  "prefill_tc_kernel_long_b1h64n262144.md"),
         "workload": "prefill bf16 B=1 H=64 N=262144 d=128 blk=128",
         "tokens_per_s": round(Nl / (ms / 5 / 1e3), 1), "ms_per_step": round(ms / 5, 4),
         "hbm_frac": round(bytes_step / (ms / 5 / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
@@ -587,7 +625,11 @@ def bench_secondary(args, device, stream, peaks):
     kt = kernel_times(la)
     la.la_timing_enable(0)
     bytes_step = Hv * Tv * BYTES_PER_TOKEN_HEAD
+    main_v = kt.get("prefill_main", {"total_ms": float("nan"), "launches": 1})
     out["varlen_prefill"] = {
+        "roofline": line_roofline(la.la_prefill_main_kernel(), bytes_step,
+                                  main_v["total_ms"] / max(main_v["launches"], 1), peaks,
+                                  "prefill_tc_kernel_varlen_t2p20.md"),
         "workload": f"packed prefill bf16 T=2^20 ({len(lens)} sequences, lengths U[1024,65536] "
                     "seed 0), H=64, d=128, blk=128",
         "tokens_per_s": round(Tv / (ms / 3 / 1e3), 1), "ms_per_step": round(ms / 3, 4),
@@ -690,6 +732,116 @@ def cpu_baseline(budget_s: float = 15.0):
             "kind": "oracle",
             "sample": f"{reps} x {cores} heads of N={N}, d={D} (fp64 recurrent form), "
                       f"{dt:.1f} s; tokens/s = token-heads/s / H ({H})"}
+
+
+def _oracle_rate(run, budget_s):
+    """Repeat ``run`` (returns the token-heads it processed) for about
+    ``budget_s`` seconds; returns (token-heads per second, reps, seconds)."""
+    t0 = time.perf_counter()
+    done = reps = 0
+    while True:
+        done += run()
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done / dt, reps, dt
+
+
+def cpu_baseline_long(budget_s: float = 5.0):
+    """The fp64 oracle on 4 sampled heads of the long-context prefill (B=1,
+    H=64, N=262144, d=128), on a token prefix sized to the time budget; the
+    full-configuration time is extrapolated from the measured rate."""
+    import torch
+    import oracle
+    from linear_attention_13_b200 import inputs
+    Hl, Nl, heads = 64, 262144, 4
+    q, k, v = inputs.qkv((1, heads, 2048, D), dtype=torch.bfloat16, device="cpu", seed=0)
+    q, k, v = (t.to(torch.float64).numpy() for t in (q, k, v))
+    t0 = time.perf_counter()
+    oracle.prefill_recurrent(q, k, v)
+    per_token = (time.perf_counter() - t0) / 2048
+    n_tok = int(min(Nl, max(2048, budget_s / max(per_token, 1e-9) / 2)))
+    q, k, v = inputs.qkv((1, heads, n_tok, D), dtype=torch.bfloat16, device="cpu", seed=0)
+    q, k, v = (t.to(torch.float64).numpy() for t in (q, k, v))
+    rate, reps, dt = _oracle_rate(lambda: (oracle.prefill_recurrent(q, k, v), heads * n_tok)[1], budget_s)
+    return {"value": round(rate / Hl, 1), "unit": UNIT, "cores": min(heads, oracle.num_threads()),
+            "kind": "oracle", "token_heads_per_s": round(rate, 1),
+            "extrapolated_full_config_s": round(Hl * Nl / rate, 1),
+            "sample": f"{reps} x {heads} sampled heads x {n_tok} tokens of B=1 H=64 N=262144 d=128 "
+                      f"(fp64 recurrent form, one thread per head), {dt:.1f} s; tokens/s = "
+                      f"token-heads/s / 64; full-configuration time extrapolated"}
+
+
+def cpu_baseline_decode(budget_s: float = 5.0):
+    """The fp64 oracle on the decode configuration (128 sequences x 64 heads,
+    d=128): one all-head step, and 16 sampled (sequence, head) trajectories of a
+    4096-token prefill plus 256 steps."""
+    import numpy as np
+    import torch
+    import oracle
+    from linear_attention_13_b200 import inputs
+    n_seq, Hd, N0, steps = 128, 64, 4096, 256
+    rng = np.random.default_rng(0)
+    S = rng.standard_normal((n_seq, Hd, D, D))
+    qq, kk, vv = (t.to(torch.float64).numpy() for t in inputs.decode_step_inputs(n_seq, Hd, D, 1))
+    t0 = time.perf_counter()
+    oracle.decode_step(qq, kk, vv, S)
+    step_s = time.perf_counter() - t0
+    del S
+    # 16 trajectories: prefill of 4096 tokens, then 256 single-token steps
+    q, k, v = inputs.qkv((1, 16, N0, D), dtype=torch.bfloat16, device="cpu", seed=0)
+    q, k, v = (t.to(torch.float64).numpy() for t in (q, k, v))
+    t0 = time.perf_counter()
+    _, st = oracle.prefill_recurrent(q, k, v)
+    for s_ in range(1, steps + 1):
+        a, b_, c = (t.to(torch.float64).numpy() for t in inputs.qkv((1, 16, D), dtype=torch.bfloat16, seed=s_))
+        _, st = oracle.decode_step(a, b_, c, st)
+    traj_s = time.perf_counter() - t0
+    head_steps = n_seq * Hd
+    return {"value": round(head_steps / step_s, 1), "unit": "head-steps/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "state_GB_per_s_fp32_equivalent": round(head_steps * 8 * D * D / step_s / 1e9, 2),
+            "all_head_step_s": round(step_s, 3),
+            "trajectories_s": round(traj_s, 2),
+            "extrapolated_256_steps_s": round(steps * step_s, 1),
+            "sample": "one step of all 128 x 64 heads (fp64 states), plus 16 sampled (sequence, head) "
+                      "trajectories of a 4096-token prefill and 256 steps; 256-step time extrapolated"}
+
+
+def cpu_baseline_varlen(budget_s: float = 5.0):
+    """The fp64 oracle on 8 sampled heads of the packed prefill (T=2^20,
+    lengths U[1024, 65536] seed 0, H=64, d=128), over the first packed
+    sequences that fit the time budget; the full time is extrapolated."""
+    import numpy as np
+    import torch
+    import oracle
+    from linear_attention_13_b200 import inputs
+    Tv, Hv, heads = 1 << 20, 64, 8
+    lens = inputs.varlen_lengths(Tv, 1024, 65536, seed=0)
+    # token budget from a short probe, then whole leading sequences
+    q, k, v = inputs.qkv((heads, 2048, D), dtype=torch.bfloat16, device="cpu", seed=0)
+    q, k, v = (t.to(torch.float64).numpy() for t in (q, k, v))
+    t0 = time.perf_counter()
+    oracle.prefill_varlen(q, k, v, np.array([0, 2048], dtype=np.int32))
+    per_token = (time.perf_counter() - t0) / 2048
+    want = int(budget_s / max(per_token, 1e-9) / 2)
+    take, acc = [], 0
+    for n in lens:
+        if acc and acc + n > want:
+            break
+        take.append(n)
+        acc += n
+    cu = inputs.cu_seqlens_from_lengths(take)
+    q, k, v = inputs.qkv((heads, acc, D), dtype=torch.bfloat16, device="cpu", seed=0)
+    q, k, v = (t.to(torch.float64).numpy() for t in (q, k, v))
+    rate, reps, dt = _oracle_rate(lambda: (oracle.prefill_varlen(q, k, v, cu), heads * acc)[1], budget_s)
+    return {"value": round(rate / Hv, 1), "unit": UNIT, "cores": min(heads, oracle.num_threads()),
+            "kind": "oracle", "token_heads_per_s": round(rate, 1),
+            "extrapolated_full_config_s": round(Hv * Tv / rate, 1),
+            "sample": f"{reps} x {heads} sampled heads x the first {len(take)} packed sequences "
+                      f"({acc} tokens) of T=2^20, H=64, d=128 (fp64 recurrent form per sequence), "
+                      f"{dt:.1f} s; tokens/s = token-heads/s / 64; full time extrapolated"}
 
 
 def bench_reference(args, dist):

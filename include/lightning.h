@@ -342,6 +342,22 @@ int la_set_wait_limit_ns(unsigned long long limit_ns, unsigned long long* previo
 int la_debug_fail_allocations(int count);
 
 /*
+ * Test hooks for the failure paths of the look-back (single pass) schedule.
+ * la_debug_skip_lookback_items -- the next look-back launch on any stream
+ *   starts its work-item tickets at `count` instead of 0: the first `count`
+ *   items are never processed, so the chunks that follow them wait for a
+ *   state prefix that is never published, and their bounded waits run out
+ *   (LA_ERR_TIMEOUT in the device status).  One launch only; 0 cancels.
+ * la_debug_occupy_sms -- launch `ctas` CTAs on `stream`, each holding most of
+ *   an SM's shared memory and waiting `duration_ns` (at most 1 s) on the
+ *   clock before it exits: other kernels then run on the remaining SMs.
+ * Both return LA_OK or LA_ERR_INVALID_ARG / LA_ERR_CUDA.  They exist for
+ * tests; nothing else calls them.
+ */
+int la_debug_skip_lookback_items(int count);
+int la_debug_occupy_sms(int ctas, unsigned long long duration_ns, void* stream);
+
+/*
  * la_binary_version -- the compute capability the library's kernels were
  * compiled for, as major * 10 + minor (100 for sm_100a), read from the
  * loaded code object on the current device; LA_ERR_CUDA if it cannot be read.

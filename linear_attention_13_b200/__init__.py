@@ -53,7 +53,8 @@ EXPORTED = ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step"
             "la_state_increment", "la_state_prefix", "la_prefill_backward",
             "la_prefill_varlen_ex", "la_decode_step_slots", "la_decode_step_q8",
             "la_state_quantize_q8", "la_state_dequantize_q8", "la_set_wait_limit_ns",
-            "la_debug_fail_allocations", "la_binary_version")
+            "la_debug_fail_allocations", "la_binary_version", "la_debug_skip_lookback_items",
+            "la_debug_occupy_sms")
 
 LA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -105,6 +106,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong)]
     lib.la_debug_fail_allocations.argtypes = [i]
     lib.la_binary_version.argtypes = []
+    lib.la_debug_skip_lookback_items.argtypes = [i]
+    lib.la_debug_occupy_sms.argtypes = [i, ctypes.c_ulonglong, vp]
     lib.la_prefill_main_kernel.restype = ctypes.c_char_p
     for name in ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_prefill_varlen_ex",
                  "la_decode_step",
@@ -113,7 +116,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                  "la_prefill_varlen_from_state", "la_state_increment", "la_state_prefix",
                  "la_prefill_backward", "la_decode_step_slots", "la_decode_step_q8",
                  "la_state_quantize_q8", "la_state_dequantize_q8", "la_set_wait_limit_ns",
-                 "la_debug_fail_allocations", "la_binary_version"):
+                 "la_debug_fail_allocations", "la_binary_version", "la_debug_skip_lookback_items",
+                 "la_debug_occupy_sms"):
         getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -238,6 +242,16 @@ def la_set_wait_limit_ns(limit_ns):
 def la_debug_fail_allocations(count):
     """Make the library's next ``count`` workspace allocations fail (tests)."""
     return load_library().la_debug_fail_allocations(count)
+
+
+def la_debug_skip_lookback_items(count):
+    """The next look-back launch skips its first ``count`` items (tests)."""
+    return load_library().la_debug_skip_lookback_items(count)
+
+
+def la_debug_occupy_sms(ctas, duration_ns, stream=None):
+    """Hold ``ctas`` SMs for ``duration_ns`` (<= 1 s) with a waiting kernel (tests)."""
+    return load_library().la_debug_occupy_sms(ctas, int(duration_ns), _stream_ptr(stream))
 
 
 def la_binary_version():

@@ -22,6 +22,19 @@
 #include "decode.cuh"
 
 namespace la {
+
+// A CTA with most of an SM's shared memory that waits (bounded, on
+// %globaltimer) and exits: la_debug_occupy_sms holds SMs away from other
+// kernels with it, so that tests can run the look-back prefill on part of the
+// GPU.  It waits on nothing but the clock.
+constexpr int kOccupySmem = 160 * 1024;
+__global__ void __launch_bounds__(32) occupy_kernel(unsigned long long duration_ns) {
+    extern __shared__ uint8_t occupied[];
+    const unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < duration_ns) __nanosleep(2000);
+    if (threadIdx.x == 0) occupied[0] = 0;
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -235,7 +248,7 @@ int make_tile_maps(tc::TileMaps* m, const void* q, const void* k, const void* v,
                    uint64_t rows, uint64_t outer) {
     if (make_tmap_bf16_tile(&m->q, q, rows, outer) || make_tmap_bf16_tile(&m->k, k, rows, outer) ||
         make_tmap_bf16_tile(&m->v, v, rows, outer) || make_tmap_bf16(&m->v_half, v, rows, outer) ||
-        make_tmap_bf16(&m->o, o, rows, outer))
+        make_tmap_bf16(&m->o, o, rows, outer) || make_tmap_bf16(&m->k_half, k, rows, outer))
         return LA_ERR_CUDA;
     return LA_OK;
 }
@@ -355,19 +368,26 @@ int choose_fused_chunk_tokens(int Z, int N, int ctas) {
     return best * kTileRows;
 }
 
-// Single pass with look-back: one launch (plus a memset of the chunk flags).
+// Items the next look-back launch skips (la_debug_skip_lookback_items: a test
+// hook; their successors' bounded waits then run out).  Consumed by one launch.
+std::atomic<int> g_skip_items{0};
+
+// Single pass with look-back: one launch (plus a memset of the chunk flags and
+// the item counter).
 int launch_fused(const tc::TileMaps& m, tc::Params p,
                  long n_chunk_slots, float* state_out, int grid, cudaStream_t stream) {
     p.state_out = state_out;
     if (n_chunk_slots > 0) {
         const size_t chain_bytes = (size_t)n_chunk_slots * kHeadDim * kHeadDim * sizeof(float);
-        const size_t flag_words = (size_t)n_chunk_slots * p.vparts * tc::kChainWarps;
+        const size_t flag_words = (size_t)n_chunk_slots * p.vparts * tc::kChainWarps + 1;  // + counter
         const size_t flag_bytes = (flag_words * sizeof(int) + 255) / 256 * 256;
         uint8_t* buf = nullptr;
         if (!ws_alloc(reinterpret_cast<void**>(&buf), chain_bytes + flag_bytes, stream)) {
             return LA_ERR_ALLOC;
         }
         p.flags = reinterpret_cast<int*>(buf);
+        p.ticket = p.flags + flag_words - 1;
+        p.ticket_base = g_skip_items.exchange(0);
         p.chain = reinterpret_cast<float*>(buf + flag_bytes);
         p.fused = 1;
         cudaMemsetAsync(p.flags, 0, flag_words * sizeof(int), stream);
@@ -552,7 +572,8 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
     if (make_tile_maps(&m, q, k, v, o, rows, H)) return LA_ERR_CUDA;
     const size_t aux_bytes = ((size_t)(num_seqs + 2) * sizeof(int32_t) + 255) / 256 * 256;
     const size_t ws_bytes = (size_t)H * max_chunks * kHeadDim * kHeadDim * sizeof(float);
-    const size_t flag_bytes = three_pass ? 0 : (size_t)H * max_chunks * tc::kChainWarps * sizeof(int);
+    const size_t flag_words = three_pass ? 0 : (size_t)H * max_chunks * tc::kChainWarps + 1;  // + counter
+    const size_t flag_bytes = flag_words * sizeof(int);
     uint8_t* buf = nullptr;
     if (!ws_alloc(reinterpret_cast<void**>(&buf), aux_bytes + ws_bytes + flag_bytes, stream)) {
         return LA_ERR_ALLOC;
@@ -593,6 +614,8 @@ int launch_prefill_varlen_bf16(const void* q, const void* k, const void* v, void
         p.fused = 1;
         p.chain = ws;
         p.flags = chunk_flags;
+        p.ticket = chunk_flags + flag_words - 1;
+        p.ticket_base = g_skip_items.exchange(0);
         p.state_out = state_out;
         {
             TimedLaunch tl(LA_KERNEL_PREFILL_TC, stream);
@@ -693,6 +716,7 @@ int launch_prefill_bf16_noalloc(const void* q, const void* k, const void* v, voi
 using namespace la;
 
 namespace {
+
 
 int decode_args_ok(const void* q, const void* k, const void* v, const void* o, int B, int H, int d,
                    la_dtype dt) {
@@ -1203,6 +1227,26 @@ int la_set_wait_limit_ns(unsigned long long limit_ns, unsigned long long* previo
         return LA_ERR_CUDA;
     }
     return LA_OK;
+}
+
+int la_debug_skip_lookback_items(int count) {
+    if (count < 0) return LA_ERR_INVALID_ARG;
+    g_skip_items.store(count);
+    return LA_OK;
+}
+
+int la_debug_occupy_sms(int ctas, unsigned long long duration_ns, void* stream) {
+    if (ctas < 1 || duration_ns > 1000000000ull) return LA_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    int st = device_setup(&dev, &sms);
+    if (st != LA_OK) return st;
+    if (cudaFuncSetAttribute(occupy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOccupySmem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    occupy_kernel<<<ctas, 32, kOccupySmem, reinterpret_cast<cudaStream_t>(stream)>>>(duration_ns);
+    return note_cuda(cudaGetLastError());
 }
 
 int la_debug_fail_allocations(int count) {

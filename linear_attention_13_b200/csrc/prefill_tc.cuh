@@ -23,11 +23,11 @@
 // or from packed sequences ([H][T][d] split by cu_seqlens, section 4 of the
 // same page: data packing), where a chunk never crosses a sequence end.
 //
-// Roles in the main kernel (one CTA of 320 threads per SM, persistent):
-//   warp 0     TMA producer (lane 0 issues; the warp zeroes packed tails)
-//   warp 1     TMEM allocator and MMA issuer (one thread)
-//   warps 2-9  two epilogue warpgroups: TMEM -> registers -> mask / convert /
-//              store, warpgroup h handling columns [64h, 64h+64) of every row
+// Three kernels carry the outputs, each a persistent, warp-specialised CTA
+// per SM (roles listed at each kernel): prefill_tc_kernel (whole value rows,
+// single pass with look-back over chunk states, or 64-token blocks),
+// prefill_seq_kernel (value columns split over two CTAs, two MMA issuers)
+// and chunk_state_kernel (the first pass of the three-pass schedule).
 #pragma once
 
 #include <cuda.h>
@@ -46,7 +46,7 @@ constexpr int kStages = 2;
 __host__ __device__ constexpr int stage_bytes(int nv) { return 2 * kTileBytes + (nv / 64) * kHalfBytes; }
 __host__ __device__ constexpr int sbar_offset(int nv) { return kStages * stage_bytes(nv); }
 __host__ __device__ constexpr int ctrl_offset(int nv) { return sbar_offset(nv) + (nv / 64) * kHalfBytes; }
-__host__ __device__ constexpr int smem_bytes(int nv) { return ctrl_offset(nv) + 256 + 1024; }
+__host__ __device__ constexpr int smem_bytes(int nv) { return ctrl_offset(nv) + 512 + 1024; }
 
 // TMEM columns (fp32 cells; 128 lanes each)
 constexpr uint32_t kColState = 0;    // S      [k-dim lanes][v-dim cols]
@@ -81,6 +81,12 @@ constexpr int kThreads = 32 * (kFirstChainWarp + kChainWarps);
 constexpr int kModeDense = 0;
 constexpr int kModeVarlen = 1;
 
+// Work items of prefill_tc_kernel pass from its producer to the other roles
+// through a ring of kRing entries; each is read by the MMA issuer, the 8
+// epilogue warps and the 4 chain warps.
+constexpr int kRing = 4;
+constexpr int kRingReaders = 1 + kEpiWarps + kChainWarps;
+
 struct Ctrl {
     uint64_t full[kStages];
     uint64_t empty[kStages];     // every MMA of the tile done (V and Q no longer read)
@@ -97,9 +103,14 @@ struct Ctrl {
     uint64_t state_free;   // epilogue finished with TMEM S / S̄ of an item
     uint64_t o_staged;     // every epilogue warp wrote its part of O (bf16) to smem
     uint64_t o_stored[kStages];  // O tile staged in stage s has left shared memory
+    uint64_t ring_full[kRing];   // ring entry written by the producer
+    uint64_t ring_free[kRing];   // ring entry read by every reader (kRingReaders)
+    uint64_t drain;              // the issuer's last MMAs complete (teardown)
+    int ring[kRing];             // item of each claimed position (n_items: no more)
     uint32_t tmem_base;
     int abort;
 };
+static_assert(sizeof(Ctrl) <= 512, "control block");
 
 // Work description shared by every kernel of the schedule.
 struct Params {
@@ -128,6 +139,11 @@ struct Params {
                                 // (non-empty sequences, longest first), or null
     const float* state_in;      // starting state of every sequence (layout of state_out),
                                 // or null (zero)
+    int* ticket;                // single pass: item counter (zeroed with the flags); a
+                                // CTA takes its items from it in increasing order, so
+                                // an item's predecessor chunk has always been taken by
+                                // a CTA that is running.  Null: items by static stride
+    int ticket_base;            // first item the counter hands out (0)
 };
 
 // One work item: rows [t0, t1) of slice z, chunk c of its sequence, value
@@ -244,7 +260,7 @@ __device__ __forceinline__ void zero_tail_rows(uint8_t* vtile, int valid, int la
 // producer thread loads.  v_half and o are {128, rows, Z} maps with a
 // {64, 128, 1} box: one half tile of V (split value columns) or of O.
 struct TileMaps {
-    CUtensorMap q, k, v, v_half, o;
+    CUtensorMap q, k, v, v_half, o, k_half;
 };
 
 // Warp-wide producer step: wait until stage `s` may be refilled, then load Q
@@ -354,6 +370,11 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
         ptx::mbar_init(bar(ctrl->state_free), kEpiWarps);
         ptx::mbar_init(bar(ctrl->o_staged), kEpiWarps);
         for (int s = 0; s < kStages; ++s) ptx::mbar_init(bar(ctrl->o_stored[s]), 1);
+        for (int i = 0; i < kRing; ++i) {
+            ptx::mbar_init(bar(ctrl->ring_full[i]), 1);
+            ptx::mbar_init(bar(ctrl->ring_free[i]), kRingReaders);
+        }
+        ptx::mbar_init(bar(ctrl->drain), 1);
         ctrl->abort = 0;
         ptx::fence_mbar_init();
     }
@@ -379,6 +400,15 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
     const int stride = gridDim.x;
     // phase A is run for chunks that have a successor (single pass only)
     auto has_phase_a = [&](const Item& it) { return fused && !it.last; };
+    // Item at ring position j (the CTA's j-th item; n_items = none), once the
+    // producer has written it; false on abort.
+    auto read_pos = [&](uint32_t j, int& item) -> bool {
+        const uint32_t slot = j % kRing;
+        if (!ptx::mbar_wait(bar(ctrl->ring_full[slot]), (j / kRing) & 1, abort_flag)) return false;
+        item = *reinterpret_cast<volatile int*>(&ctrl->ring[slot]);
+        return true;
+    };
+    auto release_pos = [&](uint32_t j) { ptx::mbar_arrive(bar(ctrl->ring_free[j % kRing])); };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -390,6 +420,9 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
         uint32_t g = 0, n_tail = 0;
         bool ok = true;
         uint32_t c_uses[kStages] = {0, 0};   // phase-C uses of each stage so far
+        // the last load into each stage (its barrier and phase parity), which
+        // the teardown after an abort lets land
+        uint32_t ld_bar0 = 0, ld_par0 = 0, ld_bar1 = 0, ld_par1 = 0;
         // One tile (rows [t, t+128) of item it) into stage g & 1.  Each operand
         // is loaded as soon as its slot is free: K once the stage's previous
         // tile finished MMA4 (k_empty), V once it finished MMA2 (empty), and Q
@@ -405,18 +438,26 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
             if (lane == 0) {
                 if (g >= 2) w = ptx::mbar_wait(bar(ctrl->k_empty[s]), ((g >> 1) + 1) & 1, abort_flag);
                 if (w) {
-                    ptx::mbar_arrive_expect_tx(fb, (phase_c ? 2 : 1) * kTileBytes + kVHalves * kHalfBytes);
+                    // K counts on the phase now; the arrival comes with V (and Q)
+                    ptx::mbar_expect_tx(fb, kTileBytes);
+                    if (s == 0) { ld_bar0 = fb; ld_par0 = tail ? (n_tail & 1) : ((g >> 1) & 1); }
+                    else { ld_bar1 = fb; ld_par1 = tail ? (n_tail & 1) : ((g >> 1) & 1); }
                     ptx::tma_load_4d(stage + kTileBytes, &maps.k, fb, 0, t, 0, it.z, pol_k);
                     if (g >= 2) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
-                }
-                if (w) {
-                    if (kVHalves == 2)
-                        ptx::tma_load_4d(stage + 2 * kTileBytes, &maps.v, fb, 0, t, 0, it.z, pol_v);
-                    else
-                        ptx::tma_load_3d(stage + 2 * kTileBytes, &maps.v_half, fb, it.vp * kNV, t, it.z, pol_v);
-                    if (phase_c && c_uses[s] > 0)
+                    if (w && phase_c && c_uses[s] > 0)
                         w = ptx::mbar_wait(bar(ctrl->o_stored[s]), (c_uses[s] - 1) & 1, abort_flag);
-                    if (w && phase_c) ptx::tma_load_4d(stage, &maps.q, fb, 0, t, 0, it.z, pol_qk);
+                    if (w) {
+                        ptx::mbar_arrive_expect_tx(fb, (phase_c ? kTileBytes : 0) + kVHalves * kHalfBytes);
+                        if (kVHalves == 2)
+                            ptx::tma_load_4d(stage + 2 * kTileBytes, &maps.v, fb, 0, t, 0, it.z, pol_v);
+                        else
+                            ptx::tma_load_3d(stage + 2 * kTileBytes, &maps.v_half, fb, it.vp * kNV, t, it.z, pol_v);
+                        if (phase_c) ptx::tma_load_4d(stage, &maps.q, fb, 0, t, 0, it.z, pol_qk);
+                    } else {
+                        // aborted after K: close the phase on K alone, so that the
+                        // teardown can wait for it to land
+                        ptx::mbar_arrive(fb);
+                    }
                 }
             }
             if (!__shfl_sync(0xffffffffu, w, 0)) return false;
@@ -438,19 +479,53 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
             for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g)
                 if (!produce(it, t, false)) ok = false;
         };
-        if ((int)blockIdx.x < n_items) {
-            const Item first = get_item(p, blockIdx.x);
+        // ---- work items: taken here -- from the ticket counter in the single
+        //      pass (so that items start in increasing order across the grid),
+        //      by a static stride otherwise -- and handed to the other roles
+        //      through the ring.  Returns the item (n_items: none), -1 on abort.
+        uint32_t n_claimed = 0;
+        bool ended = false;
+        auto claim = [&]() -> int {
+            int item = n_items, w = 1;
+            if (lane == 0) {
+                const uint32_t slot = n_claimed % kRing;
+                if (n_claimed >= (uint32_t)kRing)
+                    w = ptx::mbar_wait(bar(ctrl->ring_free[slot]), ((n_claimed / kRing) + 1) & 1, abort_flag);
+                if (w) {
+                    if (!ended) {
+                        item = p.ticket != nullptr ? p.ticket_base + atomicAdd(p.ticket, 1)
+                                                   : (int)blockIdx.x + (int)n_claimed * stride;
+                        item = min(item, n_items);
+                    }
+                    *reinterpret_cast<volatile int*>(&ctrl->ring[slot]) = item;
+                    ptx::mbar_arrive(bar(ctrl->ring_full[slot]));
+                }
+            }
+            w = __shfl_sync(0xffffffffu, w, 0);
+            item = __shfl_sync(0xffffffffu, item, 0);
+            if (!w) return -1;
+            ended = ended || item >= n_items;
+            ++n_claimed;
+            return item;
+        };
+        int cur = claim();
+        if (cur >= 0 && cur < n_items) {
+            const Item first = get_item(p, cur);
             if (has_phase_a(first)) load_phase_a(first);
         }
-        for (int item = blockIdx.x; ok && item < n_items; item += stride) {
-            const Item it = get_item(p, item);
-            if (item + stride < n_items) {
-                const Item nx = get_item(p, item + stride);
+        while (ok && cur >= 0 && cur < n_items) {
+            const Item it = get_item(p, cur);
+            const int nxi = claim();
+            if (nxi < 0) { ok = false; break; }
+            if (nxi < n_items) {
+                const Item nx = get_item(p, nxi);
                 if (has_phase_a(nx)) load_phase_a(nx);
             }
             for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g)
                 if (!produce(it, t, true)) ok = false;
+            cur = nxi;
         }
+        if (cur < 0) ok = false;
         // Wait for the last stage releases (MMA commits and O stores) so that no
         // asynchronous arrive is still pending on this CTA's shared memory when
         // it exits.
@@ -461,6 +536,11 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
             }
             for (int s = 0; ok && s < kStages; ++s)
                 if (c_uses[s] > 0) ok = ptx::mbar_wait(bar(ctrl->o_stored[s]), (c_uses[s] - 1) & 1, abort_flag);
+            if (!ok) {
+                // after an abort: let the loads already issued land (bounded)
+                if (ld_bar0) ptx::mbar_drain(ld_bar0, ld_par0);
+                if (ld_bar1) ptx::mbar_drain(ld_bar1, ld_par1);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -470,7 +550,7 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
             constexpr uint32_t id_kv = ptx::idesc_bf16(128, kNV, true, true);      // K^T V
             constexpr uint32_t id_pv = ptx::idesc_bf16(kBlk, kNV, false, true);    // P V
             uint32_t g = 0, n_sb = 0, n_a = 0, n_blk = 0;
-            bool ok = true;
+            bool ok = true, issued = false;
             // phase A: TMEM delta = K_c^T V_c over the chunk's blocks
             auto run_phase_a = [&](const Item& it) {
                 if (n_a > 0 && !ptx::mbar_wait(bar(ctrl->delta_free), (n_a - 1) & 1, abort_flag)) {
@@ -493,18 +573,24 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
                     ptx::mma_commit(bar(ctrl->k_empty[s]));
                     ptx::mma_commit(bar(ctrl->empty[s]));
                     first = false;
+                    issued = true;
                 }
                 ptx::mma_commit(bar(ctrl->delta_done));
                 ++n_a;
             };
-            if ((int)blockIdx.x < n_items) {
-                const Item first = get_item(p, blockIdx.x);
+            uint32_t pos = 0;
+            int cur = n_items;
+            if (!read_pos(0, cur)) ok = false;
+            if (ok && cur < n_items) {
+                const Item first = get_item(p, cur);
                 if (has_phase_a(first)) run_phase_a(first);
             }
-            for (int item = blockIdx.x; ok && item < n_items; item += stride) {
-                const Item it = get_item(p, item);
-                if (item + stride < n_items) {
-                    const Item nx = get_item(p, item + stride);
+            for (; ok && cur < n_items; ++pos) {
+                const Item it = get_item(p, cur);
+                int nxi = n_items;
+                if (!read_pos(pos + 1, nxi)) { ok = false; break; }
+                if (nxi < n_items) {
+                    const Item nx = get_item(p, nxi);
                     if (has_phase_a(nx)) run_phase_a(nx);
                     if (!ok) break;
                 }
@@ -564,10 +650,19 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
                         }
                         ptx::mma_commit(bar(ctrl->o_full));
                         has_state = true;
+                        issued = true;
                     }
                     if (!ok) break;
                     ptx::mma_commit(bar(ctrl->empty[s]));
                 }
+                if (!ok) break;
+                release_pos(pos);
+                cur = nxi;
+            }
+            // teardown: every MMA this thread issued has completed
+            if (issued) {
+                ptx::mma_commit(bar(ctrl->drain));
+                ptx::mbar_drain(bar(ctrl->drain), 0);
             }
         }
     } else if (warp < kFirstChainWarp) {
@@ -586,15 +681,20 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
         // stage a phase-C block occupies
         uint32_t g = 0;
         auto n_tiles = [&](const Item& x) { return (uint32_t)((x.t1 - x.t0 + kTileRows - 1) / kTileRows); };
-        if ((int)blockIdx.x < n_items) {
-            const Item first = get_item(p, blockIdx.x);
+        bool ok = true;
+        uint32_t pos = 0;
+        int cur = n_items;
+        if (!read_pos(0, cur)) ok = false;
+        if (ok && cur < n_items) {
+            const Item first = get_item(p, cur);
             if (has_phase_a(first)) g += n_tiles(first);
         }
-        bool ok = true;
-        for (int item = blockIdx.x; ok && item < n_items; item += stride) {
-            const Item it = get_item(p, item);
-            if (item + stride < n_items) {
-                const Item nx = get_item(p, item + stride);
+        for (; ok && cur < n_items; ++pos) {
+            const Item it = get_item(p, cur);
+            int nxi = n_items;
+            if (!read_pos(pos + 1, nxi)) { ok = false; break; }
+            if (nxi < n_items) {
+                const Item nx = get_item(p, nxi);
                 if (has_phase_a(nx)) g += n_tiles(nx);
             }
             for (int t = it.t0; t < it.t1; t += kTileRows, ++g, ++n_tile) {
@@ -753,6 +853,10 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
                 __syncwarp();
                 if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             }
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            if (lane == 0) release_pos(pos);
+            cur = nxi;
         }
         if (store_leader) ptx::bulk_wait_group0();
     } else {
@@ -770,7 +874,10 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
         uint32_t n_delta = 0, n_sf = 0;
         bool ok = true;
         bool first_item = true;
-        for (int item = blockIdx.x; ok && item < n_items; item += stride) {
+        for (uint32_t pos = 0; ok; ++pos) {
+            int item = n_items;
+            if (!read_pos(pos, item)) { ok = false; break; }
+            if (item >= n_items) break;
             const Item it = get_item(p, item);
             const bool phase_a = has_phase_a(it);
             const bool look = fused && it.c > 0;
@@ -881,6 +988,7 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
             __syncwarp();
             // sbar_ready counts epilogue warps: each chain warp stands for two
             if (lane == 0) ptx::mbar_arrive_cnt(bar(ctrl->sbar_ready), kEpiWarps / kChainWarps);
+            if (lane == 0) release_pos(pos);
         }
     }
 
@@ -930,13 +1038,13 @@ struct Ctrl {
     uint64_t v_empty[kStages];  // V slot of stage s read (MMA2)
     uint64_t tail_ld;
     uint64_t s_full[2];     // MMA1 complete (scores buffer b)
-    uint64_t p_ready;       // P written (8 warps)
+    uint64_t p_ready[2];    // P of block parity b written (8 warps)
     uint64_t ds_full[2];    // MMA4 complete (dS buffer b)
     uint64_t p_free[2];     // MMA2 complete: P buffer b consumed
     uint64_t mma3_done[2];  // MMA3 (or, without a state, MMA1) of the block using buffer b
     uint64_t ds_free[2];    // dS buffer read (8 warps)
-    uint64_t sbar_ready;    // S̄ written (8 warps)
-    uint64_t o_full;        // MMA2 complete
+    uint64_t sbar_ready[2]; // S̄ read by the block of parity b written (8 warps)
+    uint64_t o_full[2];     // MMA2 of block parity b complete
     uint64_t o_free[2];     // O buffer read (8 warps)
     uint64_t o_staged;      // O staged in shared memory (8 warps)
     uint64_t ost_free;      // the O staging buffer has been read by its TMA store
@@ -969,9 +1077,11 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         }
         ptx::mbar_init(bar(ctrl->ost_free), 1);
         ptx::mbar_init(bar(ctrl->tail_ld), 1);
-        ptx::mbar_init(bar(ctrl->p_ready), sq::kEpiWarps);
-        ptx::mbar_init(bar(ctrl->sbar_ready), sq::kEpiWarps);
-        ptx::mbar_init(bar(ctrl->o_full), 1);
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(bar(ctrl->p_ready[b]), sq::kEpiWarps);
+            ptx::mbar_init(bar(ctrl->sbar_ready[b]), sq::kEpiWarps);
+            ptx::mbar_init(bar(ctrl->o_full[b]), 1);
+        }
         ptx::mbar_init(bar(ctrl->o_staged), sq::kEpiWarps);
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(bar(ctrl->s_full[b]), 1);
@@ -1116,7 +1226,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                         ptx::mma_commit(bar(ctrl->s_full[b]));
                         // MMA3: O = Q S̄_{g-1} into buffer b (S̄ buffer (g-1) & 1), once
                         // the epilogue has read block g-2's O there
-                        if (!ptx::mbar_wait(bar(ctrl->sbar_ready), g & 1, abort_flag)) { ok = false; break; }
+                        if (!ptx::mbar_wait(bar(ctrl->sbar_ready[b]), par, abort_flag)) { ok = false; break; }
                         if (g >= 2 && !ptx::mbar_wait(bar(ctrl->o_free[b]), prev, abort_flag)) { ok = false; break; }
                         ptx::tc_fence_after();
                         if (has_state) {
@@ -1144,7 +1254,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                         ptx::mma_commit(bar(ctrl->ds_full[b]));
                         ptx::mma_commit(bar(ctrl->empty[s]));    // K read
                         // MMA2: O += P V (P in TMEM buffer b), after MMA3 wrote O
-                        if (!ptx::mbar_wait(bar(ctrl->p_ready), g & 1, abort_flag)) { ok = false; break; }
+                        if (!ptx::mbar_wait(bar(ctrl->p_ready[b]), par, abort_flag)) { ok = false; break; }
                         if (!ptx::mbar_wait(bar(ctrl->mma3_done[b]), par, abort_flag)) { ok = false; break; }
                         ptx::tc_fence_after();
 #pragma unroll
@@ -1152,7 +1262,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                             ptx::mma_ts(o_cols, tmem + sq::kColSP + b * 128 + p_col(kk) - kColS,
                                         ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_pv,
                                         (kk > 0 || has_state) ? 1u : 0u);
-                        ptx::mma_commit(bar(ctrl->o_full));
+                        ptx::mma_commit(bar(ctrl->o_full[b]));
                         ptx::mma_commit(bar(ctrl->p_free[b]));
                         ptx::mma_commit(bar(ctrl->v_empty[s]));  // V read
                     }
@@ -1181,6 +1291,9 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // Per block g: P(g), then S += dS_g and S̄_g, then the output of the
+        // PREVIOUS block, so that MMA2(g) (issued once P(g) is written) runs
+        // while this block's state and the previous output are handled.
         const int ew = warp - 2;             // 0..7
         const int sp = warp & 3;             // TMEM sub-partition of this warp
         const int r = sp * 32 + lane;        // tile row owned by this thread
@@ -1189,10 +1302,52 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
         uint32_t g = 0;
         bool ok = true;
+        // the block whose output is still to be drained
+        bool o_pending = false;
+        Item o_it;
+        int o_t = 0;
+        uint32_t o_g = 0;
+        // ---- O of block og: registers, release its buffer, stage as bf16 for
+        //      the store warp once it has stored the previous tile
+        auto drain_o = [&](const Item& oit, int ot, uint32_t og) -> bool {
+            const uint32_t ob = og & 1;
+            if (!ptx::mbar_wait(bar(ctrl->o_full[ob]), (og >> 1) & 1, abort_flag)) return false;
+            ptx::tc_fence_after();
+            const bool rowwise = packed && ot + kTileRows > oit.t1;
+            uint8_t* ostage = smem + sq::kOstOff;
+            uint32_t v[32];
+            ptx::tmem_ld32(tl + sq::kColO + ob * sq::kNV + c0, v);
+            ptx::tmem_ld_wait();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_free[ob]));
+            if (og >= 1 && !ptx::mbar_wait(bar(ctrl->ost_free), (og - 1) & 1, abort_flag)) return false;
+            if (!rowwise) {
+                store_row32_bf16_sw128(ostage, r, c0, v);
+                ptx::fence_proxy_async_smem();
+            } else if (ot + r < oit.t1) {
+                uint4* orow = reinterpret_cast<uint4*>(
+                    p.o + ((size_t)oit.z * p.rows + ot + r) * kHeadDim + oit.vp * sq::kNV + c0);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint4 w;
+                    w.x = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+                    w.y = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+                    w.z = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+                    w.w = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+                    orow[j] = w;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_staged));
+            return true;
+        };
         for (int item = blockIdx.x; ok && item < n_items; item += stride) {
             const Item it = get_item(p, item);
             const int vcol = it.vp * sq::kNV + c0;  // first owned column of the 128
-            // ---- running state S (row r, columns vcol..vcol+31) and S̄ for block 0
+            // ---- running state S (row r, columns vcol..vcol+31) and S̄ for block g
+            //      (S̄ buffer (g - 1) & 1, last read by MMA3 of block g - 2, which A
+            //      issued before MMA1 of block g - 1, whose s_full was observed)
             float srun[32];
             if (const float* st0 = start_state(p, it)) {
                 const float4* src = reinterpret_cast<const float4*>(st0 + (size_t)r * kHeadDim + vcol);
@@ -1207,15 +1362,14 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 uint32_t f[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
-                // S̄ buffer read by this item's first block g: (g - 1) & 1
-                store_row32_bf16_sw128(smem + sq::kSbarOff + ((g + 1) & 1) * kHalfBytes - 0, r, c0, f);
+                store_row32_bf16_sw128(smem + sq::kSbarOff + ((g + 1) & 1) * kHalfBytes, r, c0, f);
                 ptx::fence_proxy_async_smem();
             } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) srun[j] = 0.f;
             }
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready));
+            if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready[g & 1]));
 
             for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
                 const bool last_block = t + kTileRows >= it.t1;
@@ -1251,7 +1405,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(ctrl->p_ready));
+                if (lane == 0) ptx::mbar_arrive(bar(ctrl->p_ready[b]));
 
                 // ---- 2. S += dS_g; S̄_g for the next block, or the final state
                 if (!ptx::mbar_wait(bar(ctrl->ds_full[b]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
@@ -1267,15 +1421,15 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     for (int j = 0; j < 32; ++j) srun[j] += __uint_as_float(d[j]);
                 }
                 if (!last_block) {
-                    // buffer g & 1 was last read by MMA3 of block g-1, complete
-                    // since its o_full was observed below in the previous block
+                    // S̄ buffer g & 1 was last read by MMA3 of block g-1; A issued it
+                    // before MMA1(g), so s_full(g), observed above, covers it
                     uint32_t f[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
                     store_row32_bf16_sw128(smem + sq::kSbarOff + (g & 1) * kHalfBytes, r, c0, f);
                     ptx::fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready));
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready[(g + 1) & 1]));
                 } else if (p.state_out != nullptr) {
                     float4* dst = reinterpret_cast<float4*>(
                         p.state_out + (size_t)it.sidx * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim + vcol);
@@ -1284,41 +1438,17 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                         dst[j] = make_float4(srun[4 * j], srun[4 * j + 1], srun[4 * j + 2], srun[4 * j + 3]);
                 }
 
-                // ---- 3. O: registers, release buffer b, stage as bf16 for the
-                //         store warp once it has stored the previous tile
-                if (!ptx::mbar_wait(bar(ctrl->o_full), g & 1, abort_flag)) { ok = false; break; }
-                ptx::tc_fence_after();
-                const bool rowwise = packed && t + kTileRows > it.t1;
-                uint8_t* ostage = smem + sq::kOstOff;
-                {
-                    uint32_t v[32];
-                    ptx::tmem_ld32(tl + sq::kColO + b * sq::kNV + c0, v);
-                    ptx::tmem_ld_wait();
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_free[b]));
-                    if (g >= 1 && !ptx::mbar_wait(bar(ctrl->ost_free), (g - 1) & 1, abort_flag)) { ok = false; break; }
-                    if (!rowwise) {
-                        store_row32_bf16_sw128(ostage, r, c0, v);
-                        ptx::fence_proxy_async_smem();
-                    } else if (t + r < it.t1) {
-                        uint4* orow = reinterpret_cast<uint4*>(p.o + ((size_t)it.z * p.rows + t + r) * kHeadDim + vcol);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint4 w;
-                            w.x = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
-                            w.y = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
-                            w.z = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
-                            w.w = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
-                            orow[j] = w;
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_staged));
-                }
+                // ---- 3. the previous block's output
+                if (o_pending && !drain_o(o_it, o_t, o_g)) { ok = false; break; }
+                o_pending = true;
+                o_it = it;
+                o_t = t;
+                o_g = g;
             }
         }
+        if (ok && o_pending) drain_o(o_it, o_t, o_g);
     }
+
 
     ptx::tc_fence_before();
     __syncthreads();
