@@ -1033,7 +1033,8 @@ constexpr int kThreads = 32 * (4 + kEpiWarps);
 constexpr int kL2Ahead = 2;                 // tiles prefetched into L2 ahead of the load
 
 struct Ctrl {
-    uint64_t full[kStages];
+    uint64_t full_qk[kStages];  // Q and K of stage s landed (MMA1 and MMA3 need no V)
+    uint64_t full_v[kStages];   // V of stage s landed (packed tails: foreign rows cleared)
     uint64_t empty[kStages];    // Q and K slots of stage s read (MMA1, MMA3, MMA4)
     uint64_t v_empty[kStages];  // V slot of stage s read (MMA2)
     uint64_t tail_ld;
@@ -1071,7 +1072,8 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            ptx::mbar_init(bar(ctrl->full[s]), 1);
+            ptx::mbar_init(bar(ctrl->full_qk[s]), 1);
+            ptx::mbar_init(bar(ctrl->full_v[s]), 1);
             ptx::mbar_init(bar(ctrl->empty[s]), 2);   // one commit from each MMA issuer
             ptx::mbar_init(bar(ctrl->v_empty[s]), 1);
         }
@@ -1147,19 +1149,25 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 const uint32_t stage = sbase + s * sq::kStageB;
                 prefetch(it, t, sq::kL2Ahead);
                 // Q and K of block g reuse slots that block g-2's MMA1, MMA3 and MMA4
-                // have finished with; V waits for its MMA2, which comes later
+                // have finished with; V waits for its MMA2, which comes later.  Q
+                // and K complete on their own barrier, so MMA1 of block g never
+                // waits for the load of V (issued one MMA2 later)
                 const bool tail = packed && it.t1 - t < kTileRows;
-                const uint32_t fb = tail ? bar(ctrl->tail_ld) : bar(ctrl->full[s]);
+                const uint32_t fv = tail ? bar(ctrl->tail_ld) : bar(ctrl->full_v[s]);
                 int w = 1;
                 if (lane == 0) {
                     if (g >= 2) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
                     if (w) {
                         const int row = tile_row(it, t);
-                        ptx::mbar_arrive_expect_tx(fb, 2 * kTileBytes + kHalfBytes);
-                        ptx::tma_load_4d(stage, &maps.q, fb, 0, row, 0, it.z, pol_qk);
-                        ptx::tma_load_4d(stage + kTileBytes, &maps.k, fb, 0, row, 0, it.z, pol_qk);
+                        const uint32_t fqk = bar(ctrl->full_qk[s]);
+                        ptx::mbar_arrive_expect_tx(fqk, 2 * kTileBytes);
+                        ptx::tma_load_4d(stage, &maps.q, fqk, 0, row, 0, it.z, pol_qk);
+                        ptx::tma_load_4d(stage + kTileBytes, &maps.k, fqk, 0, row, 0, it.z, pol_qk);
                         if (g >= 2) w = ptx::mbar_wait(bar(ctrl->v_empty[s]), ((g >> 1) + 1) & 1, abort_flag);
-                        if (w) ptx::tma_load_3d(stage + 2 * kTileBytes, &maps.v_half, fb, it.vp * sq::kNV, row, it.z, pol_v);
+                        if (w) {
+                            ptx::mbar_arrive_expect_tx(fv, kHalfBytes);
+                            ptx::tma_load_3d(stage + 2 * kTileBytes, &maps.v_half, fv, it.vp * sq::kNV, row, it.z, pol_v);
+                        }
                     }
                 }
                 if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
@@ -1171,7 +1179,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     zero_tail_rows(smem + s * sq::kStageB + 2 * kTileBytes, it.t1 - t, lane, 1);
                     ptx::fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->full[s]));
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->full_v[s]));
                 }
             }
         }
@@ -1205,7 +1213,8 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     const uint32_t b = g & 1;
                     const uint32_t par = (g >> 1) & 1;           // phase parity of buffer b's barriers
                     const uint32_t prev = ((g >> 1) + 1) & 1;    // ... for block g - 2
-                    if (!ptx::mbar_wait(bar(ctrl->full[s]), par, abort_flag)) { ok = false; break; }
+                    if (!ptx::mbar_wait(bar(ctrl->full_qk[s]), par, abort_flag)) { ok = false; break; }
+                    if (!is_a && !ptx::mbar_wait(bar(ctrl->full_v[s]), par, abort_flag)) { ok = false; break; }
                     ptx::tc_fence_after();
                     const uint32_t sq_ = sbase + s * sq::kStageB;
                     const uint32_t sk = sq_ + kTileBytes;
