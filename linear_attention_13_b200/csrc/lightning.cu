@@ -316,9 +316,14 @@ tc::Params dense_params(int BH, int N, int chunk_tokens, void* o) {
 // would leave many SMs idle and the sequences are short enough that one CTA
 // per (head, half) finishes in time (measured on B200: at 64 heads the split
 // wins at 8K tokens and loses to chunking at 256K).
+// When the split fills 80-100 % of the SMs with one CTA per (head, half), it
+// also wins for long sequences: every tile is read once, where chunking reads
+// the K and V of every chunk with a successor twice (B200, 64 heads of 262144
+// tokens: 3.47 ms split against 3.95 ms for the best chunking).
 bool want_split_v(long slices, long N, int sms, int flags) {
     if (flags & LA_FLAG_NO_SPLIT_V) return false;
     if (flags & LA_FLAG_SPLIT_V) return true;
+    if (2 * slices * 5 >= (long)sms * 4 && 2 * slices <= (long)sms) return true;
     return slices * 4 < (long)sms * 3 && N <= 16384;
 }
 
@@ -349,8 +354,10 @@ void launch_three_pass(const tc::TileMaps& m, tc::Params p, float* ws, float* st
 }
 
 // Chunk length for the single-pass schedule: minimise rounds of work items
-// times (blocks per chunk + a per-chunk overhead of about two blocks), with
-// chunks of at least 512 tokens.
+// times the time of an item, in 128-token blocks: a chunk with a successor
+// also reads its K and V once more for the look-back (half a block's bytes
+// per block) and hands its prefix over (about two blocks).  Chunks of at least
+// 512 tokens.
 int choose_fused_chunk_tokens(int Z, int N, int ctas) {
     const int nblk = (N + kTileRows - 1) / kTileRows;
     int best = nblk;
@@ -359,7 +366,7 @@ int choose_fused_chunk_tokens(int Z, int N, int ctas) {
         const int nch = (nblk + cb - 1) / cb;
         if (nch > 1 && cb * (nch - 1) >= nblk) continue;
         const long rounds = ((long)Z * nch + ctas - 1) / ctas;
-        const double cost = (double)rounds * (cb + (nch > 1 ? 2.0 : 0.5));
+        const double cost = (double)rounds * (nch > 1 ? 1.5 * cb + 2.0 : cb + 0.5);
         if (cost < best_cost - 1e-9) {
             best_cost = cost;
             best = cb;
@@ -481,14 +488,16 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
     return st;
 }
 
-// Single pass over packed sequences: chunks of 8192 tokens (best of the
-// measured 1K-8K range on B200 for 2^20 tokens x 64 heads: fewer look-back
-// links outweigh the lost L2 reuse).
+// Single pass over packed sequences: chunks of about half a CTA's share of the
+// work, H * T / (2 * ctas) tokens, at least 8192.  A chunk with a successor
+// has its K and V read twice, so long chunks save traffic as long as the work
+// items stay small against a CTA's share (B200, 2^20 tokens x 64 heads in
+// sequences of 1K-64K tokens: 8192-token chunks 17.4 ms, one chunk per
+// sequence 12.5 ms).
 int choose_varlen_fused_chunk_tokens(int H, int T, int ctas) {
-    (void)H;
-    (void)T;
-    (void)ctas;
-    return 8192;
+    const long share = (long)H * T / (2L * std::max(ctas, 1));
+    const long t_rounded = ((long)T + kTileRows - 1) / kTileRows * kTileRows;
+    return (int)std::max(8192L, std::min(share, t_rounded));
 }
 
 // Chunk length for packed sequences: long enough to keep the chunk-state

@@ -108,11 +108,15 @@ def test_bf16_prefill_config_all_heads(blk):
     assert per_head_rel_err(host64(st), s_ref) <= TOL_STATE
 
 
-def test_bf16_long_context_sampled_heads():
-    # B=1, H=64, N=262144, d=128: 4 sampled heads (first, last, two seeded).
+@pytest.mark.parametrize("flags", [0, la.LA_FLAG_FUSED | la.LA_FLAG_NO_SPLIT_V, la.LA_FLAG_THREE_PASS],
+                         ids=["default", "single-pass", "three-pass"])
+def test_bf16_long_context_sampled_heads(flags):
+    # B=1, H=64, N=262144, d=128: 4 sampled heads (first, last, two seeded), in
+    # the default schedule (value columns split, one chunk per head) and in the
+    # chunked ones.
     B, H, N, d = 1, 64, 262144, 128
     q, k, v = inputs.qkv((B, H, N, d), dtype=torch.bfloat16, device=DEV, seed=0)
-    o, st = _run(q, k, v, 128)
+    o, st = _run(q, k, v, 128, flags=flags)
     rng = np.random.default_rng(0)
     heads = [0, H - 1] + sorted(rng.choice(np.arange(1, H - 1), 2, replace=False).tolist())
     hq, hk, hv = (host64(x[0, heads]) for x in (q, k, v))

@@ -129,15 +129,17 @@ def test_varlen_bf16_bad_seqlens_detected(flags):
     assert torch.all(o == 3.0) and torch.all(st == 3.0)
 
 
-@pytest.mark.parametrize("flags", [pytest.param(0, id="default"), pytest.param(la.LA_FLAG_SPLIT_V, id="split-v")])
-def test_varlen_bf16_packed_config_sampled_heads(flags):
+@pytest.mark.parametrize("flags,chunk", [pytest.param(0, 0, id="default"),
+                                         pytest.param(la.LA_FLAG_SPLIT_V, 0, id="split-v"),
+                                         pytest.param(la.LA_FLAG_FUSED, 8192, id="single-pass-8k")])
+def test_varlen_bf16_packed_config_sampled_heads(flags, chunk):
     # 2^20 packed tokens, lengths uniform in [1024, 65536] (seeded, last
     # trimmed), H = 64, d = 128: every sequence of 8 sampled heads.
     T, H = 1 << 20, 64
     lens = inputs.varlen_lengths(T, 1024, 65536, seed=0)
     cu = _cu(lens)
     q, k, v = inputs.qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=0)
-    o, st = la.prefill_varlen(q, k, v, cu, blk=128, flags=flags)
+    o, st = la.prefill_varlen(q, k, v, cu, blk=128, flags=flags, chunk_tokens=chunk)
     assert la.la_get_last_error() == la.LA_OK
     rng = np.random.default_rng(0)
     heads = [0, H - 1] + sorted(rng.choice(np.arange(1, H - 1), 6, replace=False).tolist())
