@@ -602,7 +602,7 @@ def bench_secondary(args, device, stream, peaks):
     out["long_prefill"] = {
         "roofline": line_roofline(la.la_prefill_main_kernel(), bytes_step,
                                   main_l["total_ms"] / max(main_l["launches"], 1), peaks,
-                                  "prefill_tc_kernel_long_b1h64n262144.md"),
+                                  "prefill_seq_kernel_long_b1h64n262144.md"),
         "workload": "prefill bf16 B=1 H=64 N=262144 d=128 blk=128",
         "tokens_per_s": round(Nl / (ms / 5 / 1e3), 1), "ms_per_step": round(ms / 5, 4),
         "hbm_frac": round(bytes_step / (ms / 5 / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
@@ -649,6 +649,11 @@ PROFILE_CASES = {
     "long_prefill_32k": "prefill bf16 B=1 H=64 N=32768 d=128 blk=128 (long-context shape, "
                         "1/8 of the length)",
     "varlen_32k": "packed prefill bf16 T=2^15, lengths U[1024,8192] seed 0, H=64, d=128",
+    "varlen_2heads": "packed prefill bf16 T=2^20, lengths U[1024,65536] seed 0 (the packed "
+                     "configuration's sequences), H=2, d=128, one chunk per sequence (the schedule "
+                     "the 64-head configuration runs)",
+    "backward": "prefill backward bf16 B=4 H=16 N=8192 d=128 blk=128 (dq causal, dk and dv "
+                "anti-causal launches)",
 }
 
 
@@ -687,6 +692,24 @@ def profile_case(args):
 
         def call():
             la.decode_step_q8(qq, kk, vv, codes, scales, out=od)
+    elif name == "varlen_2heads":
+        Tv, Hv = 1 << 20, 2
+        lens = inputs.varlen_lengths(Tv, 1024, 65536, seed=0)
+        cu = torch.from_numpy(inputs.cu_seqlens_from_lengths(lens)).to(device)
+        q, k, v = inputs.qkv((Hv, Tv, D), dtype=torch.bfloat16, device=device, seed=0)
+        o = torch.empty_like(q)
+        st = torch.empty((len(lens), Hv, D, D), dtype=torch.float32, device=device)
+
+        def call():
+            la.prefill_varlen(q, k, v, cu, blk=BLK, out=o, state_out=st, chunk_tokens=Tv,
+                              flags=la.LA_FLAG_FUSED)
+    elif name == "backward":
+        q, k, v = inputs.qkv((B, H, N, D), dtype=torch.bfloat16, device=device, seed=0)
+        do = inputs.qkv((B, H, N, D), dtype=torch.bfloat16, device=device, seed=1)[2]
+        grads = tuple(torch.empty_like(q) for _ in range(3))
+
+        def call():
+            la.prefill_backward(q, k, v, do, blk=BLK, out=grads)
     elif name == "varlen_32k":
         Tv, Hv = 1 << 15, 64
         lens = inputs.varlen_lengths(Tv, 1024, 8192, seed=0)

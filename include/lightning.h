@@ -164,11 +164,13 @@ int la_prefill_varlen_from_state(const void* q, const void* k, const void* v, vo
  *     dv_s = sum_{t >= s} (q_t . k_s) dO_t     (the anti-causal form of (k, q, dO))
  *   q, k, v, do_ : [B, H, N, d] of dt (read only); dq, dk, dv : [B, H, N, d]
  *   of dt (written).  Same dtype, d, blk rules as la_prefill.  For bf16 with
- *   blk = 128 and N <= 16384 the anti-causal forms run directly (the tiles of
- *   each sequence taken from the last) and no scratch is used; otherwise they
- *   are causal forms of the token-reversed sequence, reversed back, with five
- *   tensors of the input size of scratch from the stream-ordered allocator
- *   (LA_ERR_ALLOC if that fails).  The pages
+ *   blk = 128 the anti-causal forms run directly (the tiles of each sequence
+ *   taken from the last) and no scratch is used when N <= 16384, or for any N
+ *   when 2*B*H is between 80 % and 100 % of the SM count (one CTA pair per
+ *   sequence fills the GPU); otherwise they are causal forms of the
+ *   token-reversed sequence, reversed back, with five tensors of the input
+ *   size of scratch from the stream-ordered allocator (LA_ERR_ALLOC if that
+ *   fails).  The pages
  *   give no backward pass (training is the context of section 2 of the
  *   futurefh page); this is the derivative of the forward definition.
  */

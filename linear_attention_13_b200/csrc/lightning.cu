@@ -416,14 +416,19 @@ int launch_fused(const tc::TileMaps& m, tc::Params p,
 
 // The anti-causal form o_t = sum_{s >= t} (q_t . k_s) v_s, bf16, d = 128, 128-token
 // blocks: prefill_seq_kernel with one chunk per sequence, walking its blocks from
-// the last to the first (the state then holds suffix sums).  Sequences longer
-// than kReverseMaxN are not covered (LA_ERR_UNSUPPORTED): one CTA pair per
-// sequence would serialise too many blocks.
+// the last to the first (the state then holds suffix sums).  It runs when the
+// sequences are short (N <= kReverseMaxN) or when one CTA pair per sequence
+// fills the GPU (as the forward's split schedule); other shapes return
+// LA_ERR_UNSUPPORTED: too few CTAs would each walk too many blocks.
 constexpr int kReverseMaxN = 16384;
+
+bool reverse_direct_ok(long BH, long N, int sms) {
+    return N <= kReverseMaxN || (2 * BH * 5 >= (long)sms * 4 && 2 * BH <= (long)sms);
+}
 
 int launch_prefill_reverse_bf16(const void* q, const void* k, const void* v, void* o, int BH, int N,
                                 cudaStream_t stream, int sms) {
-    if (N > kReverseMaxN) return LA_ERR_UNSUPPORTED;
+    if (!reverse_direct_ok(BH, N, sms)) return LA_ERR_UNSUPPORTED;
     tc::TileMaps m;
     if (make_tile_maps(&m, q, k, v, o, N, BH)) return LA_ERR_CUDA;
     tc::Params p = dense_params(BH, N, ((N + kTileRows - 1) / kTileRows) * kTileRows, o);
@@ -946,9 +951,10 @@ int la_prefill_backward(const void* q, const void* k, const void* v, const void*
     // dk_s = sum_{t >= s} (v_s . dO_t) q_t and dv_s = sum_{t >= s} (k_s . q_t) dO_t are
     // anti-causal forms: (q, k, v) = (v, dO, q) and (k, q, dO).  The split kernel
     // runs them directly for 128-token blocks of bf16 sequences up to
-    // kReverseMaxN tokens; otherwise they are causal sums of the token-reversed
-    // sequence, reversed back.
-    if (dt == LA_BF16 && blk == 128 && N <= kReverseMaxN) {
+    // kReverseMaxN tokens, or of any length when one CTA pair per sequence fills
+    // the GPU; otherwise they are causal sums of the token-reversed sequence,
+    // reversed back.
+    if (dt == LA_BF16 && blk == 128 && reverse_direct_ok((long)B * H, N, sms)) {
         st = launch_prefill_reverse_bf16(v, do_, q, dk, B * H, N, s, sms);
         if (st == LA_OK) st = launch_prefill_reverse_bf16(k, q, do_, dv, B * H, N, s, sms);
         return st;

@@ -65,3 +65,18 @@ def round_like(ref: np.ndarray, dtype) -> np.ndarray:
     """Round fp64 values to ``dtype`` with round-to-nearest-even (as the GPU's
     final conversion does) and widen back to fp64."""
     return torch.from_numpy(np.ascontiguousarray(ref)).to(dtype).to(torch.float64).numpy()
+
+
+def grads_via_recurrent(orc, q, k, v, do):
+    """Gradients of sum(dO * o) from the oracle's recurrent (O(N d^2)) form:
+    dq is the causal form of (dO, v, k); dk and dv are the anti-causal forms
+    of (v, dO, q) and (k, q, dO), i.e. causal forms of the token-reversed
+    sequences, reversed back.  For long sequences, where the oracle's own
+    (quadratic) backward is too slow; pinned against it on small inputs."""
+    def rev(x):
+        return np.ascontiguousarray(np.asarray(x)[..., ::-1, :])
+    dq, _ = orc.prefill_recurrent(do, v, k)
+    dk_r, _ = orc.prefill_recurrent(rev(v), rev(do), rev(q))
+    dv_r, _ = orc.prefill_recurrent(rev(k), rev(q), rev(do))
+    return dq, rev(dk_r), rev(dv_r)
+

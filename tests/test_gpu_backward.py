@@ -7,7 +7,7 @@ import torch
 import linear_attention_13_b200 as la
 from linear_attention_13_b200 import inputs
 import oracle
-from _util import TOL_O_BF16, TOL_O_F32, host64, per_head_rel_err, round_like
+from _util import TOL_O_BF16, TOL_O_F32, grads_via_recurrent, host64, per_head_rel_err, round_like
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -70,3 +70,25 @@ def test_autograd_matches_oracle():
     refs = _grads_ref(q.detach(), k.detach(), v.detach(), w)
     for x, ref in zip((q, k, v), refs):
         assert per_head_rel_err(host64(x.grad), ref) <= TOL_O_BF16
+
+
+def test_bf16_backward_long_context_sampled_heads():
+    # B=1, H=64, N=262144 (the long-context shape): one CTA pair per head fills
+    # the GPU, so dk and dv run as anti-causal passes without reversal copies;
+    # 4 sampled heads against the recurrent-form reference
+    B, H, N = 1, 64, 262144
+    q, k, v = inputs.qkv((B, H, N, 128), dtype=torch.bfloat16, device=DEV, seed=41)
+    do = inputs.qkv((B, H, N, 128), dtype=torch.bfloat16, device=DEV, seed=42)[2]
+    la.la_timing_enable(64)
+    dq, dk, dv = la.prefill_backward(q, k, v, do)
+    torch.cuda.synchronize()
+    _, _, n_aux = la.la_timing_read(la.LA_KERNEL_AUX)
+    la.la_timing_enable(0)
+    assert la.la_get_last_error() == la.LA_OK
+    assert n_aux == 0                      # no token-reversal copies were made
+    rng = np.random.default_rng(1)
+    heads = [0, H - 1] + sorted(rng.choice(np.arange(1, H - 1), 2, replace=False).tolist())
+    hq, hk, hv, hg = (host64(x[0, heads]) for x in (q, k, v, do))
+    ref = grads_via_recurrent(oracle._get(), hq, hk, hv, hg)
+    for got, r in zip((dq, dk, dv), ref):
+        assert per_head_rel_err(host64(got[0, heads]), r) <= TOL_O_BF16

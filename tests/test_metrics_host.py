@@ -3,7 +3,8 @@
 is not hidden by a long sequence's larger outputs."""
 import numpy as np
 
-from _util import per_head_rel_err, per_seq_head_rel_err
+import oracle
+from _util import grads_via_recurrent, per_head_rel_err, per_seq_head_rel_err
 
 
 def test_packed_metric_normalises_each_sequence_by_its_own_scale():
@@ -35,3 +36,15 @@ def test_packed_metric_is_the_dense_metric_for_one_sequence():
     got = ref + 1e-3 * rng.standard_normal(ref.shape)
     cu = np.array([0, 17])
     assert per_seq_head_rel_err(got, ref, cu) == per_head_rel_err(got, ref)
+
+
+def test_recurrent_gradient_reference_equals_the_oracle_backward():
+    # the long-sequence gradient reference of the GPU tests: three recurrent
+    # forms (two on reversed tokens) equal the oracle's backward, which is
+    # pinned by finite differences
+    rng = np.random.default_rng(8)
+    q, k, v, do = (rng.standard_normal((2, 3, 37, 8)) for _ in range(4))
+    ref = oracle.prefill_backward(q, k, v, do)
+    got = grads_via_recurrent(oracle._get(), q, k, v, do)
+    for g, r in zip(got, ref):
+        np.testing.assert_allclose(g, r, rtol=0, atol=1e-11)
