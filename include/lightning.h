@@ -91,8 +91,9 @@ int la_prefill(const void* q, const void* k, const void* v, void* o, float* stat
                                   default): each chunk publishes its inclusive
                                   state prefix for the next one              */
 #define LA_FLAG_SPLIT_V    4   /* split the value columns of every head over two
-                                  CTAs (independent halves of S and O); blk 128
-                                  only, ignored with blk 64                    */
+                                  CTAs (independent halves of S and O); with
+                                  blk 64 only where each sequence is one chunk
+                                  (otherwise whole rows are kept)             */
 #define LA_FLAG_NO_SPLIT_V 8   /* never split the value columns               */
 int la_prefill_ex(const void* q, const void* k, const void* v, void* o, float* state_out,
                   int B, int H, int N, int d, int blk, la_dtype dt, void* stream,
@@ -121,7 +122,7 @@ int la_prefill_varlen(const void* q, const void* k, const void* v, void* o, floa
  *                 0 = library choice (ignored by LA_FLAG_SPLIT_V).
  *   flags: 0 = default; LA_FLAG_THREE_PASS or LA_FLAG_FUSED pick a chunked
  *          schedule over whole value rows (optionally with LA_FLAG_NO_SPLIT_V);
- *          LA_FLAG_SPLIT_V (alone; bf16, blk 128) runs every (sequence, head)
+ *          LA_FLAG_SPLIT_V (alone; bf16, blk 128 or 64) runs every (sequence, head)
  *          unchunked with its value columns split over two CTAs, longest
  *          sequences first.  Other combinations return LA_ERR_INVALID_ARG.
  */
@@ -313,8 +314,9 @@ const char* la_kernel_name(int kernel_id);
  * Name of the kernel the most recent bf16 prefill call (from any thread)
  * launched for its output pass: "prefill_tc_kernel<128>" (whole value rows,
  * chain warps), "prefill_tc_kernel<64>" (value columns split over two CTAs,
- * single pass with look-back), "prefill_tc_kernel<128,64>" (64-token blocks)
- * or "prefill_seq_kernel" (value columns split, no look-back); "" before the
+ * single pass with look-back), "prefill_tc_kernel<128,64>" (64-token blocks,
+ * whole value rows), "prefill_seq_kernel" (value columns split, no look-back)
+ * or "prefill_seq64_kernel" (the same with 64-token blocks); "" before the
  * first call.  Informational: a static string, never freed.
  */
 const char* la_prefill_main_kernel(void);

@@ -103,6 +103,8 @@ int device_setup(int* dev_out, int* sms_out) {
                                  tc::sq::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(tc::prefill_seq_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tc::sq::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(tc::prefill_seq64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::sq64::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(tc::chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tc::cs::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(simt::prefill_simt_kernel<64>,
@@ -276,13 +278,17 @@ int choose_chunk_tokens(int BH, int N, int ctas) {
 }
 
 // Main kernel for p.vparts value parts per head (1: 128 columns per CTA, 2: 64).
-// Split value columns without a look-back chain run the sequential kernel
-// with the fully double-buffered block pipeline; 64-token blocks run the
-// 128-column kernel with two blocks per tile.
+// Split value columns without a look-back chain run the sequential kernels
+// with the fully double-buffered block pipeline (prefill_seq64_kernel for
+// 64-token blocks); otherwise 64-token blocks run the 128-column kernel with
+// two blocks per tile.
 std::atomic<const char*> g_main_kernel{""};
 
 void launch_main(const tc::TileMaps& m, const tc::Params& p, int grid, cudaStream_t stream) {
-    if (p.blk == 64) {
+    if (p.blk == 64 && p.vparts == 2 && !p.fused) {
+        g_main_kernel = "prefill_seq64_kernel";
+        tc::prefill_seq64_kernel<<<grid, tc::sq64::kThreads, tc::sq64::kSmemBytes, stream>>>(m, p);
+    } else if (p.blk == 64) {
         g_main_kernel = "prefill_tc_kernel<128,64>";
         tc::prefill_tc_kernel<128, 64><<<grid, tc::kThreads, tc::smem_bytes(128), stream>>>(m, p);
     } else if (p.vparts == 2 && !p.fused) {
@@ -451,11 +457,18 @@ int launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, fl
     tc::TileMaps m;
     if (make_tile_maps(&m, q, k, v, o, N, BH)) return LA_ERR_CUDA;
     const bool three_pass = (flags & LA_FLAG_THREE_PASS) != 0;
-    // 64-token blocks keep all 128 value columns in one CTA
-    const int vparts = (blk == 128 && want_split_v(BH, N, sms, flags)) ? 2 : 1;
+    int vparts = want_split_v(BH, N, sms, flags) ? 2 : 1;
     if (!three_pass) {
+        const int asked = chunk_tokens;
         if (chunk_tokens <= 0) chunk_tokens = choose_fused_chunk_tokens(BH * vparts, N, sms);
         chunk_tokens = ((chunk_tokens + kTileRows - 1) / kTileRows) * kTileRows;
+        if (blk == 64 && vparts == 2 && chunk_tokens < N) {
+            // 64-token blocks split the value columns only in the sequential
+            // kernel (one chunk per sequence); chunked, they keep whole rows
+            vparts = 1;
+            chunk_tokens = asked > 0 ? asked : choose_fused_chunk_tokens(BH, N, sms);
+            chunk_tokens = ((chunk_tokens + kTileRows - 1) / kTileRows) * kTileRows;
+        }
         tc::Params p = dense_params(BH, N, chunk_tokens, o);
         p.vparts = vparts;
         p.blk = blk;
@@ -518,7 +531,7 @@ int choose_varlen_chunk_tokens(int H, int T, int ctas) {
 // sequences first, run by the sequential kernel.  Nothing is read twice.
 int launch_prefill_varlen_split(const void* q, const void* k, const void* v, void* o,
                                 float* state_out, const int32_t* cu_seqlens, int num_seqs, int T,
-                                int H, cudaStream_t stream, int sms, const float* state_in) {
+                                int H, int blk, cudaStream_t stream, int sms, const float* state_in) {
     const long max_items = (long)num_seqs * H * 2;
     if (max_items > (1L << 30)) return LA_ERR_UNSUPPORTED;
     tc::TileMaps m;
@@ -547,7 +560,7 @@ int launch_prefill_varlen_split(const void* q, const void* k, const void* v, voi
     std::memset(&p, 0, sizeof(p));
     p.mode = tc::kModeVarlen;
     p.vparts = 2;
-    p.blk = 128;
+    p.blk = blk;
     p.Z = H;
     p.rows = rows;
     p.chunk_tokens = chunk_tokens;
@@ -866,9 +879,9 @@ int varlen_impl(const void* q, const void* k, const void* v, void* o, const floa
     st = device_setup(&dev, &sms);
     if (st != LA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (dt == LA_BF16 && blk == 128 && (flags & LA_FLAG_SPLIT_V))
+    if (dt == LA_BF16 && (flags & LA_FLAG_SPLIT_V))
         return launch_prefill_varlen_split(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens,
-                                           H, s, sms, state_in);
+                                           H, blk, s, sms, state_in);
     if (dt == LA_BF16)
         return launch_prefill_varlen_bf16(q, k, v, o, state_out, cu_seqlens, num_seqs, total_tokens,
                                           H, blk, s, sms, (flags & LA_FLAG_THREE_PASS) != 0,

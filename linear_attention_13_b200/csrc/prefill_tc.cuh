@@ -1468,6 +1468,480 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
 }
 
 // ============================================================================
+// Sequential kernel for split value columns (64 per CTA) with 64-token blocks.
+//
+// Each 128-row tile is processed as two 64-token blocks h = 0, 1 (rows
+// [64 h, 64 h + 64)):
+//     O_h = Q_h S̄_{h-1} + tril(Q_h K_h^T)^bf16 V_h          (M = 64 MMAs)
+//     S_h = S_{h-1} + K_h^T V_h                               (M = 128, K = 64)
+// so the state is updated, and rounded to bf16 for the inter-block product,
+// every 64 tokens.  The M = 64 accumulators (scores / P, O) hold row m in TMEM
+// lane 32 (m / 16) + m % 16: lanes 0-15 of each 32-lane sub-partition.
+// A block takes 8 (Q K^T) + 8 (Q S̄) + 4 (K^T V) + 4 (P V) MMA instructions,
+// 48 per tile.  One issuing thread's MMAs complete one after another, about
+// 175 cycles each whatever their shape (B200), while the MMAs of different
+// issuing threads overlap, so four warps issue them: A the scores (MMA1), B
+// the inter-block products (MMA3), C P V (MMA2) and D the state increments
+// (MMA4).  D depends on nothing but the loads, so the state chain (dS -> S̄
+// -> Q S̄) never waits behind a P V that waits for Q S̄.
+// Every buffer is indexed by the block's position h in its tile and each of
+// its barriers completes once per tile, so phase parity = tile & 1.
+// TMEM: scores / P 2 x 64, O 2 x 64 (M = 64 layout), dS 2 x 64 columns.
+// Shared memory: two stages of Q, K, V (64 columns), O staging, and three
+// S̄ buffers of 16 KiB: block j reads S̄ buffer j mod 3.  The state step of
+// block j writes buffer (j + 1) mod 3, last read by Q S̄ of block j - 2, whose
+// output the epilogue has already drained, so that step never waits for an
+// MMA.
+// ============================================================================
+namespace sq64 {
+constexpr int kNV = 64;
+constexpr int kStageB = 2 * kTileBytes + kHalfBytes;        // 80 KiB
+constexpr int kSbarOff = kStages * kStageB;             // S̄[3]
+constexpr int kOstOff = kSbarOff + 3 * kHalfBytes;
+constexpr int kCtrlOff = kOstOff + kHalfBytes;
+constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
+constexpr uint32_t kColSP = 0;      // scores / P: 2 x 64
+constexpr uint32_t kColO = 128;     // output: 2 x 64
+constexpr uint32_t kColDS = 256;    // state increment: 2 x 64
+constexpr uint32_t kTmemCols = 512;
+constexpr int kEpiWarps = 8;
+constexpr int kStoreWarp = 2 + kEpiWarps;   // TMA stores of the staged O tiles
+constexpr int kMmaBWarp = 3 + kEpiWarps;    // issuer B: Q S̄
+constexpr int kMmaCWarp = 4 + kEpiWarps;    // issuer C: P V
+constexpr int kMmaDWarp = 5 + kEpiWarps;    // issuer D: K^T V
+constexpr int kThreads = 32 * (6 + kEpiWarps);
+constexpr int kL2Ahead = 2;
+constexpr uint32_t kRowOff = 64 * 128;      // row 64 of a 128B-swizzled 64-column half
+
+// Column, within a scores buffer, of the bf16 P pairs for keys [16 kk, 16 kk +
+// 16): the warp that converts keys [32 w, 32 w + 32) packs them into the first
+// 16 of the 32 columns it read.
+__host__ __device__ constexpr uint32_t p_col(int kk) { return kk < 2 ? kk * 8 : 32 + (kk - 2) * 8; }
+
+struct Ctrl {
+    uint64_t full_qk[kStages];  // Q and K of stage s landed
+    uint64_t full_v[kStages];   // V of stage s landed (packed tails: foreign rows cleared)
+    uint64_t empty[kStages];    // Q and K slots read: one commit each from A, B and D
+    uint64_t v_empty[kStages];  // V slot read: one commit each from C and D
+    uint64_t tail_ld;
+    uint64_t s_full[2];     // MMA1 of block h complete
+    uint64_t p_ready[2];    // P of block h written (8 warps)
+    uint64_t pv_done[2];    // MMA2 of block h complete: P consumed, O final
+    uint64_t ds_full[2];    // MMA4 of block h complete
+    uint64_t ds_free[2];    // dS of block h read (8 warps)
+    uint64_t mma3_done[2];  // MMA3 of block h complete (or none needed)
+    uint64_t sbar_ready[2]; // S̄ read by block h written (8 warps)
+    uint64_t o_free[2];     // O of block h read (8 warps)
+    uint64_t o_staged;      // both blocks of a tile staged (8 warps)
+    uint64_t ost_free;      // the staging buffer has been read by its TMA store
+    uint64_t drain;         // teardown: every MMA of the four issuers complete
+    uint32_t tmem_base;
+    int abort;
+};
+static_assert(sizeof(Ctrl) <= 512, "control block");
+}  // namespace sq64
+
+__global__ void __launch_bounds__(sq64::kThreads, 1)
+prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
+                     const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    sq64::Ctrl* ctrl = reinterpret_cast<sq64::Ctrl*>(smem + sq64::kCtrlOff);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t sbase = ptx::smem_u32(smem);
+    const uint32_t sSbar = sbase + sq64::kSbarOff;
+    auto bar = [&](uint64_t& b) { return ptx::smem_u32(&b); };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(bar(ctrl->full_qk[s]), 1);
+            ptx::mbar_init(bar(ctrl->full_v[s]), 1);
+            ptx::mbar_init(bar(ctrl->empty[s]), 3);
+            ptx::mbar_init(bar(ctrl->v_empty[s]), 2);
+        }
+        ptx::mbar_init(bar(ctrl->tail_ld), 1);
+        ptx::mbar_init(bar(ctrl->o_staged), sq64::kEpiWarps);
+        ptx::mbar_init(bar(ctrl->ost_free), 1);
+        ptx::mbar_init(bar(ctrl->drain), 4);
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(bar(ctrl->s_full[b]), 1);
+            ptx::mbar_init(bar(ctrl->p_ready[b]), sq64::kEpiWarps);
+            ptx::mbar_init(bar(ctrl->pv_done[b]), 1);
+            ptx::mbar_init(bar(ctrl->ds_full[b]), 1);
+            ptx::mbar_init(bar(ctrl->ds_free[b]), sq64::kEpiWarps);
+            ptx::mbar_init(bar(ctrl->mma3_done[b]), 1);
+            ptx::mbar_init(bar(ctrl->sbar_ready[b]), sq64::kEpiWarps);
+            ptx::mbar_init(bar(ctrl->o_free[b]), sq64::kEpiWarps);
+        }
+        ctrl->abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(ptx::smem_u32(&ctrl->tmem_base), sq64::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&maps.q);
+        ptx::prefetch_tmap(&maps.k);
+        ptx::prefetch_tmap(&maps.v_half);
+        ptx::prefetch_tmap(&maps.o);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = ctrl->tmem_base;
+    volatile int* abort_flag = &ctrl->abort;
+    const int n_items = num_items(p);
+    const bool packed = p.mode == kModeVarlen;
+    const int stride = gridDim.x;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        const uint64_t pol_qk = ptx::policy_evict_normal();   // shared with the other half
+        const uint64_t pol_v = ptx::policy_evict_first();
+        uint32_t g = 0, n_tail = 0;
+        bool ok = true;
+        // the last loads issued into each stage, barrier and phase parity, to let
+        // them land after an abort
+        uint32_t ld_qk0 = 0, ld_qk1 = 0, ld_v0 = 0, ld_v1 = 0;
+        uint32_t par_qk0 = 0, par_qk1 = 0, par_v0 = 0, par_v1 = 0;
+        auto prefetch = [&](const Item& it, int t, int ahead) {
+            const int tp = t + ahead * kTileRows;
+            if (lane == 0 && tp < it.t1) {
+                ptx::tma_prefetch_4d(&maps.q, 0, tp, 0, it.z);
+                ptx::tma_prefetch_4d(&maps.k, 0, tp, 0, it.z);
+                ptx::tma_prefetch_3d(&maps.v_half, it.vp * sq64::kNV, tp, it.z);
+            }
+        };
+        for (int item = blockIdx.x; ok && item < n_items; item += stride) {
+            const Item it = get_item(p, item);
+            for (int j = 1; j < sq64::kL2Ahead; ++j) prefetch(it, it.t0, j);
+            for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
+                const int s = g & 1;
+                const uint32_t stage = sbase + s * sq64::kStageB;
+                prefetch(it, t, sq64::kL2Ahead);
+                const bool tail = packed && it.t1 - t < kTileRows;
+                const uint32_t fv = tail ? bar(ctrl->tail_ld) : bar(ctrl->full_v[s]);
+                int w = 1;
+                if (lane == 0) {
+                    if (g >= 2) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
+                    if (w) {
+                        const uint32_t fqk = bar(ctrl->full_qk[s]);
+                        ptx::mbar_arrive_expect_tx(fqk, 2 * kTileBytes);
+                        ptx::tma_load_4d(stage, &maps.q, fqk, 0, t, 0, it.z, pol_qk);
+                        ptx::tma_load_4d(stage + kTileBytes, &maps.k, fqk, 0, t, 0, it.z, pol_qk);
+                        if (s) { ld_qk1 = fqk; par_qk1 = (g >> 1) & 1; }
+                        else   { ld_qk0 = fqk; par_qk0 = (g >> 1) & 1; }
+                        if (g >= 2) w = ptx::mbar_wait(bar(ctrl->v_empty[s]), ((g >> 1) + 1) & 1, abort_flag);
+                        if (w) {
+                            ptx::mbar_arrive_expect_tx(fv, kHalfBytes);
+                            ptx::tma_load_3d(stage + 2 * kTileBytes, &maps.v_half, fv, it.vp * sq64::kNV, t, it.z, pol_v);
+                            const uint32_t pv = tail ? (n_tail & 1) : ((g >> 1) & 1);
+                            if (s) { ld_v1 = fv; par_v1 = pv; }
+                            else   { ld_v0 = fv; par_v0 = pv; }
+                        }
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+                if (tail) {
+                    if (lane == 0) w = ptx::mbar_wait(bar(ctrl->tail_ld), n_tail & 1, abort_flag);
+                    ++n_tail;
+                    if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+                    zero_tail_rows(smem + s * sq64::kStageB + 2 * kTileBytes, it.t1 - t, lane, 1);
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->full_v[s]));
+                }
+            }
+        }
+        if (lane == 0) {
+            for (uint32_t j = (g >= 2 ? g - 2 : 0); ok && j < g; ++j) {
+                ok = ptx::mbar_wait(bar(ctrl->empty[j & 1]), (j >> 1) & 1, abort_flag);
+                if (ok) ok = ptx::mbar_wait(bar(ctrl->v_empty[j & 1]), (j >> 1) & 1, abort_flag);
+            }
+            if (!ok) {
+                // after an abort: let the loads already issued land (bounded)
+                if (ld_qk0) ptx::mbar_drain(ld_qk0, par_qk0);
+                if (ld_qk1) ptx::mbar_drain(ld_qk1, par_qk1);
+                if (ld_v0) ptx::mbar_drain(ld_v0, par_v0);
+                if (ld_v1) ptx::mbar_drain(ld_v1, par_v1);
+            }
+        }
+    } else if (warp == 1 || warp == sq64::kMmaBWarp || warp == sq64::kMmaCWarp || warp == sq64::kMmaDWarp) {
+        // ------------------------------------------------------------ MMA issuers
+        if (lane == 0) {
+            constexpr uint32_t id_qk = ptx::idesc_bf16(64, 64, false, false);        // Q_h K_h^T
+            constexpr uint32_t id_qs = ptx::idesc_bf16(64, sq64::kNV, false, true);  // Q_h S̄
+            constexpr uint32_t id_kv = ptx::idesc_bf16(128, sq64::kNV, true, true);  // K_h^T V_h
+            constexpr uint32_t id_pv = ptx::idesc_bf16(64, sq64::kNV, false, true);  // P_h V_h
+            const int role = warp == 1 ? 0 : warp == sq64::kMmaBWarp ? 1 : warp == sq64::kMmaCWarp ? 2 : 3;
+            uint32_t g = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < n_items; item += stride) {
+                const Item it = get_item(p, item);
+                bool has_state = start_state(p, it) != nullptr;
+                for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
+                    const int s = g & 1;
+                    const uint32_t tp = g & 1;        // this tile's phase of the block barriers
+                    const uint32_t pp = tp ^ 1u;      // the previous tile's
+                    if (!ptx::mbar_wait(bar(ctrl->full_qk[s]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
+                    if (role >= 2 && !ptx::mbar_wait(bar(ctrl->full_v[s]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t sq_ = sbase + s * sq64::kStageB;
+                    const uint32_t sk = sq_ + kTileBytes;
+                    const uint32_t sv = sq_ + 2 * kTileBytes;
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t roff = h * sq64::kRowOff;
+                        if (role == 0) {
+                            // MMA1: scores_h = Q_h K_h^T, once MMA2 of block h of the
+                            // previous tile has consumed the P in buffer h
+                            if (g >= 1 && !ptx::mbar_wait(bar(ctrl->pv_done[h]), pp, abort_flag)) { ok = false; break; }
+                            ptx::tc_fence_after();
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32 + roff;
+                                ptx::mma_ss(tmem + sq64::kColSP + h * 64, ptx::sdesc_sw128(sq_ + off, 16, 1024),
+                                            ptx::sdesc_sw128(sk + off, 16, 1024), id_qk, kk > 0);
+                            }
+                            ptx::mma_commit(bar(ctrl->s_full[h]));
+                        } else if (role == 1) {
+                            // MMA3: O_h = Q_h S̄ (S̄ buffer (2 g + h) mod 3), once that S̄
+                            // is written and block h of the previous tile has been drained
+                            if (!ptx::mbar_wait(bar(ctrl->sbar_ready[h]), tp, abort_flag)) { ok = false; break; }
+                            if (g >= 1 && !ptx::mbar_wait(bar(ctrl->o_free[h]), pp, abort_flag)) { ok = false; break; }
+                            ptx::tc_fence_after();
+                            if (has_state) {
+                                const uint32_t sb = sSbar + ((2 * g + h) % 3) * kHalfBytes;
+#pragma unroll
+                                for (int kk = 0; kk < 8; ++kk) {
+                                    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32 + roff;
+                                    ptx::mma_ss(tmem + sq64::kColO + h * 64, ptx::sdesc_sw128(sq_ + off, 16, 1024),
+                                                ptx::sdesc_sw128(sb + kk * 2048, kHalfBytes, 1024), id_qs, kk > 0);
+                                }
+                            }
+                            ptx::mma_commit(bar(ctrl->mma3_done[h]));
+                        } else if (role == 3) {
+                            // MMA4: dS_h = K_h^T V_h, once dS buffer h has been read
+                            if (g >= 1 && !ptx::mbar_wait(bar(ctrl->ds_free[h]), pp, abort_flag)) { ok = false; break; }
+                            ptx::tc_fence_after();
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                ptx::mma_ss(tmem + sq64::kColDS + h * 64,
+                                            ptx::sdesc_sw128(sk + roff + kk * 2048, kHalfBytes, 1024),
+                                            ptx::sdesc_sw128(sv + roff + kk * 2048, kHalfBytes, 1024), id_kv, kk > 0);
+                            ptx::mma_commit(bar(ctrl->ds_full[h]));
+                        } else {
+                            // MMA2: O_h += P_h V_h (P from TMEM), after MMA3 wrote O_h
+                            if (!ptx::mbar_wait(bar(ctrl->p_ready[h]), tp, abort_flag)) { ok = false; break; }
+                            if (!ptx::mbar_wait(bar(ctrl->mma3_done[h]), tp, abort_flag)) { ok = false; break; }
+                            ptx::tc_fence_after();
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                ptx::mma_ts(tmem + sq64::kColO + h * 64, tmem + sq64::kColSP + h * 64 + sq64::p_col(kk),
+                                            ptx::sdesc_sw128(sv + roff + kk * 2048, kHalfBytes, 1024), id_pv,
+                                            (kk > 0 || has_state) ? 1u : 0u);
+                            ptx::mma_commit(bar(ctrl->pv_done[h]));
+                            if (h == 1) ptx::mma_commit(bar(ctrl->v_empty[s]));  // V read
+                        }
+                        has_state = true;
+                    }
+                    if (!ok) break;
+                    if (role != 2) ptx::mma_commit(bar(ctrl->empty[s]));     // Q and K read
+                    if (role == 3) ptx::mma_commit(bar(ctrl->v_empty[s]));   // V read by MMA4
+                }
+            }
+            // teardown: every MMA the three issuers issued has completed
+            ptx::mma_commit(bar(ctrl->drain));
+            ptx::mbar_drain(bar(ctrl->drain), 0);
+        }
+    } else if (warp == sq64::kStoreWarp) {
+        // ------------------------------------------------------------ O stores
+        if (lane == 0) {
+            uint32_t g = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < n_items; item += stride) {
+                const Item it = get_item(p, item);
+                for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
+                    if (!ptx::mbar_wait(bar(ctrl->o_staged), g & 1, abort_flag)) { ok = false; break; }
+                    if (!(packed && t + kTileRows > it.t1)) {
+                        ptx::tma_store_3d(&maps.o, sbase + sq64::kOstOff, it.vp * sq64::kNV, t, it.z);
+                        ptx::bulk_commit_group();
+                        ptx::bulk_wait_group_read0();
+                    }
+                    ptx::mbar_arrive(bar(ctrl->ost_free));
+                }
+            }
+            ptx::bulk_wait_group0();
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        // Per block (g, h): P, then S += dS and S̄ for the next block, then the
+        // output of the previous block.
+        const int ew = warp - 2;             // 0..7
+        const int sp = warp & 3;             // TMEM sub-partition of this warp
+        const int r = sp * 32 + lane;        // state row (key dimension) of this thread
+        const int c0 = 32 * (ew >> 2);       // keys [c0, c0 + 32) of P; value columns
+                                             // [c0, c0 + 32) of S and O (of this CTA's 64)
+        const int br = 16 * sp + lane;       // row of a 64-token block (lanes 0-15)
+        const bool row_ok = lane < 16;
+        const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
+        uint8_t* ostage = smem + sq64::kOstOff;
+        uint32_t g = 0;
+        bool ok = true;
+        bool o_pending = false;
+        Item o_it;
+        int o_t = 0, o_h = 0;
+        uint32_t o_g = 0;
+        // ---- O of block (og, oh): registers, release its buffer, stage as bf16
+        //      (the tile's staging buffer once the previous tile has been stored)
+        auto drain_o = [&](const Item& oit, int ot, uint32_t og, int oh) -> bool {
+            if (!ptx::mbar_wait(bar(ctrl->pv_done[oh]), og & 1, abort_flag)) return false;
+            ptx::tc_fence_after();
+            const bool rowwise = packed && ot + kTileRows > oit.t1;
+            uint32_t v[32];
+            ptx::tmem_ld32(tl + sq64::kColO + oh * 64 + c0, v);
+            ptx::tmem_ld_wait();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(ctrl->o_free[oh]));
+            if (oh == 0 && og >= 1 && !ptx::mbar_wait(bar(ctrl->ost_free), (og - 1) & 1, abort_flag)) return false;
+            const int trow = 64 * oh + br;
+            if (!rowwise) {
+                if (row_ok) store_row32_bf16_sw128(ostage, trow, c0, v);
+                ptx::fence_proxy_async_smem();
+            } else if (row_ok && ot + trow < oit.t1) {
+                uint4* orow = reinterpret_cast<uint4*>(
+                    p.o + ((size_t)oit.z * p.rows + ot + trow) * kHeadDim + oit.vp * sq64::kNV + c0);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint4 w;
+                    w.x = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+                    w.y = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+                    w.z = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+                    w.w = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+                    orow[j] = w;
+                }
+            }
+            __syncwarp();
+            if (oh == 1 && lane == 0) ptx::mbar_arrive(bar(ctrl->o_staged));
+            return true;
+        };
+        for (int item = blockIdx.x; ok && item < n_items; item += stride) {
+            const Item it = get_item(p, item);
+            const int vcol = it.vp * sq64::kNV + c0;   // first owned column of the 128
+            // ---- running state S (row r, columns vcol..vcol+31) and the S̄ of the
+            //      item's first block 2 g (buffer 2 g mod 3, last read by MMA3 of
+            //      block 2 g - 3, drained before)
+            float srun[32];
+            if (const float* st0 = start_state(p, it)) {
+                const float4* src = reinterpret_cast<const float4*>(st0 + (size_t)r * kHeadDim + vcol);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 x = __ldg(src + j);
+                    srun[4 * j + 0] = x.x;
+                    srun[4 * j + 1] = x.y;
+                    srun[4 * j + 2] = x.z;
+                    srun[4 * j + 3] = x.w;
+                }
+                uint32_t f[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
+                store_row32_bf16_sw128(smem + sq64::kSbarOff + ((2 * g) % 3) * kHalfBytes, r, c0, f);
+                ptx::fence_proxy_async_smem();
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) srun[j] = 0.f;
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready[0]));
+
+            for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
+                const bool last_tile = t + kTileRows >= it.t1;
+                const uint32_t tp = g & 1;
+                for (int h = 0; h < 2; ++h) {
+                    // ---- 1. P_h = tril(scores_h) as bf16 pairs, in place
+                    if (!ptx::mbar_wait(bar(ctrl->s_full[h]), tp, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    {
+                        const uint32_t scol = tl + sq64::kColSP + h * 64 + c0;
+                        uint32_t pk[16];
+                        if (c0 > 16 * sp + 15) {
+                            // every key of this half lies above the diagonal for these rows
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                        } else {
+                            uint32_t v[32];
+                            ptx::tmem_ld32(scol, v);
+                            ptx::tmem_ld_wait();
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const int key = c0 + 2 * j;
+                                const float a = (key <= br) ? __uint_as_float(v[2 * j]) : 0.0f;
+                                const float b = (key + 1 <= br) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
+                                pk[j] = ptx::pack_bf16x2(a, b);
+                            }
+                        }
+                        ptx::tmem_st16(scol, pk);
+                    }
+                    ptx::tmem_st_wait();
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->p_ready[h]));
+
+                    // ---- 2. S += dS_h; S̄ for the next block, or the final state
+                    if (!ptx::mbar_wait(bar(ctrl->ds_full[h]), tp, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    {
+                        uint32_t d[32];
+                        ptx::tmem_ld32(tl + sq64::kColDS + h * 64 + c0, d);
+                        ptx::tmem_ld_wait();
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(bar(ctrl->ds_free[h]));
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) srun[j] += __uint_as_float(d[j]);
+                    }
+                    if (!(last_tile && h == 1)) {
+                        // S̄ for block j + 1 = 2 g + h + 1: buffer (j + 1) mod 3, last read
+                        // by MMA3 of block j - 2.  That MMA has completed: C issued P V of
+                        // block j - 2 only after it, and this warp has drained that output.
+                        uint32_t f[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
+                        store_row32_bf16_sw128(smem + sq64::kSbarOff + ((2 * g + h + 1) % 3) * kHalfBytes, r, c0, f);
+                        ptx::fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready[h ^ 1]));
+                    } else if (p.state_out != nullptr) {
+                        float4* dst = reinterpret_cast<float4*>(
+                            p.state_out + (size_t)it.sidx * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim + vcol);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            dst[j] = make_float4(srun[4 * j], srun[4 * j + 1], srun[4 * j + 2], srun[4 * j + 3]);
+                    }
+
+                    // ---- 3. the previous block's output
+                    if (o_pending && !drain_o(o_it, o_t, o_g, o_h)) { ok = false; break; }
+                    o_pending = true;
+                    o_it = it;
+                    o_t = t;
+                    o_g = g;
+                    o_h = h;
+                }
+            }
+        }
+        if (ok && o_pending) drain_o(o_it, o_t, o_g, o_h);
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, sq64::kTmemCols);
+    }
+}
+
+// ============================================================================
 // Pass 1: per-chunk state increment  ΔS_c = K_c^T V_c.
 // ============================================================================
 namespace cs {

@@ -126,12 +126,17 @@ def test_bf16_long_context_sampled_heads(flags):
 
 
 # ---------------------------------------------------------------- 64-token blocks
-# blk = 64 runs each 128-row tile as two blocks of 64 tokens (M = 64 MMAs); the
-# split-value flags do not apply and are ignored.
+# blk = 64 runs each 128-row tile as two blocks of 64 tokens (M = 64 MMAs):
+# with the value columns split (prefill_seq64_kernel) when every sequence is
+# one chunk or in the three-pass output pass, otherwise with whole value rows
+# (prefill_tc_kernel<128,64>).
 SCHEDULES_64 = [
     pytest.param(0, id="default"),
     pytest.param(la.LA_FLAG_FUSED, id="single-pass"),
     pytest.param(la.LA_FLAG_THREE_PASS, id="three-pass"),
+    pytest.param(la.LA_FLAG_SPLIT_V, id="split-v"),
+    pytest.param(la.LA_FLAG_NO_SPLIT_V, id="whole-rows"),
+    pytest.param(la.LA_FLAG_THREE_PASS | la.LA_FLAG_SPLIT_V, id="three-pass-splitv"),
 ]
 
 
@@ -179,11 +184,29 @@ def test_bf16_blk64_onehot_long_bit_exact(chunk, flags):
     assert np.array_equal(host64(st), s_ref)
 
 
-def test_bf16_blk64_split_flags_ignored():
+def test_bf16_blk64_split_flag_ignored_when_chunked():
+    # chunked single pass keeps whole value rows at blk 64
     q, k, v = inputs.qkv((1, 2, 700, 128), dtype=torch.bfloat16, device=DEV, seed=8)
     o1, s1 = _run(q, k, v, 64, chunk_tokens=256, flags=la.LA_FLAG_FUSED)
     o2, s2 = _run(q, k, v, 64, chunk_tokens=256, flags=la.LA_FLAG_FUSED | la.LA_FLAG_SPLIT_V)
+    assert la.la_prefill_main_kernel() == "prefill_tc_kernel<128,64>"
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+@pytest.mark.parametrize("flags,kernel", [
+    (0, "prefill_seq64_kernel"),
+    (la.LA_FLAG_NO_SPLIT_V, "prefill_tc_kernel<128,64>"),
+    (la.LA_FLAG_THREE_PASS | la.LA_FLAG_SPLIT_V, "prefill_seq64_kernel"),
+], ids=["default", "whole-rows", "three-pass-splitv"])
+def test_bf16_blk64_kernels_agree_with_the_oracle(flags, kernel):
+    # the two 64-token-block kernels on B4 H16 N8192 (every head): each within
+    # the bar, and each is the kernel the dispatch names
+    q, k, v = inputs.qkv((4, 16, 8192, 128), dtype=torch.bfloat16, device=DEV, seed=3)
+    o, st = _run(q, k, v, 64, flags=flags)
+    assert la.la_prefill_main_kernel() == kernel
+    o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16
+    assert per_head_rel_err(host64(st), s_ref) <= TOL_STATE
 
 
 def test_bf16_scaling_is_exact():

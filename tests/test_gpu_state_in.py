@@ -25,6 +25,8 @@ SCHEDULES = [
     pytest.param(la.LA_FLAG_THREE_PASS | la.LA_FLAG_SPLIT_V, 128, id="three-pass-splitv"),
     pytest.param(0, 64, id="blk64"),
     pytest.param(la.LA_FLAG_THREE_PASS, 64, id="blk64-three-pass"),
+    pytest.param(la.LA_FLAG_SPLIT_V, 64, id="blk64-splitv"),
+    pytest.param(la.LA_FLAG_FUSED | la.LA_FLAG_NO_SPLIT_V, 64, id="blk64-whole-rows"),
 ]
 
 
@@ -134,6 +136,7 @@ VARLEN_SCHEDULES = [
     pytest.param(la.LA_FLAG_THREE_PASS, 128, id="three-pass"),
     pytest.param(la.LA_FLAG_SPLIT_V, 128, id="split-v"),
     pytest.param(0, 64, id="blk64"),
+    pytest.param(la.LA_FLAG_SPLIT_V, 64, id="blk64-split-v"),
 ]
 
 

@@ -101,7 +101,8 @@ def test_varlen_bf16_onehot_bit_exact(chunk, flags, blk):
     [0, 0, 0, 5],
     [1] * 40 + [3000],
 ])
-def test_varlen_bf16_split_longest_first_exact(lens):
+@pytest.mark.parametrize("blk,kernel", [(128, "prefill_seq_kernel"), (64, "prefill_seq64_kernel")])
+def test_varlen_bf16_split_longest_first_exact(lens, blk, kernel):
     # split value columns, longest sequence first: every sequence and head is
     # produced exactly once with its own state (one-hot keys: exact)
     cu = _cu(lens)
@@ -109,9 +110,9 @@ def test_varlen_bf16_split_longest_first_exact(lens):
     q, k, v = inputs.onehot_k_qkv((H, T, 128), dtype=torch.bfloat16, device=DEV, seed=len(lens))
     o = torch.full_like(q, 3.0)
     st = torch.full((len(lens), H, 128, 128), 3.0, device=DEV)
-    o, st = la.prefill_varlen(q, k, v, cu, blk=128, out=o, state_out=st, flags=la.LA_FLAG_SPLIT_V)
+    o, st = la.prefill_varlen(q, k, v, cu, blk=blk, out=o, state_out=st, flags=la.LA_FLAG_SPLIT_V)
     assert la.la_get_last_error() == la.LA_OK
-    assert la.la_prefill_main_kernel() == "prefill_seq_kernel"
+    assert la.la_prefill_main_kernel() == kernel
     o_ref, s_ref = oracle.prefill_varlen(host64(q), host64(k), host64(v), cu.cpu().numpy())
     assert np.array_equal(host64(o), round_like(o_ref, torch.bfloat16))
     assert np.array_equal(host64(st), s_ref)
