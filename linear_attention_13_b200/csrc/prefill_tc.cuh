@@ -239,6 +239,22 @@ __device__ __forceinline__ void store_row32_bf16_sw128(uint8_t* tile, int row, i
     }
 }
 
+// The same for 16 values (col0 a multiple of 16).
+__device__ __forceinline__ void store_row16_bf16_sw128(uint8_t* tile, int row, int col0,
+                                                       const uint32_t* f) {
+    uint8_t* half = tile + (col0 >> 6) * kHalfBytes;
+    const int chunk0 = (col0 & 63) >> 3;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        uint4 w;
+        w.x = ptx::pack_bf16x2(__uint_as_float(f[8 * c + 0]), __uint_as_float(f[8 * c + 1]));
+        w.y = ptx::pack_bf16x2(__uint_as_float(f[8 * c + 2]), __uint_as_float(f[8 * c + 3]));
+        w.z = ptx::pack_bf16x2(__uint_as_float(f[8 * c + 4]), __uint_as_float(f[8 * c + 5]));
+        w.w = ptx::pack_bf16x2(__uint_as_float(f[8 * c + 6]), __uint_as_float(f[8 * c + 7]));
+        *reinterpret_cast<uint4*>(half + ptx::sw128_offset(row, chunk0 + c)) = w;
+    }
+}
+
 // Zero rows [valid, 128) of a V tile of `halves` 64-column halves, by one
 // warp.  Used for the last block of a packed sequence, whose trailing rows
 // belong to the next sequence: they must not enter K^T V.
@@ -1782,8 +1798,11 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
         const int r = sp * 32 + lane;        // state row (key dimension) of this thread
         const int c0 = 32 * (ew >> 2);       // keys [c0, c0 + 32) of P; value columns
                                              // [c0, c0 + 32) of S and O (of this CTA's 64)
-        const int br = 16 * sp + lane;       // row of a 64-token block (lanes 0-15)
-        const bool row_ok = lane < 16;
+        // P and O of a 64-token block (M = 64 layout, rows in lanes 0-15): thread
+        // lane takes row 16 sp + (lane & 15) and 16 of the warp's 32 columns,
+        // [c0 + 16 (lane >> 4), +16)
+        const int br = 16 * sp + (lane & 15);
+        const int cq = c0 + 16 * (lane >> 4);
         const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
         uint8_t* ostage = smem + sq64::kOstOff;
         uint32_t g = 0;
@@ -1798,8 +1817,8 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
             if (!ptx::mbar_wait(bar(ctrl->pv_done[oh]), og & 1, abort_flag)) return false;
             ptx::tc_fence_after();
             const bool rowwise = packed && ot + kTileRows > oit.t1;
-            uint32_t v[32];
-            ptx::tmem_ld32(tl + sq64::kColO + oh * 64 + c0, v);
+            uint32_t v[16];
+            ptx::tmem_ld16x2_16<16>(tl + sq64::kColO + oh * 64 + c0, v);
             ptx::tmem_ld_wait();
             ptx::tc_fence_before();
             __syncwarp();
@@ -1807,13 +1826,13 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
             if (oh == 0 && og >= 1 && !ptx::mbar_wait(bar(ctrl->ost_free), (og - 1) & 1, abort_flag)) return false;
             const int trow = 64 * oh + br;
             if (!rowwise) {
-                if (row_ok) store_row32_bf16_sw128(ostage, trow, c0, v);
+                store_row16_bf16_sw128(ostage, trow, cq, v);
                 ptx::fence_proxy_async_smem();
-            } else if (row_ok && ot + trow < oit.t1) {
+            } else if (ot + trow < oit.t1) {
                 uint4* orow = reinterpret_cast<uint4*>(
-                    p.o + ((size_t)oit.z * p.rows + ot + trow) * kHeadDim + oit.vp * sq64::kNV + c0);
+                    p.o + ((size_t)oit.z * p.rows + ot + trow) * kHeadDim + oit.vp * sq64::kNV + cq);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < 2; ++j) {
                     uint4 w;
                     w.x = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
                     w.y = ptx::pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
@@ -1863,25 +1882,27 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                     if (!ptx::mbar_wait(bar(ctrl->s_full[h]), tp, abort_flag)) { ok = false; break; }
                     ptx::tc_fence_after();
                     {
+                        // keys [cq, cq + 16) of row br; packed into columns [c0, c0 + 8)
+                        // (threads 0-15) and [c0 + 8, c0 + 16) (threads 16-31)
                         const uint32_t scol = tl + sq64::kColSP + h * 64 + c0;
-                        uint32_t pk[16];
+                        uint32_t pk[8];
                         if (c0 > 16 * sp + 15) {
-                            // every key of this half lies above the diagonal for these rows
+                            // every key of the warp's 32 lies above the diagonal for its rows
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                            for (int j = 0; j < 8; ++j) pk[j] = 0u;
                         } else {
-                            uint32_t v[32];
-                            ptx::tmem_ld32(scol, v);
+                            uint32_t v[16];
+                            ptx::tmem_ld16x2_16<16>(scol, v);
                             ptx::tmem_ld_wait();
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const int key = c0 + 2 * j;
+                            for (int j = 0; j < 8; ++j) {
+                                const int key = cq + 2 * j;
                                 const float a = (key <= br) ? __uint_as_float(v[2 * j]) : 0.0f;
                                 const float b = (key + 1 <= br) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
                                 pk[j] = ptx::pack_bf16x2(a, b);
                             }
                         }
-                        ptx::tmem_st16(scol, pk);
+                        ptx::tmem_st16x2_8<8>(scol, pk);
                     }
                     ptx::tmem_st_wait();
                     ptx::tc_fence_before();
