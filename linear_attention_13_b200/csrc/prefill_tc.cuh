@@ -1025,17 +1025,23 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
 //   * the state increment of each block, dS_i = K_i^T V_i, goes to one of two
 //     TMEM buffers; the running state S (fp32) lives in the epilogue's
 //     registers (32 values per thread), which add dS_i and write the bf16 copy
-//     S̄_i for the next block's Q S̄ into one of two shared-memory buffers;
+//     S̄_i for the next block's Q S̄ into one of three shared-memory buffers;
 //   * scores / P and the output accumulator are double-buffered in TMEM.
-// MMA order per block i: QK^T -> K^T V -> Q S̄_{i-1} -> P V.  TMEM: scores
-// 2 x 128, O 2 x 64, dS 2 x 64 columns.  Shared memory: two stages of
-// Q, K (128 x 128) and V (128 x 64), S̄ 2 x 16 KiB.
+// One issuing thread's MMAs complete one after another, about 175 cycles
+// each whatever their shape (B200), while those of different threads
+// overlap, so each product has its own issuing warp: A QK^T (MMA1), B Q S̄
+// (MMA3), C P V (MMA2), D K^T V (MMA4), 8 MMAs per block each.  Block i reads
+// S̄ buffer i mod 3; the state step of block i writes buffer (i + 1) mod 3,
+// last read by Q S̄ of block i - 2, whose output the epilogue has already
+// drained.  TMEM: scores 2 x 128, O 2 x 64, dS 2 x 64 columns.  Shared
+// memory: two stages of Q, K (128 x 128) and V (128 x 64), S̄ 3 x 16 KiB, O
+// staging 16 KiB.
 // ============================================================================
 namespace sq {
 constexpr int kNV = 64;
 constexpr int kStageB = 2 * kTileBytes + kHalfBytes;        // 80 KiB
-constexpr int kSbarOff = kStages * kStageB;                 // S̄[2], 16 KiB each
-constexpr int kOstOff = kSbarOff + 2 * kHalfBytes;          // O staging, 16 KiB
+constexpr int kSbarOff = kStages * kStageB;                 // S̄[3], 16 KiB each
+constexpr int kOstOff = kSbarOff + 3 * kHalfBytes;          // O staging, 16 KiB
 constexpr int kCtrlOff = kOstOff + kHalfBytes;
 constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
 constexpr uint32_t kColSP = 0;      // scores / P: 2 x 128
@@ -1044,15 +1050,17 @@ constexpr uint32_t kColDS = 384;    // state increment: 2 x 64
 constexpr uint32_t kTmemCols = 512;
 constexpr int kEpiWarps = 8;
 constexpr int kStoreWarp = 2 + kEpiWarps;   // TMA stores of the staged O tiles
-constexpr int kMmaBWarp = 3 + kEpiWarps;    // second MMA issuer
-constexpr int kThreads = 32 * (4 + kEpiWarps);
+constexpr int kMmaBWarp = 3 + kEpiWarps;    // issuer B: Q S̄
+constexpr int kMmaCWarp = 4 + kEpiWarps;    // issuer C: P V
+constexpr int kMmaDWarp = 5 + kEpiWarps;    // issuer D: K^T V
+constexpr int kThreads = 32 * (6 + kEpiWarps);
 constexpr int kL2Ahead = 2;                 // tiles prefetched into L2 ahead of the load
 
 struct Ctrl {
     uint64_t full_qk[kStages];  // Q and K of stage s landed (MMA1 and MMA3 need no V)
     uint64_t full_v[kStages];   // V of stage s landed (packed tails: foreign rows cleared)
-    uint64_t empty[kStages];    // Q and K slots of stage s read (MMA1, MMA3, MMA4)
-    uint64_t v_empty[kStages];  // V slot of stage s read (MMA2)
+    uint64_t empty[kStages];    // Q and K slots of stage s read (A, B, D)
+    uint64_t v_empty[kStages];  // V slot of stage s read (C, D)
     uint64_t tail_ld;
     uint64_t s_full[2];     // MMA1 complete (scores buffer b)
     uint64_t p_ready[2];    // P of block parity b written (8 warps)
@@ -1065,6 +1073,7 @@ struct Ctrl {
     uint64_t o_free[2];     // O buffer read (8 warps)
     uint64_t o_staged;      // O staged in shared memory (8 warps)
     uint64_t ost_free;      // the O staging buffer has been read by its TMA store
+    uint64_t drain;         // teardown: every MMA of the four issuers complete
     uint32_t tmem_base;
     int abort;
 };
@@ -1090,11 +1099,12 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(bar(ctrl->full_qk[s]), 1);
             ptx::mbar_init(bar(ctrl->full_v[s]), 1);
-            ptx::mbar_init(bar(ctrl->empty[s]), 2);   // one commit from each MMA issuer
-            ptx::mbar_init(bar(ctrl->v_empty[s]), 1);
+            ptx::mbar_init(bar(ctrl->empty[s]), 3);
+            ptx::mbar_init(bar(ctrl->v_empty[s]), 2);
         }
         ptx::mbar_init(bar(ctrl->ost_free), 1);
         ptx::mbar_init(bar(ctrl->tail_ld), 1);
+        ptx::mbar_init(bar(ctrl->drain), 4);
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(bar(ctrl->p_ready[b]), sq::kEpiWarps);
             ptx::mbar_init(bar(ctrl->sbar_ready[b]), sq::kEpiWarps);
@@ -1205,20 +1215,17 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 if (ok) ok = ptx::mbar_wait(bar(ctrl->v_empty[j & 1]), (j >> 1) & 1, abort_flag);
             }
         }
-    } else if (warp == 1 || warp == sq::kMmaBWarp) {
+    } else if (warp == 1 || warp == sq::kMmaBWarp || warp == sq::kMmaCWarp || warp == sq::kMmaDWarp) {
         // ------------------------------------------------------------ MMA issuers
-        // One thread issues tcgen05 MMAs at about half the tensor core's rate for
-        // these shapes, so two warps issue: A the products with Q (MMA1 scores,
-        // MMA3 inter-block), B those with V (MMA4 state increment, MMA2 P V).
-        // Every resource either one reuses is double-buffered by block parity b
-        // and guarded by a barrier of that buffer, so neither can run two blocks
-        // ahead of the other.  Both release a stage (empty[s] counts 2).
+        // A: MMA1 scores = Q K^T; B: MMA3 O = Q S̄; C: MMA2 O += P V; D: MMA4
+        // dS = K^T V.  Every resource one of them reuses is double-buffered by
+        // block parity b and guarded by a barrier of that buffer.
         if (lane == 0) {
-            const bool is_a = warp == 1;
             constexpr uint32_t id_qk = ptx::idesc_bf16(128, 128, false, false);  // Q K^T
             constexpr uint32_t id_qs = ptx::idesc_bf16(128, sq::kNV, false, true);   // Q S̄
             constexpr uint32_t id_kv = ptx::idesc_bf16(128, sq::kNV, true, true);    // K^T V
             constexpr uint32_t id_pv = ptx::idesc_bf16(128, sq::kNV, false, true);   // P V
+            const int role = warp == 1 ? 0 : warp == sq::kMmaBWarp ? 1 : warp == sq::kMmaCWarp ? 2 : 3;
             uint32_t g = 0;
             bool ok = true;
             for (int item = blockIdx.x; ok && item < n_items; item += stride) {
@@ -1229,33 +1236,32 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     const uint32_t b = g & 1;
                     const uint32_t par = (g >> 1) & 1;           // phase parity of buffer b's barriers
                     const uint32_t prev = ((g >> 1) + 1) & 1;    // ... for block g - 2
-                    if (!ptx::mbar_wait(bar(ctrl->full_qk[s]), par, abort_flag)) { ok = false; break; }
-                    if (!is_a && !ptx::mbar_wait(bar(ctrl->full_v[s]), par, abort_flag)) { ok = false; break; }
-                    ptx::tc_fence_after();
+                    if (role != 2 && !ptx::mbar_wait(bar(ctrl->full_qk[s]), par, abort_flag)) { ok = false; break; }
+                    if (role >= 2 && !ptx::mbar_wait(bar(ctrl->full_v[s]), par, abort_flag)) { ok = false; break; }
                     const uint32_t sq_ = sbase + s * sq::kStageB;
                     const uint32_t sk = sq_ + kTileBytes;
                     const uint32_t sv = sq_ + 2 * kTileBytes;
-                    const uint32_t sp_cols = tmem + sq::kColSP + b * 128;
                     const uint32_t o_cols = tmem + sq::kColO + b * sq::kNV;
-                    if (is_a) {
-                        // MMA1: scores = Q K^T into buffer b, once MMA2 of block g-2
-                        // has consumed the P there
+                    if (role == 0) {
+                        // MMA1 into scores buffer b, once MMA2 of block g-2 consumed its P
                         if (g >= 2 && !ptx::mbar_wait(bar(ctrl->p_free[b]), prev, abort_flag)) { ok = false; break; }
                         ptx::tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
                             const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                            ptx::mma_ss(sp_cols, ptx::sdesc_sw128(sq_ + off, 16, 1024),
+                            ptx::mma_ss(tmem + sq::kColSP + b * 128, ptx::sdesc_sw128(sq_ + off, 16, 1024),
                                         ptx::sdesc_sw128(sk + off, 16, 1024), id_qk, kk > 0);
                         }
                         ptx::mma_commit(bar(ctrl->s_full[b]));
-                        // MMA3: O = Q S̄_{g-1} into buffer b (S̄ buffer (g-1) & 1), once
-                        // the epilogue has read block g-2's O there
+                        ptx::mma_commit(bar(ctrl->empty[s]));
+                    } else if (role == 1) {
+                        // MMA3: O = Q S̄_{g-1} (S̄ buffer g mod 3) into O buffer b, once that
+                        // S̄ is written and the epilogue has read block g-2's O there
                         if (!ptx::mbar_wait(bar(ctrl->sbar_ready[b]), par, abort_flag)) { ok = false; break; }
                         if (g >= 2 && !ptx::mbar_wait(bar(ctrl->o_free[b]), prev, abort_flag)) { ok = false; break; }
                         ptx::tc_fence_after();
                         if (has_state) {
-                            const uint32_t sb = sSbar + ((g + 1) & 1) * kHalfBytes;
+                            const uint32_t sb = sSbar + (g % 3) * kHalfBytes;
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk) {
                                 const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
@@ -1265,19 +1271,18 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                         }
                         ptx::mma_commit(bar(ctrl->mma3_done[b]));
                         ptx::mma_commit(bar(ctrl->empty[s]));
-                    } else {
-                        // MMA4: dS = K^T V into buffer b, once block g-2's dS has been read
-                        // and this block's MMA1 has completed: MMA1 -> P -> MMA2 is the
-                        // critical chain, so MMA4 runs while the epilogue builds P
+                    } else if (role == 3) {
+                        // MMA4: dS = K^T V into dS buffer b, once block g-2's dS was read
                         if (g >= 2 && !ptx::mbar_wait(bar(ctrl->ds_free[b]), prev, abort_flag)) { ok = false; break; }
-                        if (!ptx::mbar_wait(bar(ctrl->s_full[b]), par, abort_flag)) { ok = false; break; }
                         ptx::tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
                             ptx::mma_ss(tmem + sq::kColDS + b * sq::kNV, ptx::sdesc_sw128(sk + kk * 2048, kHalfBytes, 1024),
                                         ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_kv, kk > 0);
                         ptx::mma_commit(bar(ctrl->ds_full[b]));
-                        ptx::mma_commit(bar(ctrl->empty[s]));    // K read
+                        ptx::mma_commit(bar(ctrl->empty[s]));      // K read
+                        ptx::mma_commit(bar(ctrl->v_empty[s]));    // V read by MMA4
+                    } else {
                         // MMA2: O += P V (P in TMEM buffer b), after MMA3 wrote O
                         if (!ptx::mbar_wait(bar(ctrl->p_ready[b]), par, abort_flag)) { ok = false; break; }
                         if (!ptx::mbar_wait(bar(ctrl->mma3_done[b]), par, abort_flag)) { ok = false; break; }
@@ -1289,11 +1294,14 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                                         (kk > 0 || has_state) ? 1u : 0u);
                         ptx::mma_commit(bar(ctrl->o_full[b]));
                         ptx::mma_commit(bar(ctrl->p_free[b]));
-                        ptx::mma_commit(bar(ctrl->v_empty[s]));  // V read
+                        ptx::mma_commit(bar(ctrl->v_empty[s]));    // V read by MMA2
                     }
                     has_state = true;
                 }
             }
+            // teardown: every MMA the four issuers issued has completed
+            ptx::mma_commit(bar(ctrl->drain));
+            ptx::mbar_drain(bar(ctrl->drain), 0);
         }
     } else if (warp == sq::kStoreWarp) {
         // ------------------------------------------------------------ O stores
@@ -1327,6 +1335,18 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
         uint32_t g = 0;
         bool ok = true;
+        // Arrive on sbar_ready for block gb once the barrier's phase for block
+        // gb - 2 has completed.  Without that wait a warp two blocks ahead of a
+        // slower one could complete the phase of block gb - 2 in its place: the
+        // issuers order each MMA4 only after the dS read two blocks back, which
+        // comes before that block's S̄ is written.
+        auto sbar_arrive = [&](uint32_t gb) -> bool {
+            if (gb >= 2 && !ptx::mbar_wait(bar(ctrl->sbar_ready[gb & 1]), ((gb - 2) >> 1) & 1, abort_flag))
+                return false;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready[gb & 1]));
+            return true;
+        };
         // the block whose output is still to be drained
         bool o_pending = false;
         Item o_it;
@@ -1371,8 +1391,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
             const Item it = get_item(p, item);
             const int vcol = it.vp * sq::kNV + c0;  // first owned column of the 128
             // ---- running state S (row r, columns vcol..vcol+31) and S̄ for block g
-            //      (S̄ buffer (g - 1) & 1, last read by MMA3 of block g - 2, which A
-            //      issued before MMA1 of block g - 1, whose s_full was observed)
+            //      (S̄ buffer g mod 3, last read by MMA3 of block g - 3, drained before)
             float srun[32];
             if (const float* st0 = start_state(p, it)) {
                 const float4* src = reinterpret_cast<const float4*>(st0 + (size_t)r * kHeadDim + vcol);
@@ -1387,14 +1406,13 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 uint32_t f[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
-                store_row32_bf16_sw128(smem + sq::kSbarOff + ((g + 1) & 1) * kHalfBytes, r, c0, f);
+                store_row32_bf16_sw128(smem + sq::kSbarOff + (g % 3) * kHalfBytes, r, c0, f);
                 ptx::fence_proxy_async_smem();
             } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) srun[j] = 0.f;
             }
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready[g & 1]));
+            if (!sbar_arrive(g)) { ok = false; break; }
 
             for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
                 const bool last_block = t + kTileRows >= it.t1;
@@ -1402,22 +1420,25 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 // ---- 1. P = tril(scores) as bf16 pairs, in place in buffer b
                 if (!ptx::mbar_wait(bar(ctrl->s_full[b]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
-                {
-                    const uint32_t scol = tl + sq::kColSP + b * 128 + k0;
-                    uint32_t pk[32];
-                    // keys [k0, k0 + 64) all masked for this warp's rows: above the
-                    // diagonal (causal) or below it (anti-causal)
-                    if (kRev ? (k0 + 63 < sp * 32) : (k0 > sp * 32 + 31)) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) pk[j] = 0u;
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    // keys [kq, kq + 32), packed into columns [k0 + 16 q2, +16): the
+                    // second half's store lands on columns the first half has read
+                    const int kq = k0 + 32 * q2;
+                    const uint32_t scol = tl + sq::kColSP + b * 128 + kq;
+                    uint32_t pk[16];
+                    // all masked for this warp's rows: above the diagonal (causal) or
+                    // below it (anti-causal)
+                    if (kRev ? (kq + 31 < sp * 32) : (kq > sp * 32 + 31)) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) pk[j] = 0u;
                     } else {
-                        uint32_t v[64];
-                        ptx::tmem_ld32(scol, *reinterpret_cast<uint32_t(*)[32]>(v));
-                        ptx::tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                        uint32_t v[32];
+                        ptx::tmem_ld32(scol, v);
                         ptx::tmem_ld_wait();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int key = k0 + 2 * j;
+                        for (int j = 0; j < 16; ++j) {
+                            const int key = kq + 2 * j;
                             const bool keep_a = kRev ? key >= r : key <= r;
                             const bool keep_b = kRev ? key + 1 >= r : key + 1 <= r;
                             const float a = keep_a ? __uint_as_float(v[2 * j]) : 0.0f;
@@ -1425,7 +1446,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                             pk[j] = ptx::pack_bf16x2(a, bb);
                         }
                     }
-                    ptx::tmem_st32(scol, pk);
+                    ptx::tmem_st16(tl + sq::kColSP + b * 128 + k0 + 16 * q2, pk);
                 }
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
@@ -1446,15 +1467,15 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     for (int j = 0; j < 32; ++j) srun[j] += __uint_as_float(d[j]);
                 }
                 if (!last_block) {
-                    // S̄ buffer g & 1 was last read by MMA3 of block g-1; A issued it
-                    // before MMA1(g), so s_full(g), observed above, covers it
+                    // S̄ buffer (g + 1) mod 3, last read by MMA3 of block g - 2.  That MMA
+                    // has completed: C issued P V of block g - 2 only after it, and this
+                    // warp has drained that output.
                     uint32_t f[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
-                    store_row32_bf16_sw128(smem + sq::kSbarOff + (g & 1) * kHalfBytes, r, c0, f);
+                    store_row32_bf16_sw128(smem + sq::kSbarOff + ((g + 1) % 3) * kHalfBytes, r, c0, f);
                     ptx::fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready[(g + 1) & 1]));
+                    if (!sbar_arrive(g + 1)) { ok = false; break; }
                 } else if (p.state_out != nullptr) {
                     float4* dst = reinterpret_cast<float4*>(
                         p.state_out + (size_t)it.sidx * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim + vcol);
@@ -1807,6 +1828,16 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
         uint8_t* ostage = smem + sq64::kOstOff;
         uint32_t g = 0;
         bool ok = true;
+        // Arrive on sbar_ready[x] for tile gt once the barrier's phase for tile
+        // gt - 1 has completed, so that a warp running ahead of a slower one
+        // never completes an earlier phase in its place (the state increments
+        // are issued without waiting for any S̄).
+        auto sbar_arrive = [&](int x, uint32_t gt) -> bool {
+            if (gt >= 1 && !ptx::mbar_wait(bar(ctrl->sbar_ready[x]), (gt - 1) & 1, abort_flag)) return false;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready[x]));
+            return true;
+        };
         bool o_pending = false;
         Item o_it;
         int o_t = 0, o_h = 0;
@@ -1871,8 +1902,7 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
 #pragma unroll
                 for (int j = 0; j < 32; ++j) srun[j] = 0.f;
             }
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready[0]));
+            if (!sbar_arrive(0, g)) { ok = false; break; }
 
             for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
                 const bool last_tile = t + kTileRows >= it.t1;
@@ -1931,8 +1961,8 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                         for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
                         store_row32_bf16_sw128(smem + sq64::kSbarOff + ((2 * g + h + 1) % 3) * kHalfBytes, r, c0, f);
                         ptx::fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready[h ^ 1]));
+                        // block (g, 1) for h = 0, block (g + 1, 0) for h = 1
+                        if (!sbar_arrive(h ^ 1, g + h)) { ok = false; break; }
                     } else if (p.state_out != nullptr) {
                         float4* dst = reinterpret_cast<float4*>(
                             p.state_out + (size_t)it.sidx * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim + vcol);

@@ -125,6 +125,26 @@ def test_bf16_long_context_sampled_heads(flags):
     assert per_head_rel_err(host64(st[0, heads]), s_ref) <= TOL_STATE
 
 
+@pytest.mark.parametrize("blk", [128, 64])
+def test_bf16_many_items_per_cta_sampled_heads(blk):
+    # The split kernels with many multi-tile work items per CTA (three-pass
+    # output pass, 1024-token chunks of B1 H64 N32768: about 28 items per CTA).
+    # Every item starts from a prefix state written into shared memory by eight
+    # epilogue warps while the previous item is still in flight, so a barrier
+    # hand-off that lets one warp's arrival stand in for another's shows up as a
+    # wrong first tile of some chunk.  Three calls, eight sampled heads.
+    B, H, N, d = 1, 64, 32768, 128
+    q, k, v = inputs.qkv((B, H, N, d), dtype=torch.bfloat16, device=DEV, seed=21)
+    heads = [0, H - 1] + sorted(np.random.default_rng(blk).choice(np.arange(1, H - 1), 6, replace=False).tolist())
+    hq, hk, hv = (host64(x[0, heads]) for x in (q, k, v))
+    o_ref, s_ref = oracle.prefill_recurrent(hq, hk, hv)
+    for _ in range(3):
+        o, st = _run(q, k, v, blk, chunk_tokens=1024, flags=la.LA_FLAG_THREE_PASS | la.LA_FLAG_SPLIT_V)
+        assert la.la_prefill_main_kernel() == ("prefill_seq_kernel" if blk == 128 else "prefill_seq64_kernel")
+        assert per_head_rel_err(host64(o[0, heads]), o_ref) <= TOL_O_BF16
+        assert per_head_rel_err(host64(st[0, heads]), s_ref) <= TOL_STATE
+
+
 # ---------------------------------------------------------------- 64-token blocks
 # blk = 64 runs each 128-row tile as two blocks of 64 tokens (M = 64 MMAs):
 # with the value columns split (prefill_seq64_kernel) when every sequence is
