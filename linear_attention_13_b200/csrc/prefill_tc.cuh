@@ -1025,23 +1025,27 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
 //   * the state increment of each block, dS_i = K_i^T V_i, goes to one of two
 //     TMEM buffers; the running state S (fp32) lives in the epilogue's
 //     registers (32 values per thread), which add dS_i and write the bf16 copy
-//     S̄_i for the next block's Q S̄ into one of three shared-memory buffers;
+//     S̄_i for the next block's Q S̄ into one of two shared-memory buffers;
 //   * scores / P and the output accumulator are double-buffered in TMEM.
 // One issuing thread's MMAs complete one after another, about 175 cycles
 // each whatever their shape (B200), while those of different threads
 // overlap, so each product has its own issuing warp: A QK^T (MMA1), B Q S̄
-// (MMA3), C P V (MMA2), D K^T V (MMA4), 8 MMAs per block each.  Block i reads
-// S̄ buffer i mod 3; the state step of block i writes buffer (i + 1) mod 3,
-// last read by Q S̄ of block i - 2, whose output the epilogue has already
-// drained.  TMEM: scores 2 x 128, O 2 x 64, dS 2 x 64 columns.  Shared
-// memory: two stages of Q, K (128 x 128) and V (128 x 64), S̄ 3 x 16 KiB, O
-// staging 16 KiB.
+// (MMA3), C P V (MMA2), D K^T V (MMA4), 8 MMAs per block each.
+// V is last read by P V, the end of the block's dependency chain (QK^T -> P
+// -> P V), so V has three slots of its own while Q and K share two stages:
+// the load of block i + 3's V waits only for P V of block i.  Block i reads
+// S̄ buffer i & 1; the state step of block i writes buffer (i + 1) & 1 once Q
+// S̄ of block i - 1 has completed.  TMEM: scores 2 x 128, O 2 x 64, dS 2 x 64
+// columns.  Shared memory: two stages of Q and K (128 x 128), three V slots
+// (128 x 64), S̄ 2 x 16 KiB, O staging 16 KiB.
 // ============================================================================
 namespace sq {
 constexpr int kNV = 64;
-constexpr int kStageB = 2 * kTileBytes + kHalfBytes;        // 80 KiB
-constexpr int kSbarOff = kStages * kStageB;                 // S̄[3], 16 KiB each
-constexpr int kOstOff = kSbarOff + 3 * kHalfBytes;          // O staging, 16 KiB
+constexpr int kStageB = 2 * kTileBytes;                     // Q, K: 64 KiB
+constexpr int kVSlots = 3;
+constexpr int kVOff = kStages * kStageB;                    // V[3], 16 KiB each
+constexpr int kSbarOff = kVOff + kVSlots * kHalfBytes;      // S̄[2], 16 KiB each
+constexpr int kOstOff = kSbarOff + 2 * kHalfBytes;          // O staging, 16 KiB
 constexpr int kCtrlOff = kOstOff + kHalfBytes;
 constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
 constexpr uint32_t kColSP = 0;      // scores / P: 2 x 128
@@ -1058,9 +1062,9 @@ constexpr int kL2Ahead = 2;                 // tiles prefetched into L2 ahead of
 
 struct Ctrl {
     uint64_t full_qk[kStages];  // Q and K of stage s landed (MMA1 and MMA3 need no V)
-    uint64_t full_v[kStages];   // V of stage s landed (packed tails: foreign rows cleared)
+    uint64_t full_v[kVSlots];   // V of slot v landed (packed tails: foreign rows cleared)
     uint64_t empty[kStages];    // Q and K slots of stage s read (A, B, D)
-    uint64_t v_empty[kStages];  // V slot of stage s read (C, D)
+    uint64_t v_empty[kVSlots];  // V slot v read (C, D)
     uint64_t tail_ld;
     uint64_t s_full[2];     // MMA1 complete (scores buffer b)
     uint64_t p_ready[2];    // P of block parity b written (8 warps)
@@ -1098,9 +1102,11 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(bar(ctrl->full_qk[s]), 1);
-            ptx::mbar_init(bar(ctrl->full_v[s]), 1);
             ptx::mbar_init(bar(ctrl->empty[s]), 3);
-            ptx::mbar_init(bar(ctrl->v_empty[s]), 2);
+        }
+        for (int v = 0; v < sq::kVSlots; ++v) {
+            ptx::mbar_init(bar(ctrl->full_v[v]), 1);
+            ptx::mbar_init(bar(ctrl->v_empty[v]), 2);
         }
         ptx::mbar_init(bar(ctrl->ost_free), 1);
         ptx::mbar_init(bar(ctrl->tail_ld), 1);
@@ -1172,14 +1178,15 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
             for (int j = 1; j < sq::kL2Ahead; ++j) prefetch(it, it.t0, j);
             for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
                 const int s = g & 1;
+                const int vs = g % sq::kVSlots;
                 const uint32_t stage = sbase + s * sq::kStageB;
+                const uint32_t vslot = sbase + sq::kVOff + vs * kHalfBytes;
                 prefetch(it, t, sq::kL2Ahead);
-                // Q and K of block g reuse slots that block g-2's MMA1, MMA3 and MMA4
-                // have finished with; V waits for its MMA2, which comes later.  Q
-                // and K complete on their own barrier, so MMA1 of block g never
-                // waits for the load of V (issued one MMA2 later)
+                // Q and K of block g reuse the stage that block g-2's MMA1, MMA3 and
+                // MMA4 have finished with; V reuses the slot of block g-3, freed by
+                // its MMA2 and MMA4
                 const bool tail = packed && it.t1 - t < kTileRows;
-                const uint32_t fv = tail ? bar(ctrl->tail_ld) : bar(ctrl->full_v[s]);
+                const uint32_t fv = tail ? bar(ctrl->tail_ld) : bar(ctrl->full_v[vs]);
                 int w = 1;
                 if (lane == 0) {
                     if (g >= 2) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
@@ -1189,10 +1196,11 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                         ptx::mbar_arrive_expect_tx(fqk, 2 * kTileBytes);
                         ptx::tma_load_4d(stage, &maps.q, fqk, 0, row, 0, it.z, pol_qk);
                         ptx::tma_load_4d(stage + kTileBytes, &maps.k, fqk, 0, row, 0, it.z, pol_qk);
-                        if (g >= 2) w = ptx::mbar_wait(bar(ctrl->v_empty[s]), ((g >> 1) + 1) & 1, abort_flag);
+                        if (g >= sq::kVSlots)
+                            w = ptx::mbar_wait(bar(ctrl->v_empty[vs]), ((g / sq::kVSlots) + 1) & 1, abort_flag);
                         if (w) {
                             ptx::mbar_arrive_expect_tx(fv, kHalfBytes);
-                            ptx::tma_load_3d(stage + 2 * kTileBytes, &maps.v_half, fv, it.vp * sq::kNV, row, it.z, pol_v);
+                            ptx::tma_load_3d(vslot, &maps.v_half, fv, it.vp * sq::kNV, row, it.z, pol_v);
                         }
                     }
                 }
@@ -1202,18 +1210,18 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     if (lane == 0) w = ptx::mbar_wait(bar(ctrl->tail_ld), n_tail & 1, abort_flag);
                     ++n_tail;
                     if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-                    zero_tail_rows(smem + s * sq::kStageB + 2 * kTileBytes, it.t1 - t, lane, 1);
+                    zero_tail_rows(smem + sq::kVOff + vs * kHalfBytes, it.t1 - t, lane, 1);
                     ptx::fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->full_v[s]));
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->full_v[vs]));
                 }
             }
         }
         if (lane == 0) {
-            for (uint32_t j = (g >= 2 ? g - 2 : 0); ok && j < g; ++j) {
+            for (uint32_t j = (g >= 2 ? g - 2 : 0); ok && j < g; ++j)
                 ok = ptx::mbar_wait(bar(ctrl->empty[j & 1]), (j >> 1) & 1, abort_flag);
-                if (ok) ok = ptx::mbar_wait(bar(ctrl->v_empty[j & 1]), (j >> 1) & 1, abort_flag);
-            }
+            for (uint32_t j = (g >= sq::kVSlots ? g - sq::kVSlots : 0); ok && j < g; ++j)
+                ok = ptx::mbar_wait(bar(ctrl->v_empty[j % sq::kVSlots]), (j / sq::kVSlots) & 1, abort_flag);
         }
     } else if (warp == 1 || warp == sq::kMmaBWarp || warp == sq::kMmaCWarp || warp == sq::kMmaDWarp) {
         // ------------------------------------------------------------ MMA issuers
@@ -1236,11 +1244,15 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     const uint32_t b = g & 1;
                     const uint32_t par = (g >> 1) & 1;           // phase parity of buffer b's barriers
                     const uint32_t prev = ((g >> 1) + 1) & 1;    // ... for block g - 2
+                    const int vs = g % sq::kVSlots;
                     if (role != 2 && !ptx::mbar_wait(bar(ctrl->full_qk[s]), par, abort_flag)) { ok = false; break; }
-                    if (role >= 2 && !ptx::mbar_wait(bar(ctrl->full_v[s]), par, abort_flag)) { ok = false; break; }
+                    if (role >= 2 && !ptx::mbar_wait(bar(ctrl->full_v[vs]), (g / sq::kVSlots) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     const uint32_t sq_ = sbase + s * sq::kStageB;
                     const uint32_t sk = sq_ + kTileBytes;
-                    const uint32_t sv = sq_ + 2 * kTileBytes;
+                    const uint32_t sv = sbase + sq::kVOff + vs * kHalfBytes;
                     const uint32_t o_cols = tmem + sq::kColO + b * sq::kNV;
                     if (role == 0) {
                         // MMA1 into scores buffer b, once MMA2 of block g-2 consumed its P
@@ -1255,13 +1267,13 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                         ptx::mma_commit(bar(ctrl->s_full[b]));
                         ptx::mma_commit(bar(ctrl->empty[s]));
                     } else if (role == 1) {
-                        // MMA3: O = Q S̄_{g-1} (S̄ buffer g mod 3) into O buffer b, once that
+                        // MMA3: O = Q S̄_{g-1} (S̄ buffer g & 1) into O buffer b, once that
                         // S̄ is written and the epilogue has read block g-2's O there
                         if (!ptx::mbar_wait(bar(ctrl->sbar_ready[b]), par, abort_flag)) { ok = false; break; }
                         if (g >= 2 && !ptx::mbar_wait(bar(ctrl->o_free[b]), prev, abort_flag)) { ok = false; break; }
                         ptx::tc_fence_after();
                         if (has_state) {
-                            const uint32_t sb = sSbar + (g % 3) * kHalfBytes;
+                            const uint32_t sb = sSbar + (g & 1) * kHalfBytes;
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk) {
                                 const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
@@ -1281,7 +1293,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                                         ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_kv, kk > 0);
                         ptx::mma_commit(bar(ctrl->ds_full[b]));
                         ptx::mma_commit(bar(ctrl->empty[s]));      // K read
-                        ptx::mma_commit(bar(ctrl->v_empty[s]));    // V read by MMA4
+                        ptx::mma_commit(bar(ctrl->v_empty[vs]));   // V read by MMA4
                     } else {
                         // MMA2: O += P V (P in TMEM buffer b), after MMA3 wrote O
                         if (!ptx::mbar_wait(bar(ctrl->p_ready[b]), par, abort_flag)) { ok = false; break; }
@@ -1294,7 +1306,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                                         (kk > 0 || has_state) ? 1u : 0u);
                         ptx::mma_commit(bar(ctrl->o_full[b]));
                         ptx::mma_commit(bar(ctrl->p_free[b]));
-                        ptx::mma_commit(bar(ctrl->v_empty[s]));    // V read by MMA2
+                        ptx::mma_commit(bar(ctrl->v_empty[vs]));   // V read by MMA2
                     }
                     has_state = true;
                 }
@@ -1391,7 +1403,8 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
             const Item it = get_item(p, item);
             const int vcol = it.vp * sq::kNV + c0;  // first owned column of the 128
             // ---- running state S (row r, columns vcol..vcol+31) and S̄ for block g
-            //      (S̄ buffer g mod 3, last read by MMA3 of block g - 3, drained before)
+            //      (S̄ buffer g & 1, last read by MMA3 of block g - 2, whose output
+            //      this warp has drained)
             float srun[32];
             if (const float* st0 = start_state(p, it)) {
                 const float4* src = reinterpret_cast<const float4*>(st0 + (size_t)r * kHeadDim + vcol);
@@ -1406,7 +1419,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 uint32_t f[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
-                store_row32_bf16_sw128(smem + sq::kSbarOff + (g % 3) * kHalfBytes, r, c0, f);
+                store_row32_bf16_sw128(smem + sq::kSbarOff + (g & 1) * kHalfBytes, r, c0, f);
                 ptx::fence_proxy_async_smem();
             } else {
 #pragma unroll
@@ -1423,27 +1436,36 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
 #pragma unroll
                 for (int q2 = 0; q2 < 2; ++q2) {
                     // keys [kq, kq + 32), packed into columns [k0 + 16 q2, +16): the
-                    // second half's store lands on columns the first half has read
+                    // second half's store lands on columns the first half has read.
+                    // The warp's rows are [32 sp, 32 sp + 32): a chunk wholly on the
+                    // kept side of the diagonal is packed as is, one wholly on the
+                    // other side is zero (not loaded), only kq = 32 sp is masked.
                     const int kq = k0 + 32 * q2;
                     const uint32_t scol = tl + sq::kColSP + b * 128 + kq;
+                    const bool none = kRev ? (kq < sp * 32) : (kq > sp * 32);
+                    const bool all = kRev ? (kq > sp * 32) : (kq < sp * 32);
                     uint32_t pk[16];
-                    // all masked for this warp's rows: above the diagonal (causal) or
-                    // below it (anti-causal)
-                    if (kRev ? (kq + 31 < sp * 32) : (kq > sp * 32 + 31)) {
+                    if (none) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) pk[j] = 0u;
                     } else {
                         uint32_t v[32];
                         ptx::tmem_ld32(scol, v);
                         ptx::tmem_ld_wait();
+                        if (all) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int key = kq + 2 * j;
-                            const bool keep_a = kRev ? key >= r : key <= r;
-                            const bool keep_b = kRev ? key + 1 >= r : key + 1 <= r;
-                            const float a = keep_a ? __uint_as_float(v[2 * j]) : 0.0f;
-                            const float bb = keep_b ? __uint_as_float(v[2 * j + 1]) : 0.0f;
-                            pk[j] = ptx::pack_bf16x2(a, bb);
+                            for (int j = 0; j < 16; ++j)
+                                pk[j] = ptx::pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+                        } else {
+                            // the diagonal chunk: keys kq + i against row kq + lane
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const bool keep_a = kRev ? 2 * j >= lane : 2 * j <= lane;
+                                const bool keep_b = kRev ? 2 * j + 1 >= lane : 2 * j + 1 <= lane;
+                                const float a = keep_a ? __uint_as_float(v[2 * j]) : 0.0f;
+                                const float bb = keep_b ? __uint_as_float(v[2 * j + 1]) : 0.0f;
+                                pk[j] = ptx::pack_bf16x2(a, bb);
+                            }
                         }
                     }
                     ptx::tmem_st16(tl + sq::kColSP + b * 128 + k0 + 16 * q2, pk);
@@ -1467,13 +1489,16 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     for (int j = 0; j < 32; ++j) srun[j] += __uint_as_float(d[j]);
                 }
                 if (!last_block) {
-                    // S̄ buffer (g + 1) mod 3, last read by MMA3 of block g - 2.  That MMA
-                    // has completed: C issued P V of block g - 2 only after it, and this
-                    // warp has drained that output.
+                    // S̄ buffer (g + 1) & 1, last read by MMA3 of block g - 1.  Its phase
+                    // cannot run ahead: MMA3 of block g + 1 needs the S̄ written here.
+                    if (g >= 1 && !ptx::mbar_wait(bar(ctrl->mma3_done[(g + 1) & 1]), ((g - 1) >> 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     uint32_t f[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
-                    store_row32_bf16_sw128(smem + sq::kSbarOff + ((g + 1) % 3) * kHalfBytes, r, c0, f);
+                    store_row32_bf16_sw128(smem + sq::kSbarOff + ((g + 1) & 1) * kHalfBytes, r, c0, f);
                     ptx::fence_proxy_async_smem();
                     if (!sbar_arrive(g + 1)) { ok = false; break; }
                 } else if (p.state_out != nullptr) {
@@ -1924,12 +1949,19 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                             uint32_t v[16];
                             ptx::tmem_ld16x2_16<16>(scol, v);
                             ptx::tmem_ld_wait();
+                            if (c0 + 31 <= 16 * sp) {
+                                // every key at or below every row of the warp
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                const int key = cq + 2 * j;
-                                const float a = (key <= br) ? __uint_as_float(v[2 * j]) : 0.0f;
-                                const float b = (key + 1 <= br) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
-                                pk[j] = ptx::pack_bf16x2(a, b);
+                                for (int j = 0; j < 8; ++j)
+                                    pk[j] = ptx::pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) {
+                                    const int key = cq + 2 * j;
+                                    const float a = (key <= br) ? __uint_as_float(v[2 * j]) : 0.0f;
+                                    const float b = (key + 1 <= br) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
+                                    pk[j] = ptx::pack_bf16x2(a, b);
+                                }
                             }
                         }
                         ptx::tmem_st16x2_8<8>(scol, pk);
