@@ -1052,9 +1052,17 @@ constexpr uint32_t kColSP = 0;      // scores / P: 2 x 128
 constexpr uint32_t kColO = 256;     // output: 2 x 64
 constexpr uint32_t kColDS = 384;    // state increment: 2 x 64
 constexpr uint32_t kTmemCols = 512;
+// Warp w runs on SM sub-partition w % 4 and its epilogue work is on TMEM lanes
+// [32 (w % 4), +32).  Under the causal mask the P conversion of sub-partition
+// i covers i + 1 chunks of 32 keys, and a warp issuing MMAs takes issue slots
+// from the warps beside it, so the issuers sit on the sub-partitions with the
+// least P work: A and C on 0, D on 1 (with the producer), B on 2, and only the
+// store warp on 3.  Warps 2-9 form the epilogue, two per sub-partition.
 constexpr int kEpiWarps = 8;
-constexpr int kStoreWarp = 2 + kEpiWarps;   // TMA stores of the staged O tiles
-constexpr int kMmaBWarp = 3 + kEpiWarps;    // issuer B: Q S̄
+constexpr int kMmaAWarp = 0;                // issuer A: Q K^T
+constexpr int kProducerWarp = 1;            // TMA loads; allocates TMEM
+constexpr int kMmaBWarp = 2 + kEpiWarps;    // issuer B: Q S̄
+constexpr int kStoreWarp = 3 + kEpiWarps;   // TMA stores of the staged O tiles
 constexpr int kMmaCWarp = 4 + kEpiWarps;    // issuer C: P V
 constexpr int kMmaDWarp = 5 + kEpiWarps;    // issuer D: K^T V
 constexpr int kThreads = 32 * (6 + kEpiWarps);
@@ -1154,7 +1162,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         else return t;
     };
 
-    if (warp == 0) {
+    if (warp == sq::kProducerWarp) {
         // ------------------------------------------------------------ producer
         // the other CTA of the head reads the same Q and K: normal L2 priority
         // for them, evict-first for this CTA's own V half
@@ -1223,7 +1231,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
             for (uint32_t j = (g >= sq::kVSlots ? g - sq::kVSlots : 0); ok && j < g; ++j)
                 ok = ptx::mbar_wait(bar(ctrl->v_empty[j % sq::kVSlots]), (j / sq::kVSlots) & 1, abort_flag);
         }
-    } else if (warp == 1 || warp == sq::kMmaBWarp || warp == sq::kMmaCWarp || warp == sq::kMmaDWarp) {
+    } else if (warp == sq::kMmaAWarp || warp == sq::kMmaBWarp || warp == sq::kMmaCWarp || warp == sq::kMmaDWarp) {
         // ------------------------------------------------------------ MMA issuers
         // A: MMA1 scores = Q K^T; B: MMA3 O = Q S̄; C: MMA2 O += P V; D: MMA4
         // dS = K^T V.  Every resource one of them reuses is double-buffered by
@@ -1233,7 +1241,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
             constexpr uint32_t id_qs = ptx::idesc_bf16(128, sq::kNV, false, true);   // Q S̄
             constexpr uint32_t id_kv = ptx::idesc_bf16(128, sq::kNV, true, true);    // K^T V
             constexpr uint32_t id_pv = ptx::idesc_bf16(128, sq::kNV, false, true);   // P V
-            const int role = warp == 1 ? 0 : warp == sq::kMmaBWarp ? 1 : warp == sq::kMmaCWarp ? 2 : 3;
+            const int role = warp == sq::kMmaAWarp ? 0 : warp == sq::kMmaBWarp ? 1 : warp == sq::kMmaCWarp ? 2 : 3;
             uint32_t g = 0;
             bool ok = true;
             for (int item = blockIdx.x; ok && item < n_items; item += stride) {
