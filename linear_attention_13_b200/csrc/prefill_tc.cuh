@@ -1557,17 +1557,18 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
 // Every buffer is indexed by the block's position h in its tile and each of
 // its barriers completes once per tile, so phase parity = tile & 1.
 // TMEM: scores / P 2 x 64, O 2 x 64 (M = 64 layout), dS 2 x 64 columns.
-// Shared memory: two stages of Q, K, V (64 columns), O staging, and three
-// S̄ buffers of 16 KiB: block j reads S̄ buffer j mod 3.  The state step of
-// block j writes buffer (j + 1) mod 3, last read by Q S̄ of block j - 2, whose
-// output the epilogue has already drained, so that step never waits for an
-// MMA.
+// Shared memory: two stages of Q and K, three V slots (64 columns; V is
+// last read by P V, the end of the chain), two S̄ buffers of 16 KiB (block h
+// of a tile reads buffer h; the state step writes the other one once Q S̄ of
+// the previous block has completed) and O staging.
 // ============================================================================
 namespace sq64 {
 constexpr int kNV = 64;
-constexpr int kStageB = 2 * kTileBytes + kHalfBytes;        // 80 KiB
-constexpr int kSbarOff = kStages * kStageB;             // S̄[3]
-constexpr int kOstOff = kSbarOff + 3 * kHalfBytes;
+constexpr int kStageB = 2 * kTileBytes;                     // Q, K: 64 KiB
+constexpr int kVSlots = 3;
+constexpr int kVOff = kStages * kStageB;                    // V[3]
+constexpr int kSbarOff = kVOff + kVSlots * kHalfBytes;      // S̄[2]
+constexpr int kOstOff = kSbarOff + 2 * kHalfBytes;
 constexpr int kCtrlOff = kOstOff + kHalfBytes;
 constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
 constexpr uint32_t kColSP = 0;      // scores / P: 2 x 64
@@ -1590,9 +1591,9 @@ __host__ __device__ constexpr uint32_t p_col(int kk) { return kk < 2 ? kk * 8 : 
 
 struct Ctrl {
     uint64_t full_qk[kStages];  // Q and K of stage s landed
-    uint64_t full_v[kStages];   // V of stage s landed (packed tails: foreign rows cleared)
+    uint64_t full_v[kVSlots];   // V of slot v landed (packed tails: foreign rows cleared)
     uint64_t empty[kStages];    // Q and K slots read: one commit each from A, B and D
-    uint64_t v_empty[kStages];  // V slot read: one commit each from C and D
+    uint64_t v_empty[kVSlots];  // V slot read: one commit each from C and D
     uint64_t tail_ld;
     uint64_t s_full[2];     // MMA1 of block h complete
     uint64_t p_ready[2];    // P of block h written (8 warps)
@@ -1625,9 +1626,11 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(bar(ctrl->full_qk[s]), 1);
-            ptx::mbar_init(bar(ctrl->full_v[s]), 1);
             ptx::mbar_init(bar(ctrl->empty[s]), 3);
-            ptx::mbar_init(bar(ctrl->v_empty[s]), 2);
+        }
+        for (int v = 0; v < sq64::kVSlots; ++v) {
+            ptx::mbar_init(bar(ctrl->full_v[v]), 1);
+            ptx::mbar_init(bar(ctrl->v_empty[v]), 2);
         }
         ptx::mbar_init(bar(ctrl->tail_ld), 1);
         ptx::mbar_init(bar(ctrl->o_staged), sq64::kEpiWarps);
@@ -1688,10 +1691,12 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
             for (int j = 1; j < sq64::kL2Ahead; ++j) prefetch(it, it.t0, j);
             for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
                 const int s = g & 1;
+                const int vs = g % sq64::kVSlots;
                 const uint32_t stage = sbase + s * sq64::kStageB;
+                const uint32_t vslot = sbase + sq64::kVOff + vs * kHalfBytes;
                 prefetch(it, t, sq64::kL2Ahead);
                 const bool tail = packed && it.t1 - t < kTileRows;
-                const uint32_t fv = tail ? bar(ctrl->tail_ld) : bar(ctrl->full_v[s]);
+                const uint32_t fv = tail ? bar(ctrl->tail_ld) : bar(ctrl->full_v[vs]);
                 int w = 1;
                 if (lane == 0) {
                     if (g >= 2) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
@@ -1702,11 +1707,12 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                         ptx::tma_load_4d(stage + kTileBytes, &maps.k, fqk, 0, t, 0, it.z, pol_qk);
                         if (s) { ld_qk1 = fqk; par_qk1 = (g >> 1) & 1; }
                         else   { ld_qk0 = fqk; par_qk0 = (g >> 1) & 1; }
-                        if (g >= 2) w = ptx::mbar_wait(bar(ctrl->v_empty[s]), ((g >> 1) + 1) & 1, abort_flag);
+                        if (g >= sq64::kVSlots)
+                            w = ptx::mbar_wait(bar(ctrl->v_empty[vs]), ((g / sq64::kVSlots) + 1) & 1, abort_flag);
                         if (w) {
                             ptx::mbar_arrive_expect_tx(fv, kHalfBytes);
-                            ptx::tma_load_3d(stage + 2 * kTileBytes, &maps.v_half, fv, it.vp * sq64::kNV, t, it.z, pol_v);
-                            const uint32_t pv = tail ? (n_tail & 1) : ((g >> 1) & 1);
+                            ptx::tma_load_3d(vslot, &maps.v_half, fv, it.vp * sq64::kNV, t, it.z, pol_v);
+                            const uint32_t pv = tail ? (n_tail & 1) : ((g / sq64::kVSlots) & 1);
                             if (s) { ld_v1 = fv; par_v1 = pv; }
                             else   { ld_v0 = fv; par_v0 = pv; }
                         }
@@ -1717,18 +1723,18 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                     if (lane == 0) w = ptx::mbar_wait(bar(ctrl->tail_ld), n_tail & 1, abort_flag);
                     ++n_tail;
                     if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-                    zero_tail_rows(smem + s * sq64::kStageB + 2 * kTileBytes, it.t1 - t, lane, 1);
+                    zero_tail_rows(smem + sq64::kVOff + vs * kHalfBytes, it.t1 - t, lane, 1);
                     ptx::fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->full_v[s]));
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->full_v[vs]));
                 }
             }
         }
         if (lane == 0) {
-            for (uint32_t j = (g >= 2 ? g - 2 : 0); ok && j < g; ++j) {
+            for (uint32_t j = (g >= 2 ? g - 2 : 0); ok && j < g; ++j)
                 ok = ptx::mbar_wait(bar(ctrl->empty[j & 1]), (j >> 1) & 1, abort_flag);
-                if (ok) ok = ptx::mbar_wait(bar(ctrl->v_empty[j & 1]), (j >> 1) & 1, abort_flag);
-            }
+            for (uint32_t j = (g >= sq64::kVSlots ? g - sq64::kVSlots : 0); ok && j < g; ++j)
+                ok = ptx::mbar_wait(bar(ctrl->v_empty[j % sq64::kVSlots]), (j / sq64::kVSlots) & 1, abort_flag);
             if (!ok) {
                 // after an abort: let the loads already issued land (bounded)
                 if (ld_qk0) ptx::mbar_drain(ld_qk0, par_qk0);
@@ -1755,11 +1761,15 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                     const uint32_t tp = g & 1;        // this tile's phase of the block barriers
                     const uint32_t pp = tp ^ 1u;      // the previous tile's
                     if (!ptx::mbar_wait(bar(ctrl->full_qk[s]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
-                    if (role >= 2 && !ptx::mbar_wait(bar(ctrl->full_v[s]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
+                    const int vs = g % sq64::kVSlots;
+                    if (role >= 2 && !ptx::mbar_wait(bar(ctrl->full_v[vs]), (g / sq64::kVSlots) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     ptx::tc_fence_after();
                     const uint32_t sq_ = sbase + s * sq64::kStageB;
                     const uint32_t sk = sq_ + kTileBytes;
-                    const uint32_t sv = sq_ + 2 * kTileBytes;
+                    const uint32_t sv = sbase + sq64::kVOff + vs * kHalfBytes;
                     for (int h = 0; h < 2; ++h) {
                         const uint32_t roff = h * sq64::kRowOff;
                         if (role == 0) {
@@ -1775,13 +1785,13 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                             }
                             ptx::mma_commit(bar(ctrl->s_full[h]));
                         } else if (role == 1) {
-                            // MMA3: O_h = Q_h S̄ (S̄ buffer (2 g + h) mod 3), once that S̄
+                            // MMA3: O_h = Q_h S̄ (S̄ buffer h), once that S̄
                             // is written and block h of the previous tile has been drained
                             if (!ptx::mbar_wait(bar(ctrl->sbar_ready[h]), tp, abort_flag)) { ok = false; break; }
                             if (g >= 1 && !ptx::mbar_wait(bar(ctrl->o_free[h]), pp, abort_flag)) { ok = false; break; }
                             ptx::tc_fence_after();
                             if (has_state) {
-                                const uint32_t sb = sSbar + ((2 * g + h) % 3) * kHalfBytes;
+                                const uint32_t sb = sSbar + h * kHalfBytes;
 #pragma unroll
                                 for (int kk = 0; kk < 8; ++kk) {
                                     const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32 + roff;
@@ -1811,13 +1821,13 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                                             ptx::sdesc_sw128(sv + roff + kk * 2048, kHalfBytes, 1024), id_pv,
                                             (kk > 0 || has_state) ? 1u : 0u);
                             ptx::mma_commit(bar(ctrl->pv_done[h]));
-                            if (h == 1) ptx::mma_commit(bar(ctrl->v_empty[s]));  // V read
+                            if (h == 1) ptx::mma_commit(bar(ctrl->v_empty[vs]));  // V read
                         }
                         has_state = true;
                     }
                     if (!ok) break;
                     if (role != 2) ptx::mma_commit(bar(ctrl->empty[s]));     // Q and K read
-                    if (role == 3) ptx::mma_commit(bar(ctrl->v_empty[s]));   // V read by MMA4
+                    if (role == 3) ptx::mma_commit(bar(ctrl->v_empty[vs]));  // V read by MMA4
                 }
             }
             // teardown: every MMA the three issuers issued has completed
@@ -1913,8 +1923,8 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
             const Item it = get_item(p, item);
             const int vcol = it.vp * sq64::kNV + c0;   // first owned column of the 128
             // ---- running state S (row r, columns vcol..vcol+31) and the S̄ of the
-            //      item's first block 2 g (buffer 2 g mod 3, last read by MMA3 of
-            //      block 2 g - 3, drained before)
+            //      item's first block (buffer 0, last read by MMA3 of block 0 of the
+            //      previous tile, whose output this warp has drained)
             float srun[32];
             if (const float* st0 = start_state(p, it)) {
                 const float4* src = reinterpret_cast<const float4*>(st0 + (size_t)r * kHeadDim + vcol);
@@ -1929,7 +1939,7 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                 uint32_t f[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
-                store_row32_bf16_sw128(smem + sq64::kSbarOff + ((2 * g) % 3) * kHalfBytes, r, c0, f);
+                store_row32_bf16_sw128(smem + sq64::kSbarOff, r, c0, f);
                 ptx::fence_proxy_async_smem();
             } else {
 #pragma unroll
@@ -1993,13 +2003,19 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                         for (int j = 0; j < 32; ++j) srun[j] += __uint_as_float(d[j]);
                     }
                     if (!(last_tile && h == 1)) {
-                        // S̄ for block j + 1 = 2 g + h + 1: buffer (j + 1) mod 3, last read
-                        // by MMA3 of block j - 2.  That MMA has completed: C issued P V of
-                        // block j - 2 only after it, and this warp has drained that output.
+                        // S̄ for the next block: buffer h ^ 1, last read by MMA3 of the
+                        // previous block, block 1 of the previous tile (h = 0) or block 0
+                        // of this one (h = 1).  Its phase cannot run ahead: the next MMA3
+                        // of that block position needs the S̄ written here.
+                        if ((g >= 1 || h == 1) &&
+                            !ptx::mbar_wait(bar(ctrl->mma3_done[h ^ 1]), h == 0 ? (tp ^ 1u) : tp, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
                         uint32_t f[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
-                        store_row32_bf16_sw128(smem + sq64::kSbarOff + ((2 * g + h + 1) % 3) * kHalfBytes, r, c0, f);
+                        store_row32_bf16_sw128(smem + sq64::kSbarOff + (h ^ 1) * kHalfBytes, r, c0, f);
                         ptx::fence_proxy_async_smem();
                         // block (g, 1) for h = 0, block (g + 1, 0) for h = 1
                         if (!sbar_arrive(h ^ 1, g + h)) { ok = false; break; }
