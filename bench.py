@@ -469,8 +469,7 @@ def bench_secondary(args, device, stream, peaks):
     kern64 = la.la_prefill_main_kernel()
     out["prefill_blk64"] = {
         "roofline": line_roofline(kern64, B * H * N * BYTES_PER_TOKEN_HEAD, k_ms, peaks,
-                                  ("prefill_seq64_kernel_b4h16n8192.md" if kern64 == "prefill_seq64_kernel"
-                                   else "prefill_tc_kernel_128_64_b4h16n8192.md")),
+                                  "prefill_seq64_kernel_b4h16n8192.md" if kern64 == "prefill_seq64_kernel" else None),
         "workload": f"prefill bf16 B={B} H={H} N={N} d={D} blk=64",
         "tokens_per_s": round(B * N / (ms / n64 / 1e3), 1), "ms_per_step": round(ms / n64, 5),
         "hbm_frac": round(B * H * N * BYTES_PER_TOKEN_HEAD / (k_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
