@@ -57,16 +57,22 @@ PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "prefill_seq_kernel_b4h16n8192.
 
 def kernel_source_sha256() -> str:
     """Hash of the kernel sources (csrc/*.cuh, which hold every __global__ and
-    __device__ function): identifies the kernel version an ncu capture was
-    taken of.  lightning.cu (host-side validation, dispatch and launches) is
-    not part of it."""
+    __device__ function) without their comments and blank space: identifies
+    the kernel version an ncu capture was taken of, so that an edit of a
+    comment does not invalidate a capture.  lightning.cu (host-side
+    validation, dispatch and launches) is not part of it."""
     import hashlib
+    import re
     csrc = os.path.join(ROOT, "linear_attention_13_b200", "csrc")
     h = hashlib.sha256()
     for name in sorted(os.listdir(csrc)):
         if name.endswith(".cuh"):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                text = f.read()
+            text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+            text = re.sub(r"//[^\n]*", " ", text)
+            text = " ".join(text.split())
+            h.update(name.encode() + b"\0" + text.encode())
     return h.hexdigest()
 
 

@@ -23,11 +23,12 @@
 // or from packed sequences ([H][T][d] split by cu_seqlens, section 4 of the
 // same page: data packing), where a chunk never crosses a sequence end.
 //
-// Three kernels carry the outputs, each a persistent, warp-specialised CTA
+// Four kernels carry the outputs, each a persistent, warp-specialised CTA
 // per SM (roles listed at each kernel): prefill_tc_kernel (whole value rows,
 // single pass with look-back over chunk states, or 64-token blocks),
-// prefill_seq_kernel (value columns split over two CTAs, two MMA issuers)
-// and chunk_state_kernel (the first pass of the three-pass schedule).
+// prefill_seq_kernel and prefill_seq64_kernel (value columns split over two
+// CTAs, one MMA issuer per product, 128- or 64-token blocks) and
+// chunk_state_kernel (the first pass of the three-pass schedule).
 #pragma once
 
 #include <cuda.h>
