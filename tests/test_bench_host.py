@@ -38,18 +38,22 @@ def test_traffic_null_when_summary_missing_or_malformed(tmp_path):
     assert bench.captured_traffic("prefill_seq_kernel", path) is None
 
 
-def test_source_hash_covers_kernel_sources_only(tmp_path, monkeypatch):
-    # a copy of the source tree: host code (lightning.cu) may change without
-    # invalidating a capture, any kernel header may not
+def test_source_hash_covers_kernel_code_only(tmp_path, monkeypatch):
+    # a copy of the source tree: host code (lightning.cu) and comments in the
+    # kernel headers may change without invalidating a capture, kernel code
+    # may not
     src = os.path.join(bench.ROOT, "linear_attention_13_b200", "csrc")
     dst = tmp_path / "linear_attention_13_b200" / "csrc"
     shutil.copytree(src, dst)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     h0 = bench.kernel_source_sha256()
     assert len(h0) == 64
-    (dst / "lightning.cu").write_text((dst / "lightning.cu").read_text() + "\n// host-side edit\n")
+    (dst / "lightning.cu").write_text((dst / "lightning.cu").read_text() + "\nstatic int host_edit = 1;\n")
     assert bench.kernel_source_sha256() == h0
-    (dst / "decode.cuh").write_text((dst / "decode.cuh").read_text() + "\n// kernel edit\n")
+    text = (dst / "decode.cuh").read_text()
+    (dst / "decode.cuh").write_text(text + "\n// a comment\n/* and a\n   block comment */\n")
+    assert bench.kernel_source_sha256() == h0
+    (dst / "decode.cuh").write_text(text + "\nstatic constexpr int kEdit = 1;\n")
     assert bench.kernel_source_sha256() != h0
 
 
