@@ -48,6 +48,7 @@ UNIT = "tokens/s"
 B, H, N, D, BLK = 4, 16, 8192, 128, 128
 BYTES_PER_TOKEN_HEAD = 8 * D                       # q,k,v read + o write, bf16
 FLOPS_PER_TOKEN_HEAD = 4 * BLK * D + 4 * D * D     # dense-tile count (blk 128)
+USEFUL_FLOPS_PER_TOKEN_HEAD = 2 * (BLK + 1) * D + 4 * D * D   # the causal half of the tile
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
@@ -341,6 +342,10 @@ def bench_ours(args, dist):
     tensor = {"tflops": round(step_tflops, 2), "peak_tflops": peaks["bf16_tflops"],
               "frac_of_peak": round(step_tflops / peaks["bf16_tflops"], 4),
               "flops_per_token_head": FLOPS_PER_TOKEN_HEAD,
+              "useful_tflops": round(step_tflops * USEFUL_FLOPS_PER_TOKEN_HEAD / FLOPS_PER_TOKEN_HEAD, 2),
+              "useful_frac_of_peak": round(step_tflops * USEFUL_FLOPS_PER_TOKEN_HEAD / FLOPS_PER_TOKEN_HEAD /
+                                           peaks["bf16_tflops"], 4),
+              "useful_flops_per_token_head": USEFUL_FLOPS_PER_TOKEN_HEAD,
               "step_hbm_frac": round(bytes_step / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
 
     e2e = bench_e2e(args, dist, device, stream, q, k, v)
