@@ -1171,6 +1171,10 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         const uint64_t pol_v = ptx::policy_evict_first();
         uint32_t g = 0, n_tail = 0;
         bool ok = true;
+        // the last loads issued into each stage and V slot (barrier, phase parity),
+        // to let them land after an abort
+        uint32_t ld_qk0 = 0, ld_qk1 = 0, par_qk0 = 0, par_qk1 = 0;
+        uint32_t ld_v0 = 0, ld_v1 = 0, ld_v2 = 0, par_v0 = 0, par_v1 = 0, par_v2 = 0;
         // L2 prefetch of the tile `ahead` tiles after row t of the item (the
         // loads into shared memory then find it there)
         auto prefetch = [&](const Item& it, int t, int ahead) {
@@ -1205,11 +1209,17 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                         ptx::mbar_arrive_expect_tx(fqk, 2 * kTileBytes);
                         ptx::tma_load_4d(stage, &maps.q, fqk, 0, row, 0, it.z, pol_qk);
                         ptx::tma_load_4d(stage + kTileBytes, &maps.k, fqk, 0, row, 0, it.z, pol_qk);
+                        if (s) { ld_qk1 = fqk; par_qk1 = (g >> 1) & 1; }
+                        else   { ld_qk0 = fqk; par_qk0 = (g >> 1) & 1; }
                         if (g >= sq::kVSlots)
                             w = ptx::mbar_wait(bar(ctrl->v_empty[vs]), ((g / sq::kVSlots) + 1) & 1, abort_flag);
                         if (w) {
                             ptx::mbar_arrive_expect_tx(fv, kHalfBytes);
                             ptx::tma_load_3d(vslot, &maps.v_half, fv, it.vp * sq::kNV, row, it.z, pol_v);
+                            const uint32_t pv = tail ? (n_tail & 1) : ((g / sq::kVSlots) & 1);
+                            if (vs == 0)      { ld_v0 = fv; par_v0 = pv; }
+                            else if (vs == 1) { ld_v1 = fv; par_v1 = pv; }
+                            else              { ld_v2 = fv; par_v2 = pv; }
                         }
                     }
                 }
@@ -1231,6 +1241,14 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 ok = ptx::mbar_wait(bar(ctrl->empty[j & 1]), (j >> 1) & 1, abort_flag);
             for (uint32_t j = (g >= sq::kVSlots ? g - sq::kVSlots : 0); ok && j < g; ++j)
                 ok = ptx::mbar_wait(bar(ctrl->v_empty[j % sq::kVSlots]), (j / sq::kVSlots) & 1, abort_flag);
+            if (!ok) {
+                // after an abort: let the loads already issued land (bounded)
+                if (ld_qk0) ptx::mbar_drain(ld_qk0, par_qk0);
+                if (ld_qk1) ptx::mbar_drain(ld_qk1, par_qk1);
+                if (ld_v0) ptx::mbar_drain(ld_v0, par_v0);
+                if (ld_v1) ptx::mbar_drain(ld_v1, par_v1);
+                if (ld_v2) ptx::mbar_drain(ld_v2, par_v2);
+            }
         }
     } else if (warp == sq::kMmaAWarp || warp == sq::kMmaBWarp || warp == sq::kMmaCWarp || warp == sq::kMmaDWarp) {
         // ------------------------------------------------------------ MMA issuers
