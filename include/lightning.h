@@ -362,6 +362,16 @@ int la_debug_skip_lookback_items(int count);
 int la_debug_occupy_sms(int ctas, unsigned long long duration_ns, void* stream);
 
 /*
+ * la_debug_stall_split_load -- the next launch of a split-value-column kernel
+ * (prefill_seq_kernel, prefill_seq64_kernel) leaves the loads of the `tile`-th
+ * tile each CTA processes (counted from 0) unissued: the MMA issuers' bounded
+ * waits for it run out, LA_ERR_TIMEOUT is recorded, and every role leaves after
+ * letting its own loads and MMAs complete.  One launch only; -1 cancels.
+ * Returns LA_OK or LA_ERR_INVALID_ARG.  A test hook; nothing else calls it.
+ */
+int la_debug_stall_split_load(int tile);
+
+/*
  * la_binary_version -- the compute capability the library's kernels were
  * compiled for, as major * 10 + minor (100 for sm_100a), read from the
  * loaded code object on the current device; LA_ERR_CUDA if it cannot be read.

@@ -54,7 +54,7 @@ EXPORTED = ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_decode_step"
             "la_prefill_varlen_ex", "la_decode_step_slots", "la_decode_step_q8",
             "la_state_quantize_q8", "la_state_dequantize_q8", "la_set_wait_limit_ns",
             "la_debug_fail_allocations", "la_binary_version", "la_debug_skip_lookback_items",
-            "la_debug_occupy_sms")
+            "la_debug_occupy_sms", "la_debug_stall_split_load")
 
 LA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -108,6 +108,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la_binary_version.argtypes = []
     lib.la_debug_skip_lookback_items.argtypes = [i]
     lib.la_debug_occupy_sms.argtypes = [i, ctypes.c_ulonglong, vp]
+    lib.la_debug_stall_split_load.argtypes = [i]
     lib.la_prefill_main_kernel.restype = ctypes.c_char_p
     for name in ("la_prefill", "la_prefill_ex", "la_prefill_varlen", "la_prefill_varlen_ex",
                  "la_decode_step",
@@ -117,7 +118,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                  "la_prefill_backward", "la_decode_step_slots", "la_decode_step_q8",
                  "la_state_quantize_q8", "la_state_dequantize_q8", "la_set_wait_limit_ns",
                  "la_debug_fail_allocations", "la_binary_version", "la_debug_skip_lookback_items",
-                 "la_debug_occupy_sms"):
+                 "la_debug_occupy_sms", "la_debug_stall_split_load"):
         getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -247,6 +248,12 @@ def la_debug_fail_allocations(count):
 def la_debug_skip_lookback_items(count):
     """The next look-back launch skips its first ``count`` items (tests)."""
     return load_library().la_debug_skip_lookback_items(count)
+
+
+def la_debug_stall_split_load(tile):
+    """The next split-kernel launch leaves the loads of each CTA's ``tile``-th
+    tile unissued (tests); -1 cancels."""
+    return load_library().la_debug_stall_split_load(tile)
 
 
 def la_debug_occupy_sms(ctas, duration_ns, stream=None):

@@ -284,7 +284,13 @@ int choose_chunk_tokens(int BH, int N, int ctas) {
 // two blocks per tile.
 std::atomic<const char*> g_main_kernel{""};
 
-void launch_main(const tc::TileMaps& m, const tc::Params& p, int grid, cudaStream_t stream) {
+// Tile (counted per CTA, plus one) whose loads the next split-kernel launch
+// leaves unissued (la_debug_stall_split_load: a test hook), or 0.
+std::atomic<int> g_stall_tile{0};
+
+void launch_main(const tc::TileMaps& m, const tc::Params& p0, int grid, cudaStream_t stream) {
+    tc::Params p = p0;
+    if (p.vparts == 2 && !p.fused) p.stall_tile = g_stall_tile.exchange(0);
     if (p.blk == 64 && p.vparts == 2 && !p.fused) {
         g_main_kernel = "prefill_seq64_kernel";
         tc::prefill_seq64_kernel<<<grid, tc::sq64::kThreads, tc::sq64::kSmemBytes, stream>>>(m, p);
@@ -1260,6 +1266,12 @@ int la_set_wait_limit_ns(unsigned long long limit_ns, unsigned long long* previo
 int la_debug_skip_lookback_items(int count) {
     if (count < 0) return LA_ERR_INVALID_ARG;
     g_skip_items.store(count);
+    return LA_OK;
+}
+
+int la_debug_stall_split_load(int tile) {
+    if (tile < -1) return LA_ERR_INVALID_ARG;
+    g_stall_tile.store(tile + 1);
     return LA_OK;
 }
 

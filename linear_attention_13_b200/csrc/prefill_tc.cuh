@@ -145,6 +145,8 @@ struct Params {
                                 // an item's predecessor chunk has always been taken by
                                 // a CTA that is running.  Null: items by static stride
     int ticket_base;            // first item the counter hands out (0)
+    int stall_tile;             // split kernels: 1 + the CTA tile count whose loads the
+                                // producer leaves unissued (a test hook), or 0
 };
 
 // One work item: rows [t0, t1) of slice z, chunk c of its sequence, value
@@ -1200,6 +1202,9 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 // its MMA2 and MMA4
                 const bool tail = packed && it.t1 - t < kTileRows;
                 const uint32_t fv = tail ? bar(ctrl->tail_ld) : bar(ctrl->full_v[vs]);
+                // test hook: this tile's loads stay unissued, so the waits for them
+                // run out and the kernel aborts
+                if (g + 1 == (uint32_t)p.stall_tile) continue;
                 int w = 1;
                 if (lane == 0) {
                     if (g >= 2) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);
@@ -1716,6 +1721,9 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                 prefetch(it, t, sq64::kL2Ahead);
                 const bool tail = packed && it.t1 - t < kTileRows;
                 const uint32_t fv = tail ? bar(ctrl->tail_ld) : bar(ctrl->full_v[vs]);
+                // test hook: this tile's loads stay unissued, so the waits for them
+                // run out and the kernel aborts
+                if (g + 1 == (uint32_t)p.stall_tile) continue;
                 int w = 1;
                 if (lane == 0) {
                     if (g >= 2) w = ptx::mbar_wait(bar(ctrl->empty[s]), ((g >> 1) + 1) & 1, abort_flag);

@@ -169,7 +169,37 @@ def test_lookback_progresses_while_another_kernel_holds_most_sms(flags):
     assert per_head_rel_err(host64(s), s_ref) <= TOL_STATE
 
 
+@pytest.mark.parametrize("blk,kernel", [(128, "prefill_seq_kernel"), (64, "prefill_seq64_kernel")])
+def test_split_kernel_wait_runs_out_with_timeout_and_the_next_call_works(blk, kernel):
+    # The split kernels (value columns over two CTAs, one chunk per head): the
+    # loads of every CTA's fourth tile are left unissued, so the MMA issuers'
+    # bounded waits (5 ms here) run out, LA_ERR_TIMEOUT is recorded, and each
+    # role leaves after letting its own loads and MMAs land -- the next call on
+    # the same context is correct.
+    q, k, v = inputs.qkv((1, 2, 2048, 128), dtype=torch.bfloat16, device=DEV, seed=16)
+    la.prefill(q, k, v, blk=blk, chunk_tokens=2048, flags=la.LA_FLAG_SPLIT_V)
+    torch.cuda.synchronize()
+    assert la.la_get_last_error() == la.LA_OK
+    assert la.la_prefill_main_kernel() == kernel
+    la.la_set_wait_limit_ns(5_000_000)
+    try:
+        assert la.la_debug_stall_split_load(3) == la.LA_OK
+        la.prefill(q, k, v, blk=blk, chunk_tokens=2048, flags=la.LA_FLAG_SPLIT_V)
+        torch.cuda.synchronize()
+        assert la.la_get_last_error() == la.LA_ERR_TIMEOUT
+    finally:
+        la.la_debug_stall_split_load(-1)
+        la.la_set_wait_limit_ns(0)
+    o, s = la.prefill(q, k, v, blk=blk, chunk_tokens=2048, flags=la.LA_FLAG_SPLIT_V)
+    torch.cuda.synchronize()
+    assert la.la_get_last_error() == la.LA_OK
+    o_ref, s_ref = oracle.prefill_recurrent(host64(q), host64(k), host64(v))
+    assert per_head_rel_err(host64(o), o_ref) <= TOL_O_BF16
+    assert per_head_rel_err(host64(s), s_ref) <= TOL_STATE
+
+
 def test_debug_hooks_validate_their_arguments():
+    assert la.la_debug_stall_split_load(-2) == la.LA_ERR_INVALID_ARG
     assert la.la_debug_skip_lookback_items(-1) == la.LA_ERR_INVALID_ARG
     assert la.la_debug_occupy_sms(0, 1000) == la.LA_ERR_INVALID_ARG
     assert la.la_debug_occupy_sms(1, 2_000_000_000) == la.LA_ERR_INVALID_ARG
