@@ -56,18 +56,19 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "prefill_seq_kernel_b4h16n8192.md")
 
 
-def kernel_source_sha256() -> str:
+def kernel_source_sha256(files=None) -> str:
     """Hash of the kernel sources (csrc/*.cuh, which hold every __global__ and
-    __device__ function) without their comments and blank space: identifies
-    the kernel version an ncu capture was taken of, so that an edit of a
-    comment does not invalidate a capture.  lightning.cu (host-side
-    validation, dispatch and launches) is not part of it."""
+    __device__ function; or only the headers named in ``files``) without their
+    comments and blank space: identifies the kernel version an ncu capture was
+    taken of, so that an edit of a comment, or of another kernel's header,
+    does not invalidate a capture.  lightning.cu (host-side validation,
+    dispatch and launches) is not part of it."""
     import hashlib
     import re
     csrc = os.path.join(ROOT, "linear_attention_13_b200", "csrc")
     h = hashlib.sha256()
     for name in sorted(os.listdir(csrc)):
-        if name.endswith(".cuh"):
+        if name.endswith(".cuh") and (files is None or name in files):
             with open(os.path.join(csrc, name), encoding="utf-8") as f:
                 text = f.read()
             text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
@@ -91,7 +92,9 @@ def captured_traffic(kernel: str, path: str = PROFILE_SUMMARY):
         if ":" in line and line.startswith("- "):
             k, v = line[2:].split(":", 1)
             fields[k.strip()] = v.strip().strip("`")
-    if fields.get("source_sha256") != kernel_source_sha256() or fields.get("kernel") != kernel:
+    files = fields.get("source_files")
+    files = set(files.split()) if files else None
+    if fields.get("source_sha256") != kernel_source_sha256(files) or fields.get("kernel") != kernel:
         return None
     try:
         traffic = float(fields["traffic_bytes_per_launch"])

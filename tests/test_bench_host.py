@@ -57,6 +57,27 @@ def test_source_hash_covers_kernel_code_only(tmp_path, monkeypatch):
     assert bench.kernel_source_sha256() != h0
 
 
+def test_summary_source_files_limit_the_hash(tmp_path, monkeypatch):
+    # a summary that names its kernel's headers stays valid when another
+    # kernel's header changes, and not when one of its own does
+    src = os.path.join(bench.ROOT, "linear_attention_13_b200", "csrc")
+    dst = tmp_path / "linear_attention_13_b200" / "csrc"
+    shutil.copytree(src, dst)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    files = {"common.cuh", "decode.cuh", "ptx.cuh"}
+    path = tmp_path / "s.md"
+    path.write_text("- kernel: `decode_step_kernel`\n- traffic_bytes_per_launch: `123`\n"
+                    "- source_files: `common.cuh decode.cuh ptx.cuh`\n"
+                    "- source_sha256: `%s`\n" % bench.kernel_source_sha256(files))
+    assert bench.captured_traffic("decode_step_kernel", str(path)) == 123
+    text = (dst / "prefill_tc.cuh").read_text()
+    (dst / "prefill_tc.cuh").write_text(text + "\nstatic constexpr int kEdit = 1;\n")
+    assert bench.captured_traffic("decode_step_kernel", str(path)) == 123
+    text = (dst / "decode.cuh").read_text()
+    (dst / "decode.cuh").write_text(text + "\nstatic constexpr int kEdit = 1;\n")
+    assert bench.captured_traffic("decode_step_kernel", str(path)) is None
+
+
 def test_committed_summary_names_the_headline_kernel():
     fields = {}
     for line in open(bench.PROFILE_SUMMARY).read().splitlines():
