@@ -1379,17 +1379,15 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
         uint32_t g = 0;
         bool ok = true;
-        // Arrive on sbar_ready for block gb once the barrier's phase for block
-        // gb - 2 has completed.  Without that wait a warp two blocks ahead of a
-        // slower one could complete the phase of block gb - 2 in its place: the
-        // issuers order each MMA4 only after the dS read two blocks back, which
-        // comes before that block's S̄ is written.
-        auto sbar_arrive = [&](uint32_t gb) -> bool {
-            if (gb >= 2 && !ptx::mbar_wait(bar(ctrl->sbar_ready[gb & 1]), ((gb - 2) >> 1) & 1, abort_flag))
-                return false;
+        // Arrive on sbar_ready for block gb.  Eight warps arrive once per block,
+        // so a warp two blocks ahead of a slower one could complete the slower
+        // one's phase in its place.  It cannot get there: a warp reaches the
+        // state step of block g only after MMA4(g), which waits for every warp's
+        // ds_free of block g - 2, and each warp arrives on ds_free only after
+        // its S̄ arrival of that step (below).
+        auto sbar_arrive = [&](uint32_t gb) {
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready[gb & 1]));
-            return true;
         };
         // the block whose output is still to be drained
         bool o_pending = false;
@@ -1457,7 +1455,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
 #pragma unroll
                 for (int j = 0; j < 32; ++j) srun[j] = 0.f;
             }
-            if (!sbar_arrive(g)) { ok = false; break; }
+            sbar_arrive(g);
 
             for (int t = it.t0; t < it.t1; t += kTileRows, ++g) {
                 const bool last_block = t + kTileRows >= it.t1;
@@ -1515,8 +1513,6 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     ptx::tmem_ld32(tl + sq::kColDS + b * sq::kNV + c0, d);
                     ptx::tmem_ld_wait();
                     ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->ds_free[b]));
 #pragma unroll
                     for (int j = 0; j < 32; ++j) srun[j] += __uint_as_float(d[j]);
                 }
@@ -1532,7 +1528,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     for (int j = 0; j < 32; ++j) f[j] = __float_as_uint(srun[j]);
                     store_row32_bf16_sw128(smem + sq::kSbarOff + ((g + 1) & 1) * kHalfBytes, r, c0, f);
                     ptx::fence_proxy_async_smem();
-                    if (!sbar_arrive(g + 1)) { ok = false; break; }
+                    sbar_arrive(g + 1);
                 } else if (p.state_out != nullptr) {
                     float4* dst = reinterpret_cast<float4*>(
                         p.state_out + (size_t)it.sidx * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim + vcol);
@@ -1540,6 +1536,8 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     for (int j = 0; j < 8; ++j)
                         dst[j] = make_float4(srun[4 * j], srun[4 * j + 1], srun[4 * j + 2], srun[4 * j + 3]);
                 }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(ctrl->ds_free[b]));
 
                 // ---- 3. the previous block's output
                 if (o_pending && !drain_o(o_it, o_t, o_g)) { ok = false; break; }
@@ -1898,15 +1896,14 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
         uint8_t* ostage = smem + sq64::kOstOff;
         uint32_t g = 0;
         bool ok = true;
-        // Arrive on sbar_ready[x] for tile gt once the barrier's phase for tile
-        // gt - 1 has completed, so that a warp running ahead of a slower one
-        // never completes an earlier phase in its place (the state increments
-        // are issued without waiting for any S̄).
-        auto sbar_arrive = [&](int x, uint32_t gt) -> bool {
-            if (gt >= 1 && !ptx::mbar_wait(bar(ctrl->sbar_ready[x]), (gt - 1) & 1, abort_flag)) return false;
+        // Arrive on sbar_ready[x] for tile gt.  A warp running ahead of a slower
+        // one cannot complete the slower one's phase: it reaches the next state
+        // step of block position h only after MMA4 of that block, which waits for
+        // every warp's ds_free of the same position a tile earlier, and each warp
+        // arrives on ds_free only after its S̄ arrival of that step.
+        auto sbar_arrive = [&](int x) {
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(bar(ctrl->sbar_ready[x]));
-            return true;
         };
         bool o_pending = false;
         Item o_it;
@@ -1972,7 +1969,7 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
 #pragma unroll
                 for (int j = 0; j < 32; ++j) srun[j] = 0.f;
             }
-            if (!sbar_arrive(0, g)) { ok = false; break; }
+            sbar_arrive(0);
 
             for (int t = it.t0; ok && t < it.t1; t += kTileRows, ++g) {
                 const bool last_tile = t + kTileRows >= it.t1;
@@ -2024,8 +2021,6 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                         ptx::tmem_ld32(tl + sq64::kColDS + h * 64 + c0, d);
                         ptx::tmem_ld_wait();
                         ptx::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(bar(ctrl->ds_free[h]));
 #pragma unroll
                         for (int j = 0; j < 32; ++j) srun[j] += __uint_as_float(d[j]);
                     }
@@ -2045,7 +2040,7 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                         store_row32_bf16_sw128(smem + sq64::kSbarOff + (h ^ 1) * kHalfBytes, r, c0, f);
                         ptx::fence_proxy_async_smem();
                         // block (g, 1) for h = 0, block (g + 1, 0) for h = 1
-                        if (!sbar_arrive(h ^ 1, g + h)) { ok = false; break; }
+                        sbar_arrive(h ^ 1);
                     } else if (p.state_out != nullptr) {
                         float4* dst = reinterpret_cast<float4*>(
                             p.state_out + (size_t)it.sidx * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim + vcol);
@@ -2053,6 +2048,8 @@ prefill_seq64_kernel(const __grid_constant__ TileMaps maps,
                         for (int j = 0; j < 8; ++j)
                             dst[j] = make_float4(srun[4 * j], srun[4 * j + 1], srun[4 * j + 2], srun[4 * j + 3]);
                     }
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(bar(ctrl->ds_free[h]));
 
                     // ---- 3. the previous block's output
                     if (o_pending && !drain_o(o_it, o_t, o_g, o_h)) { ok = false; break; }
