@@ -1025,11 +1025,14 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
 // One work item is a whole sequence (or a chunk of the three-pass schedule)
 // for one half of the value columns.  The block loop is pipelined so that the
 // tensor cores never wait for the epilogue:
-//   * the state increment of each block, dS_i = K_i^T V_i, goes to one of two
-//     TMEM buffers; the running state S (fp32) lives in the epilogue's
-//     registers (32 values per thread), which add dS_i and write the bf16 copy
-//     S̄_i for the next block's Q S̄ into one of two shared-memory buffers;
-//   * scores / P and the output accumulator are double-buffered in TMEM.
+//   * the state increment of each block, dS_i = K_i^T V_i, goes to one TMEM
+//     buffer; the running state S (fp32) lives in the epilogue's registers (32
+//     values per thread), which add dS_i and write the bf16 copy S̄_i for the
+//     next block's Q S̄ into one of two shared-memory buffers;
+//   * scores / P are double-buffered in TMEM and the output accumulator is
+//     triple-buffered, so that Q S̄ of block i (the first product into O) waits
+//     for the epilogue to have read the output of block i - 3, not i - 2: the
+//     epilogue drains a block's output last in its turn of the next block.
 // One issuing thread's MMAs complete one after another, about 175 cycles
 // each whatever their shape (B200), while those of different threads
 // overlap, so each product has its own issuing warp: A QK^T (MMA1), B Q S̄
@@ -1038,7 +1041,7 @@ prefill_tc_kernel(const __grid_constant__ TileMaps maps,
 // -> P V), so V has three slots of its own while Q and K share two stages:
 // the load of block i + 3's V waits only for P V of block i.  Block i reads
 // S̄ buffer i & 1; the state step of block i writes buffer (i + 1) & 1 once Q
-// S̄ of block i - 1 has completed.  TMEM: scores 2 x 128, O 2 x 64, dS 2 x 64
+// S̄ of block i - 1 has completed.  TMEM: scores 2 x 128, O 3 x 64, dS 64
 // columns.  Shared memory: two stages of Q and K (128 x 128), three V slots
 // (128 x 64), S̄ 2 x 16 KiB, O staging 16 KiB.
 // ============================================================================
@@ -1052,8 +1055,9 @@ constexpr int kOstOff = kSbarOff + 2 * kHalfBytes;          // O staging, 16 KiB
 constexpr int kCtrlOff = kOstOff + kHalfBytes;
 constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
 constexpr uint32_t kColSP = 0;      // scores / P: 2 x 128
-constexpr uint32_t kColO = 256;     // output: 2 x 64
-constexpr uint32_t kColDS = 384;    // state increment: 2 x 64
+constexpr int kOBufs = 3;           // O accumulators: block g uses g % 3
+constexpr uint32_t kColO = 256;     // output: 3 x 64
+constexpr uint32_t kColDS = 448;    // state increment: 1 x 64
 constexpr uint32_t kTmemCols = 512;
 // Warp w runs on SM sub-partition w % 4 and its epilogue work is on TMEM lanes
 // [32 (w % 4), +32).  Under the causal mask the P conversion of sub-partition
@@ -1079,13 +1083,13 @@ struct Ctrl {
     uint64_t tail_ld;
     uint64_t s_full[2];     // MMA1 complete (scores buffer b)
     uint64_t p_ready[2];    // P of block parity b written (8 warps)
-    uint64_t ds_full[2];    // MMA4 complete (dS buffer b)
+    uint64_t ds_full;       // MMA4 complete (the dS buffer)
     uint64_t p_free[2];     // MMA2 complete: P buffer b consumed
     uint64_t mma3_done[2];  // MMA3 (or, without a state, MMA1) of the block using buffer b
-    uint64_t ds_free[2];    // dS buffer read (8 warps)
+    uint64_t ds_free;       // dS buffer read (8 warps)
     uint64_t sbar_ready[2]; // S̄ read by the block of parity b written (8 warps)
-    uint64_t o_full[2];     // MMA2 of block parity b complete
-    uint64_t o_free[2];     // O buffer read (8 warps)
+    uint64_t o_full[kOBufs]; // MMA2 of a block using O buffer g % 3 complete
+    uint64_t o_free[kOBufs]; // O buffer read (8 warps)
     uint64_t o_staged;      // O staged in shared memory (8 warps)
     uint64_t ost_free;      // the O staging buffer has been read by its TMA store
     uint64_t drain;         // teardown: every MMA of the four issuers complete
@@ -1125,16 +1129,18 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(bar(ctrl->p_ready[b]), sq::kEpiWarps);
             ptx::mbar_init(bar(ctrl->sbar_ready[b]), sq::kEpiWarps);
-            ptx::mbar_init(bar(ctrl->o_full[b]), 1);
+        }
+        for (int ob = 0; ob < sq::kOBufs; ++ob) {
+            ptx::mbar_init(bar(ctrl->o_full[ob]), 1);
+            ptx::mbar_init(bar(ctrl->o_free[ob]), sq::kEpiWarps);
         }
         ptx::mbar_init(bar(ctrl->o_staged), sq::kEpiWarps);
+        ptx::mbar_init(bar(ctrl->ds_full), 1);
+        ptx::mbar_init(bar(ctrl->ds_free), sq::kEpiWarps);
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(bar(ctrl->s_full[b]), 1);
-            ptx::mbar_init(bar(ctrl->ds_full[b]), 1);
             ptx::mbar_init(bar(ctrl->p_free[b]), 1);
             ptx::mbar_init(bar(ctrl->mma3_done[b]), 1);
-            ptx::mbar_init(bar(ctrl->ds_free[b]), sq::kEpiWarps);
-            ptx::mbar_init(bar(ctrl->o_free[b]), sq::kEpiWarps);
         }
         ctrl->abort = 0;
         ptx::fence_mbar_init();
@@ -1258,8 +1264,9 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
     } else if (warp == sq::kMmaAWarp || warp == sq::kMmaBWarp || warp == sq::kMmaCWarp || warp == sq::kMmaDWarp) {
         // ------------------------------------------------------------ MMA issuers
         // A: MMA1 scores = Q K^T; B: MMA3 O = Q S̄; C: MMA2 O += P V; D: MMA4
-        // dS = K^T V.  Every resource one of them reuses is double-buffered by
-        // block parity b and guarded by a barrier of that buffer.
+        // dS = K^T V.  Every resource one of them reuses is buffered (scores / P
+        // and S̄ by block parity b, O by g % 3, dS once) and guarded by a
+        // barrier of that buffer.
         if (lane == 0) {
             constexpr uint32_t id_qk = ptx::idesc_bf16(128, 128, false, false);  // Q K^T
             constexpr uint32_t id_qs = ptx::idesc_bf16(128, sq::kNV, false, true);   // Q S̄
@@ -1285,7 +1292,8 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                     const uint32_t sq_ = sbase + s * sq::kStageB;
                     const uint32_t sk = sq_ + kTileBytes;
                     const uint32_t sv = sbase + sq::kVOff + vs * kHalfBytes;
-                    const uint32_t o_cols = tmem + sq::kColO + b * sq::kNV;
+                    const uint32_t ob = g % sq::kOBufs;
+                    const uint32_t o_cols = tmem + sq::kColO + ob * sq::kNV;
                     if (role == 0) {
                         // MMA1 into scores buffer b, once MMA2 of block g-2 consumed its P
                         if (g >= 2 && !ptx::mbar_wait(bar(ctrl->p_free[b]), prev, abort_flag)) { ok = false; break; }
@@ -1299,10 +1307,14 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                         ptx::mma_commit(bar(ctrl->s_full[b]));
                         ptx::mma_commit(bar(ctrl->empty[s]));
                     } else if (role == 1) {
-                        // MMA3: O = Q S̄_{g-1} (S̄ buffer g & 1) into O buffer b, once that
-                        // S̄ is written and the epilogue has read block g-2's O there
+                        // MMA3: O = Q S̄_{g-1} (S̄ buffer g & 1) into O buffer g % 3, once
+                        // that S̄ is written and the epilogue has read block g-3's O there
                         if (!ptx::mbar_wait(bar(ctrl->sbar_ready[b]), par, abort_flag)) { ok = false; break; }
-                        if (g >= 2 && !ptx::mbar_wait(bar(ctrl->o_free[b]), prev, abort_flag)) { ok = false; break; }
+                        if (g >= sq::kOBufs &&
+                            !ptx::mbar_wait(bar(ctrl->o_free[ob]), ((g / sq::kOBufs) + 1) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
                         ptx::tc_fence_after();
                         if (has_state) {
                             const uint32_t sb = sSbar + (g & 1) * kHalfBytes;
@@ -1316,14 +1328,14 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                         ptx::mma_commit(bar(ctrl->mma3_done[b]));
                         ptx::mma_commit(bar(ctrl->empty[s]));
                     } else if (role == 3) {
-                        // MMA4: dS = K^T V into dS buffer b, once block g-2's dS was read
-                        if (g >= 2 && !ptx::mbar_wait(bar(ctrl->ds_free[b]), prev, abort_flag)) { ok = false; break; }
+                        // MMA4: dS = K^T V, once the state step has read block g-1's dS
+                        if (g >= 1 && !ptx::mbar_wait(bar(ctrl->ds_free), (g - 1) & 1, abort_flag)) { ok = false; break; }
                         ptx::tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            ptx::mma_ss(tmem + sq::kColDS + b * sq::kNV, ptx::sdesc_sw128(sk + kk * 2048, kHalfBytes, 1024),
+                            ptx::mma_ss(tmem + sq::kColDS, ptx::sdesc_sw128(sk + kk * 2048, kHalfBytes, 1024),
                                         ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_kv, kk > 0);
-                        ptx::mma_commit(bar(ctrl->ds_full[b]));
+                        ptx::mma_commit(bar(ctrl->ds_full));
                         ptx::mma_commit(bar(ctrl->empty[s]));      // K read
                         ptx::mma_commit(bar(ctrl->v_empty[vs]));   // V read by MMA4
                     } else {
@@ -1336,7 +1348,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                             ptx::mma_ts(o_cols, tmem + sq::kColSP + b * 128 + p_col(kk) - kColS,
                                         ptx::sdesc_sw128(sv + kk * 2048, kHalfBytes, 1024), id_pv,
                                         (kk > 0 || has_state) ? 1u : 0u);
-                        ptx::mma_commit(bar(ctrl->o_full[b]));
+                        ptx::mma_commit(bar(ctrl->o_full[ob]));
                         ptx::mma_commit(bar(ctrl->p_free[b]));
                         ptx::mma_commit(bar(ctrl->v_empty[vs]));   // V read by MMA2
                     }
@@ -1383,7 +1395,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         // so a warp two blocks ahead of a slower one could complete the slower
         // one's phase in its place.  It cannot get there: a warp reaches the
         // state step of block g only after MMA4(g), which waits for every warp's
-        // ds_free of block g - 2, and each warp arrives on ds_free only after
+        // ds_free of block g - 1, and each warp arrives on ds_free only after
         // its S̄ arrival of that step (below).
         auto sbar_arrive = [&](uint32_t gb) {
             __syncwarp();
@@ -1397,8 +1409,8 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
         // ---- O of block og: registers, release its buffer, stage as bf16 for
         //      the store warp once it has stored the previous tile
         auto drain_o = [&](const Item& oit, int ot, uint32_t og) -> bool {
-            const uint32_t ob = og & 1;
-            if (!ptx::mbar_wait(bar(ctrl->o_full[ob]), (og >> 1) & 1, abort_flag)) return false;
+            const uint32_t ob = og % sq::kOBufs;
+            if (!ptx::mbar_wait(bar(ctrl->o_full[ob]), (og / sq::kOBufs) & 1, abort_flag)) return false;
             ptx::tc_fence_after();
             const bool rowwise = packed && ot + kTileRows > oit.t1;
             uint8_t* ostage = smem + sq::kOstOff;
@@ -1506,11 +1518,11 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                 if (lane == 0) ptx::mbar_arrive(bar(ctrl->p_ready[b]));
 
                 // ---- 2. S += dS_g; S̄_g for the next block, or the final state
-                if (!ptx::mbar_wait(bar(ctrl->ds_full[b]), (g >> 1) & 1, abort_flag)) { ok = false; break; }
+                if (!ptx::mbar_wait(bar(ctrl->ds_full), g & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
                 {
                     uint32_t d[32];
-                    ptx::tmem_ld32(tl + sq::kColDS + b * sq::kNV + c0, d);
+                    ptx::tmem_ld32(tl + sq::kColDS + c0, d);
                     ptx::tmem_ld_wait();
                     ptx::tc_fence_before();
 #pragma unroll
@@ -1537,7 +1549,7 @@ prefill_seq_kernel(const __grid_constant__ TileMaps maps,
                         dst[j] = make_float4(srun[4 * j], srun[4 * j + 1], srun[4 * j + 2], srun[4 * j + 3]);
                 }
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(ctrl->ds_free[b]));
+                if (lane == 0) ptx::mbar_arrive(bar(ctrl->ds_free));
 
                 // ---- 3. the previous block's output
                 if (o_pending && !drain_o(o_it, o_t, o_g)) { ok = false; break; }
